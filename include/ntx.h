@@ -1,0 +1,249 @@
+/*
+ * ntx.h -- C ABI of libntx: batch-1 Llama decode over GGUF block-quantized
+ * weights on NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute follows the statement of the method in three pages:
+ *   [README]  "NTransformer" -- 主な成果 (key results), 主な機能 (features),
+ *             アーキテクチャ概要 (architecture overview), NVMeダイレクトストリーミング.
+ *   [ShowHN]  "Show HN: NVMe経由でCPUをバイパスして単一のRTX 3090上で動作するLlama 3.1 70B"
+ *             -- 量子化フォーマット対応表 (format table), 3層アダプティブキャッシュ詳細 (3-tier cache).
+ *   [Article] "RTX 3090 1枚でLlama 70B — NVMe-to-GPU直結でCPUバイパスする革新技術"
+ *             -- SLEP ストリーミングパイプライン, レイヤースキップ機構 (layer skip).
+ *
+ * Conventions (all calls):
+ *  - Pointers are caller-owned.  "device" pointers address CUDA device memory
+ *    of the current device; "host" pointers are ordinary or pinned host memory
+ *    as stated.  The library never frees caller memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls only enqueue work on it and return; results are ready when the
+ *    stream has reached them.  No call synchronises unless documented.
+ *  - Every call returns an int status: NTX_OK (0) or a negative NTX_ERR_*.
+ *    A failed argument check enqueues nothing.  ntx_last_error() returns a
+ *    thread-local description of the most recent failure on the calling thread.
+ *  - No exception crosses the ABI; kernels never trap.  A kernel that gives up
+ *    waiting (bounded waits only) records a code in a device status word that
+ *    ntx_device_status() reads.
+ *  - Floating-point activations are fp32; the KV cache is IEEE fp16 stored as
+ *    uint16_t bit patterns; quantized weights are raw GGUF block bytes.
+ */
+#ifndef NTX_H
+#define NTX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NTX_API __attribute__((visibility("default")))
+#else
+#define NTX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status */
+#define NTX_OK 0
+#define NTX_ERR_INVALID_ARG (-1) /* null pointer, negative size, bad flag        */
+#define NTX_ERR_SHAPE (-2)       /* size not a multiple of the block, over limit */
+#define NTX_ERR_QTYPE (-3)       /* unsupported weight type                      */
+#define NTX_ERR_ALIGN (-4)       /* pointer misaligned for the call              */
+#define NTX_ERR_CUDA (-5)        /* CUDA launch / runtime error                  */
+#define NTX_ERR_TIMEOUT (-6)     /* a bounded wait ran out                       */
+#define NTX_ERR_NOMEM (-7)       /* host allocation or workspace too small       */
+
+/* ------------------------------------------------------------ weight types
+ * GGUF type ids.  Block layouts ([ShowHN] 量子化フォーマット対応表 gives the
+ * bits per weight and block lengths; the byte layout is GGUF's):
+ *   Q8_0: 34 B per 32 weights  = fp16 d | int8 q[32];            w = d q
+ *   Q4_0: 18 B per 32 weights  = fp16 d | 16 B, byte j = q_j | q_(j+16) << 4;
+ *                                                                 w = d (q - 8)
+ *   Q6_K: 210 B per 256 weights = ql[128] | qh[64] | int8 sc[16] | fp16 d;
+ *         element n (h = n/128, g = (n%128)/32, l = n%32): low 4 bits in
+ *         ql[64h + 32(g%2) + l] (low nibble if g < 2, else high), high 2 bits
+ *         at bit 2g of qh[32h + l];                               w = d sc[n/16] (q - 32)
+ * Weight matrices are row-major (out x in) with each row a run of K/block
+ * blocks. */
+#define NTX_F32 0
+#define NTX_F16 1
+#define NTX_Q4_0 2
+#define NTX_Q8_0 8
+#define NTX_Q6_K 14
+
+NTX_API const char* ntx_last_error(void);
+NTX_API int ntx_version(void); /* major*10000 + minor*100 + patch */
+
+/* Reads and clears the device status word of the current device (0 = no
+ * kernel gave up a bounded wait since the last read).  Synchronises the
+ * device.  Returns NTX_OK and stores the word in *code. */
+NTX_API int ntx_device_status(int* code);
+
+/* Number of SMs the kernels size their grids for on the current device. */
+NTX_API int ntx_sm_count(void);
+
+/* Tuning: persistent GEMV CTAs per SM (1..4, default 1) for launches made
+ * after the call, process-wide.  Workspace sizes do not depend on it. */
+NTX_API int ntx_set_gemv_ctas_per_sm(int ctas_per_sm);
+
+/* ------------------------------------------------------------ per-op calls */
+
+/* Dequantize n weights ([README] 主な機能: GGUF Q4_0/Q8_0/Q6_K; [ShowHN]
+ * 量子化フォーマット対応表).  blocks: device, n/block_elems consecutive blocks,
+ * 2-byte aligned.  out: device fp32[n].  Exact: every value d*sc*(q-off) is
+ * representable in fp32.  NTX_ERR_SHAPE if n is not a multiple of the block
+ * length; NTX_ERR_QTYPE for other types. */
+NTX_API int ntx_dequant(int qtype, const void* blocks, float* out, int64_t n, void* stream);
+
+/* Quantized GEMV y = W_deq x (+ residual) with fp32 accumulation ([README]
+ * アーキテクチャ概要: the GEMV kernel; decode cost is weight bytes over
+ * memory bandwidth, [Article] VRAMの壁).
+ *   W: device, M rows of K/block_elems blocks (row-major), 16-byte aligned.
+ *   x: device fp32[K].  y: device fp32[M], must not overlap x.
+ *   residual: device fp32[M] or NULL; may be y itself (y = W x + y).
+ * Limits: 1 <= M <= 2^31-1, block_elems | K, K <= 262144.  Shapes with
+ * K % 256 == 0 (Q8_0, Q4_0) or K % 2048 == 0 (Q6_K) take the bulk-copy
+ * pipeline; other K take a slower generic kernel with the same results.
+ * Errors: NTX_ERR_QTYPE, NTX_ERR_SHAPE, NTX_ERR_ALIGN (W, x, y or residual
+ * not 16-B aligned), NTX_ERR_INVALID_ARG (NULL, y overlapping x, residual
+ * partially overlapping y). */
+NTX_API int ntx_gemv_q(int qtype, const void* W, int64_t M, int64_t K, const float* x, float* y, const float* residual,
+               void* stream);
+
+/* RMSNorm y_i = w_i x_i / sqrt(mean_j x_j^2 + eps) ([README] 主な機能:
+ * RMSNorm).  x, w, y: device fp32[n]; y may alias x.  1 <= n <= 2^20. */
+NTX_API int ntx_rmsnorm(const float* x, const float* w, float* y, int64_t n, float eps, void* stream);
+
+/* Rotary position embedding in place ([README] 主な機能: RoPE): for every
+ * head of q (n_q_heads x head_dim fp32) and of k (n_kv_heads x head_dim, may
+ * be NULL when n_kv_heads == 0) the adjacent pair (2i, 2i+1) turns by the
+ * angle pos * theta^(-2i/head_dim).  head_dim even, <= 256; pos >= 0.
+ * Angles are formed in fp64, the rotation in fp32. */
+NTX_API int ntx_rope(float* q, float* k, int n_q_heads, int n_kv_heads, int head_dim, int pos, float theta, void* stream);
+
+/* Grouped-query decode attention over an fp16 KV cache ([README] 主な機能:
+ * GQA, KV cache; アーキテクチャ概要: softmax).  For query head h (reading KV
+ * head h / (n_q_heads/n_kv_heads)):  out_h = sum_{p < n_ctx} softmax_p(q_h.k_p
+ * / sqrt(head_dim)) v_p, split over positions and merged with a log-sum-exp
+ * combine.
+ *   q: device fp32[n_q_heads * head_dim].  out: device fp32, same size.
+ *   k_cache, v_cache: device fp16 bits, [n_kv_heads][max_ctx][head_dim],
+ *     16-byte aligned; positions 0..n_ctx-1 are read (n_ctx counts the current
+ *     token, whose k, v the caller has already stored).
+ *   workspace: device, >= ntx_attn_workspace_bytes(...) bytes, 16-B aligned;
+ *     scratch only, contents on entry ignored.
+ * Limits: head_dim == 128, n_kv_heads | n_q_heads, group n_q_heads/n_kv_heads
+ * in {1, 2, 4, 8}, 1 <= n_ctx <= max_ctx. */
+NTX_API size_t ntx_attn_workspace_bytes(int n_q_heads, int n_kv_heads, int head_dim, int max_ctx);
+NTX_API int ntx_attn_decode(const float* q, const uint16_t* k_cache, const uint16_t* v_cache, float* out, int n_q_heads,
+                    int n_kv_heads, int head_dim, int n_ctx, int max_ctx, void* workspace, size_t ws_bytes,
+                    void* stream);
+
+/* SwiGLU out_i = silu(gate_i) up_i, silu(z) = z / (1 + e^-z) ([README]
+ * 主な機能: SwiGLU).  Device fp32[n] each; out may alias either input. */
+NTX_API int ntx_swiglu(const float* gate, const float* up, float* out, int64_t n, void* stream);
+
+/* ------------------------------------------------------------ layer / model */
+typedef struct {
+  int32_t hidden;     /* H */
+  int32_t n_heads;    /* Hq */
+  int32_t n_kv_heads; /* Hkv */
+  int32_t head_dim;   /* D (128) */
+  int32_t ffn;        /* F */
+  int32_t vocab;      /* V */
+  int32_t n_layers;   /* L */
+  float eps;          /* RMSNorm epsilon */
+  float theta;        /* RoPE base */
+  int32_t max_ctx;    /* KV cache capacity in positions */
+  float skip_threshold; /* cosine layer-skip threshold tau */
+} ntx_model_config;
+
+/* One layer's weights inside one contiguous blob at `base` (device memory or
+ * a device slot the layer was streamed into).  Offsets are in bytes from base
+ * and 256-B aligned: wq (Hq*D x H), wk, wv (Hkv*D x H), wo (H x Hq*D),
+ * wg, wu (F x H), wd (H x F) as quantized blocks of `qtype`; attn_norm and
+ * ffn_norm as fp32[H].  The same layout serves resident and pinned-host
+ * copies, so streaming a layer is one contiguous copy. */
+typedef struct {
+  int32_t qtype;
+  const void* base;
+  uint64_t off_wq, off_wk, off_wv, off_wo, off_wg, off_wu, off_wd, off_attn_norm, off_ffn_norm;
+} ntx_layer_weights;
+
+/* Fills the canonical offsets of a layer blob for cfg and qtype (base left
+ * NULL) and returns the blob size in bytes, 0 on bad arguments. */
+NTX_API uint64_t ntx_layer_layout(const ntx_model_config* cfg, int qtype, ntx_layer_weights* out);
+
+/* Workspace one ntx_decode_layer call needs (device bytes). */
+NTX_API size_t ntx_layer_workspace_bytes(const ntx_model_config* cfg);
+
+/* One pre-norm Llama decode layer for one token at position pos ([README]
+ * 主な機能: Llama architecture RoPE, GQA, SwiGLU, RMSNorm, KV cache;
+ * [Article] レイヤースキップ機構 for the cosine):
+ *   n1 = RMSNorm(h) w_attn; q,k,v = Wq n1, Wk n1, Wv n1; RoPE(q), RoPE(k);
+ *   k, v -> fp16 cache row pos; a = GQA attention over rows 0..pos;
+ *   h1 = h + Wo a; n2 = RMSNorm(h1) w_ffn; h = h1 + Wd (silu(Wg n2) (Wu n2)).
+ *   hidden: device fp32[H], read and overwritten with the layer output.
+ *   k_cache, v_cache: device fp16 bits [Hkv][max_ctx][D] of this layer.
+ *   cos_out: device float or NULL; receives cos(h_in, h_out).
+ *   workspace: device scratch >= ntx_layer_workspace_bytes(cfg), 256-B aligned.
+ * Limits: head_dim 128; query group in {1, 2, 4, 8}; H, F and Hq*D
+ * multiples of 256 (Q8_0, Q4_0) or 2048 (Q6_K); 0 <= pos < max_ctx; weight
+ * offsets 16-B aligned.  hidden, base and the caches 16-B aligned. */
+NTX_API int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_weights* w, uint16_t* k_cache, uint16_t* v_cache,
+                     float* hidden, int pos, float* cos_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Decode engine: the per-token forward over all layers ([README] 3-Tier
+ * adaptive cache, 4 data paths 1-2; [ShowHN] 3層アダプティブキャッシュ詳細:
+ * tier A resident, tier B pinned RAM + H2D into double buffers; [Article]
+ * SLEP ストリーミングパイプライン: copy of the next layer overlapped with the
+ * current layer's compute).
+ *   layers[l].base: device memory (tier_map[l] == 0) or pinned host memory
+ *     (tier_map[l] == 1) holding the layer blob (ntx_layer_layout order).
+ *   slot0, slot1: device buffers of slot_bytes each (>= the largest host
+ *     layer) into which host layers are copied; may be NULL if no layer is
+ *     on the host.
+ *   embed: device fp16 bits [V][H].  final_norm: device fp32[H].
+ *   head: device quantized [V x H] of head_qtype.
+ *   k_caches[l], v_caches[l]: device fp16 bits [Hkv][max_ctx][D].
+ *   workspace: device scratch >= ntx_engine_workspace_bytes(cfg).
+ *   compute_stream / copy_stream: distinct streams; copy_stream may be NULL
+ *     when no layer is on the host.
+ * The engine owns only its events, a pinned 16-byte parameter block and the
+ * captured CUDA graphs; the caller keeps every buffer alive until
+ * ntx_engine_destroy. */
+typedef struct ntx_engine ntx_engine;
+
+#define NTX_CALIBRATE_SKIP 1 /* run every layer, record cosines, fix the skip set {l : cos_l >= tau} */
+#define NTX_USE_SKIP 2       /* skip the layers of the recorded set (not computed, not streamed) */
+#define NTX_NO_GRAPH 4       /* launch kernel by kernel instead of replaying the captured graph */
+
+NTX_API size_t ntx_engine_workspace_bytes(const ntx_model_config* cfg);
+NTX_API int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_weights* layers, const int8_t* tier_map,
+                      void* slot0, void* slot1, size_t slot_bytes, const uint16_t* embed, const float* final_norm,
+                      const void* head, int head_qtype, uint16_t* const* k_caches, uint16_t* const* v_caches,
+                      void* workspace, size_t ws_bytes, void* compute_stream, void* copy_stream,
+                      ntx_engine** out);
+
+/* One decode step for `token` at position `pos` (0 <= pos < max_ctx):
+ * embed -> layers -> final RMSNorm -> head -> greedy argmax (ties -> lowest id).
+ *   token: a token id in [0, V), or -1 to use the engine's previous argmax
+ *     (device-side, no host round trip).
+ *   logits: device fp32[V] or NULL.  next_token: device int32 or NULL.
+ *   cos_out: device fp32[L] or NULL; receives cos(h_in, h_out) of every
+ *     layer computed in this step (skipped layers are left untouched).
+ * With NTX_CALIBRATE_SKIP the call waits for the step to finish (it reads the
+ * cosines back to fix the skip set); otherwise it only enqueues. */
+NTX_API int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* logits, int32_t* next_token, int flags,
+                    float* cos_out);
+
+/* Copies the recorded skip set (1 = skipped) into mask_host[L]; returns the
+ * number of skipped layers, or a negative error. */
+NTX_API int ntx_engine_skip_mask(ntx_engine* e, uint8_t* mask_host);
+
+NTX_API void ntx_engine_destroy(ntx_engine* e);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NTX_H */

@@ -1,0 +1,665 @@
+// api.cu -- the extern "C" boundary of libntx: argument checks, error
+// reporting, the layer blob layout, the single-layer call and the decode
+// engine (resident + pinned-host tiers, double-buffered device slots, cosine
+// layer skip, CUDA-graph replay of the per-token launch sequence).
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "launch.h"
+#include "ntx.h"
+
+namespace {
+
+thread_local std::string t_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(NTX_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int block_elems(int qt) { return qt == NTX_Q6_K ? 256 : ((qt == NTX_Q8_0 || qt == NTX_Q4_0) ? 32 : 0); }
+int block_bytes(int qt) { return qt == NTX_Q6_K ? 210 : (qt == NTX_Q8_0 ? 34 : (qt == NTX_Q4_0 ? 18 : 0)); }
+bool qtype_ok(int qt) { return qt == NTX_Q8_0 || qt == NTX_Q4_0 || qt == NTX_Q6_K; }
+
+int64_t mat_bytes(int qt, int64_t M, int64_t K) { return M * (K / block_elems(qt)) * block_bytes(qt); }
+
+uint64_t align256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+// K constraint of the fused (bulk-copy) GEMV path.
+bool k_ok_fused(int qt, int64_t K) { return qt == NTX_Q6_K ? K % 2048 == 0 : K % 256 == 0; }
+
+int check_config(const ntx_model_config* c, int qtype) {
+  if (!c) return fail(NTX_ERR_INVALID_ARG, "config is NULL");
+  if (!qtype_ok(qtype)) return fail(NTX_ERR_QTYPE, "unsupported weight type %d", qtype);
+  if (c->hidden <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 || c->ffn <= 0 || c->n_layers < 0 || c->max_ctx <= 0)
+    return fail(NTX_ERR_SHAPE, "non-positive dimension in config");
+  if (c->head_dim != 128) return fail(NTX_ERR_SHAPE, "head_dim %d unsupported (128 only)", c->head_dim);
+  if (c->n_heads % c->n_kv_heads) return fail(NTX_ERR_SHAPE, "n_heads %% n_kv_heads != 0");
+  const int G = c->n_heads / c->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(NTX_ERR_SHAPE, "query group %d unsupported (1,2,4,8)", G);
+  const int64_t Q = (int64_t)c->n_heads * c->head_dim;
+  if (!k_ok_fused(qtype, c->hidden) || !k_ok_fused(qtype, c->ffn) || !k_ok_fused(qtype, Q))
+    return fail(NTX_ERR_SHAPE, "hidden/ffn/heads*head_dim must be multiples of %d for type %d",
+                qtype == NTX_Q6_K ? 2048 : 256, qtype);
+  if (!(c->eps >= 0.f) || !(c->theta > 0.f)) return fail(NTX_ERR_INVALID_ARG, "bad eps/theta");
+  return NTX_OK;
+}
+
+// ------------------------------------------------------------ workspace
+struct Carve {
+  uint8_t* base;
+  uint64_t off = 0;
+  template <class T>
+  T* take(uint64_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = align256(off + count * sizeof(T));
+    return p;
+  }
+};
+
+int max_parts() { return ntx::sm_count() * 4; }
+
+struct LayerWs {
+  float *q, *attn_out, *attn_part, *h1, *u, *stats_in, *stats_o, *stats_down, *cos_tmp;
+};
+
+uint64_t carve_layer(const ntx_model_config* c, int n_split, uint8_t* base, LayerWs* w) {
+  Carve k{base};
+  const int64_t Q = (int64_t)c->n_heads * c->head_dim;
+  const int P = max_parts();
+  LayerWs t;
+  t.q = k.take<float>(Q);
+  t.attn_out = k.take<float>(Q);
+  t.attn_part = k.take<float>((uint64_t)c->n_heads * n_split * (c->head_dim + 2));
+  t.h1 = k.take<float>(c->hidden);
+  t.u = k.take<float>(c->ffn);
+  t.stats_in = k.take<float>((uint64_t)P * 4);
+  t.stats_o = k.take<float>((uint64_t)P * 4);
+  t.stats_down = k.take<float>((uint64_t)P * 4);
+  t.cos_tmp = k.take<float>(4);
+  if (w) *w = t;
+  return k.off;
+}
+
+}  // namespace
+
+// ======================================================================
+extern "C" {
+
+const char* ntx_last_error(void) { return t_err.c_str(); }
+
+int ntx_version(void) { return 100; }
+
+int ntx_device_status(int* code) {
+  if (!code) return fail(NTX_ERR_INVALID_ARG, "code is NULL");
+  const int e = ntx::read_device_status(code);
+  if (e) return cuda_fail((cudaError_t)e, "ntx_device_status");
+  return NTX_OK;
+}
+
+int ntx_sm_count(void) { return ntx::sm_count(); }
+
+int ntx_dequant(int qtype, const void* blocks, float* out, int64_t n, void* stream) {
+  if (!qtype_ok(qtype)) return fail(NTX_ERR_QTYPE, "unsupported weight type %d", qtype);
+  if (n < 0 || n % block_elems(qtype)) return fail(NTX_ERR_SHAPE, "n=%lld not a multiple of %d", (long long)n,
+                                                   block_elems(qtype));
+  if (n == 0) return NTX_OK;
+  if (!blocks || !out) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(out, 4)) return fail(NTX_ERR_ALIGN, "out not 4-byte aligned");
+  const cudaError_t e = ntx::launch_dequant(qtype, blocks, out, n / block_elems(qtype), S(stream));
+  return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_dequant");
+}
+
+int ntx_gemv_q(int qtype, const void* W, int64_t M, int64_t K, const float* x, float* y, const float* residual,
+               void* stream) {
+  if (!qtype_ok(qtype)) return fail(NTX_ERR_QTYPE, "unsupported weight type %d", qtype);
+  if (M < 1 || M > 2147483647LL || K < 1 || K > 262144 || K % block_elems(qtype))
+    return fail(NTX_ERR_SHAPE, "bad shape M=%lld K=%lld for type %d", (long long)M, (long long)K, qtype);
+  if (!W || !x || !y) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(W, 16) || !aligned(x, 16) || !aligned(y, 16) || (residual && !aligned(residual, 16)))
+    return fail(NTX_ERR_ALIGN, "W, x, y, residual must be 16-byte aligned");
+  if (ranges_overlap(x, (size_t)K * 4, y, (size_t)M * 4)) return fail(NTX_ERR_INVALID_ARG, "y overlaps x");
+  if (residual && residual != y && ranges_overlap(residual, (size_t)M * 4, y, (size_t)M * 4))
+    return fail(NTX_ERR_INVALID_ARG, "residual partially overlaps y");
+  const cudaError_t e = ntx::launch_gemv(qtype, W, M, K, x, y, residual, S(stream), false);
+  return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_gemv_q");
+}
+
+int ntx_set_gemv_ctas_per_sm(int cps) {
+  if (cps < 1 || cps > 4) return fail(NTX_ERR_INVALID_ARG, "ctas per SM must be 1..4");
+  ntx::set_gemv_ctas_per_sm(cps);
+  return NTX_OK;
+}
+
+int ntx_rmsnorm(const float* x, const float* w, float* y, int64_t n, float eps, void* stream) {
+  if (n < 1 || n > (1 << 20)) return fail(NTX_ERR_SHAPE, "n=%lld out of range", (long long)n);
+  if (!x || !w || !y) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  if (!(eps >= 0.f)) return fail(NTX_ERR_INVALID_ARG, "eps must be >= 0");
+  if (!aligned(x, 4) || !aligned(w, 4) || !aligned(y, 4)) return fail(NTX_ERR_ALIGN, "pointers must be 4-byte aligned");
+  const cudaError_t e = ntx::launch_rmsnorm(x, w, y, n, eps, S(stream));
+  return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_rmsnorm");
+}
+
+int ntx_rope(float* q, float* k, int n_q_heads, int n_kv_heads, int head_dim, int pos, float theta, void* stream) {
+  if (head_dim < 2 || head_dim > 256 || head_dim % 2) return fail(NTX_ERR_SHAPE, "head_dim %d", head_dim);
+  if (n_q_heads < 0 || n_kv_heads < 0 || pos < 0) return fail(NTX_ERR_INVALID_ARG, "negative heads or pos");
+  if ((n_q_heads > 0 && !q) || (n_kv_heads > 0 && !k)) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  if (!(theta > 0.f)) return fail(NTX_ERR_INVALID_ARG, "theta must be > 0");
+  const cudaError_t e = ntx::launch_rope(q, k, n_q_heads, n_kv_heads, head_dim, pos, theta, S(stream));
+  return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_rope");
+}
+
+size_t ntx_attn_workspace_bytes(int n_q_heads, int n_kv_heads, int head_dim, int max_ctx) {
+  if (n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || max_ctx <= 0) return 0;
+  const int ns = ntx::attn_splits(n_kv_heads, max_ctx);
+  return (size_t)n_q_heads * ns * (head_dim + 2) * sizeof(float);
+}
+
+int ntx_attn_decode(const float* q, const uint16_t* k_cache, const uint16_t* v_cache, float* out, int n_q_heads,
+                    int n_kv_heads, int head_dim, int n_ctx, int max_ctx, void* workspace, size_t ws_bytes,
+                    void* stream) {
+  if (head_dim != 128) return fail(NTX_ERR_SHAPE, "head_dim %d unsupported (128 only)", head_dim);
+  if (n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads) return fail(NTX_ERR_SHAPE, "bad head counts");
+  const int G = n_q_heads / n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(NTX_ERR_SHAPE, "query group %d unsupported", G);
+  if (n_ctx < 1 || n_ctx > max_ctx) return fail(NTX_ERR_SHAPE, "n_ctx %d outside [1, max_ctx=%d]", n_ctx, max_ctx);
+  if (!q || !k_cache || !v_cache || !out || !workspace) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(q, 16) || !aligned(out, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(workspace, 16))
+    return fail(NTX_ERR_ALIGN, "q, caches and workspace must be 16-byte aligned");
+  if (ws_bytes < ntx_attn_workspace_bytes(n_q_heads, n_kv_heads, head_dim, max_ctx))
+    return fail(NTX_ERR_NOMEM, "workspace too small (%zu < %zu)", ws_bytes,
+                ntx_attn_workspace_bytes(n_q_heads, n_kv_heads, head_dim, max_ctx));
+  const int ns = ntx::attn_splits(n_kv_heads, n_ctx);
+  const cudaError_t e = ntx::launch_attn(q, k_cache, v_cache, out, static_cast<float*>(workspace), n_q_heads,
+                                         n_kv_heads, n_ctx, nullptr, max_ctx, ns, S(stream), false);
+  return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_attn_decode");
+}
+
+int ntx_swiglu(const float* gate, const float* up, float* out, int64_t n, void* stream) {
+  if (n < 0) return fail(NTX_ERR_SHAPE, "n < 0");
+  if (n == 0) return NTX_OK;
+  if (!gate || !up || !out) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  const cudaError_t e = ntx::launch_swiglu(gate, up, out, n, S(stream));
+  return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_swiglu");
+}
+
+uint64_t ntx_layer_layout(const ntx_model_config* cfg, int qtype, ntx_layer_weights* out) {
+  if (!cfg || !out || !qtype_ok(qtype) || cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 ||
+      cfg->n_kv_heads <= 0 || cfg->head_dim <= 0)
+    return 0;
+  const int64_t H = cfg->hidden, F = cfg->ffn, Q = (int64_t)cfg->n_heads * cfg->head_dim,
+                KV = (int64_t)cfg->n_kv_heads * cfg->head_dim;
+  if (H % block_elems(qtype) || F % block_elems(qtype) || Q % block_elems(qtype)) return 0;
+  ntx_layer_weights w;
+  memset(&w, 0, sizeof w);
+  w.qtype = qtype;
+  uint64_t o = 0;
+  w.off_wq = o; o = align256(o + mat_bytes(qtype, Q, H));
+  w.off_wk = o; o = align256(o + mat_bytes(qtype, KV, H));
+  w.off_wv = o; o = align256(o + mat_bytes(qtype, KV, H));
+  w.off_wo = o; o = align256(o + mat_bytes(qtype, H, Q));
+  w.off_wg = o; o = align256(o + mat_bytes(qtype, F, H));
+  w.off_wu = o; o = align256(o + mat_bytes(qtype, F, H));
+  w.off_wd = o; o = align256(o + mat_bytes(qtype, H, F));
+  w.off_attn_norm = o; o = align256(o + 4 * H);
+  w.off_ffn_norm = o; o = align256(o + 4 * H);
+  *out = w;
+  return o;
+}
+
+size_t ntx_layer_workspace_bytes(const ntx_model_config* cfg) {
+  if (!cfg || cfg->n_kv_heads <= 0 || cfg->max_ctx <= 0) return 0;
+  return carve_layer(cfg, ntx::attn_splits(cfg->n_kv_heads, cfg->max_ctx), nullptr, nullptr);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Extent of a layer blob given its offsets (for copies and bounds).
+uint64_t layer_extent(const ntx_model_config* c, const ntx_layer_weights* w) {
+  const int qt = w->qtype;
+  const int64_t H = c->hidden, F = c->ffn, Q = (int64_t)c->n_heads * c->head_dim,
+                KV = (int64_t)c->n_kv_heads * c->head_dim;
+  uint64_t e = 0;
+  auto upd = [&](uint64_t off, uint64_t n) { if (off + n > e) e = off + n; };
+  upd(w->off_wq, mat_bytes(qt, Q, H));
+  upd(w->off_wk, mat_bytes(qt, KV, H));
+  upd(w->off_wv, mat_bytes(qt, KV, H));
+  upd(w->off_wo, mat_bytes(qt, H, Q));
+  upd(w->off_wg, mat_bytes(qt, F, H));
+  upd(w->off_wu, mat_bytes(qt, F, H));
+  upd(w->off_wd, mat_bytes(qt, H, F));
+  upd(w->off_attn_norm, 4 * H);
+  upd(w->off_ffn_norm, 4 * H);
+  return e;
+}
+
+int check_offsets(const ntx_layer_weights* w) {
+  const uint64_t offs[7] = {w->off_wq, w->off_wk, w->off_wv, w->off_wo, w->off_wg, w->off_wu, w->off_wd};
+  for (uint64_t o : offs)
+    if (o % 16) return fail(NTX_ERR_ALIGN, "weight matrix offsets must be 16-byte aligned");
+  if (w->off_attn_norm % 16 || w->off_ffn_norm % 16) return fail(NTX_ERR_ALIGN, "norm offsets must be 16-byte aligned");
+  return NTX_OK;
+}
+
+ntx::LayerArgs layer_args(const ntx_model_config* c, const uint8_t* base, int qtype, const ntx_layer_weights* w) {
+  ntx::LayerArgs a;
+  memset(&a, 0, sizeof a);
+  a.qtype = qtype;
+  a.H = c->hidden; a.Hq = c->n_heads; a.Hkv = c->n_kv_heads; a.D = c->head_dim; a.F = c->ffn;
+  a.max_ctx = c->max_ctx; a.eps = c->eps; a.theta = c->theta;
+  a.wq = base + w->off_wq; a.wk = base + w->off_wk; a.wv = base + w->off_wv; a.wo = base + w->off_wo;
+  a.wg = base + w->off_wg; a.wu = base + w->off_wu; a.wd = base + w->off_wd;
+  a.attn_norm = reinterpret_cast<const float*>(base + w->off_attn_norm);
+  a.ffn_norm = reinterpret_cast<const float*>(base + w->off_ffn_norm);
+  return a;
+}
+
+}  // namespace
+
+extern "C" int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_weights* w, uint16_t* k_cache,
+                                uint16_t* v_cache, float* hidden, int pos, float* cos_out, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  if (!w) return fail(NTX_ERR_INVALID_ARG, "weights NULL");
+  int rc = check_config(cfg, w->qtype);
+  if (rc) return rc;
+  if (!w->base || !k_cache || !v_cache || !hidden || !workspace) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  if (pos < 0 || pos >= cfg->max_ctx) return fail(NTX_ERR_SHAPE, "pos %d outside [0, max_ctx)", pos);
+  if ((rc = check_offsets(w))) return rc;
+  if (!aligned(w->base, 16) || !aligned(hidden, 16) || !aligned(workspace, 256) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16))
+    return fail(NTX_ERR_ALIGN, "base, hidden, caches must be 16-byte and workspace 256-byte aligned");
+  if (ws_bytes < ntx_layer_workspace_bytes(cfg)) return fail(NTX_ERR_NOMEM, "workspace too small");
+  const int n_split = ntx::attn_splits(cfg->n_kv_heads, pos + 1);
+  LayerWs ws;
+  carve_layer(cfg, ntx::attn_splits(cfg->n_kv_heads, cfg->max_ctx), static_cast<uint8_t*>(workspace), &ws);
+  ntx::LayerArgs a = layer_args(cfg, static_cast<const uint8_t*>(w->base), w->qtype, w);
+  a.k_cache = k_cache; a.v_cache = v_cache; a.hidden = hidden;
+  const int nin = ntx::layer_stats_parts(cfg->hidden);
+  a.stats_in = ws.stats_in; a.n_stats_in = nin;
+  a.stats_o = ws.stats_o; a.stats_down = ws.stats_down;
+  a.q = ws.q; a.attn_out = ws.attn_out; a.attn_part = ws.attn_part; a.h1 = ws.h1; a.u = ws.u;
+  a.pos = pos; a.pos_dev = nullptr; a.n_split = n_split;
+  cudaStream_t s = S(stream);
+  cudaError_t e = ntx::launch_sumsq(hidden, cfg->hidden, ws.stats_in, nin, s, false);
+  if (e == cudaSuccess) e = ntx::launch_layer(a, s, true);
+  if (e == cudaSuccess && cos_out)
+    e = ntx::launch_cos_finalize(ws.stats_down, ntx::layer_stats_parts(cfg->hidden), nullptr, 1, 0, cos_out, s, true);
+  return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_decode_layer");
+}
+
+// ======================================================================
+// Decode engine
+struct ntx_engine {
+  ntx_model_config cfg;
+  std::vector<ntx_layer_weights> layers;
+  std::vector<int8_t> tier;
+  std::vector<uint64_t> extent;
+  uint8_t* slot[2];
+  size_t slot_bytes;
+  const uint16_t* embed;
+  const float* final_norm;
+  const void* head;
+  int head_qtype;
+  std::vector<uint16_t*> kc, vc;
+  cudaStream_t cs, xs;
+  int n_split;
+  int dev;
+  // workspace regions
+  float *hidden, *q, *attn_out, *attn_part, *h1, *u, *stats_embed, *stats_o, *stats_down, *arg_parts, *cos_int,
+      *logits_int;
+  int *params, *token_state, *layer_list;
+  int64_t stats_stride;  // floats between layers in stats_down
+  // pinned parameter ring
+  int* pinned;
+  cudaEvent_t ring_ev[64];
+  int ring_pos;
+  cudaEvent_t copy_done[2], slot_free[2], fork_ev, join_ev;
+  // skip set
+  std::vector<uint8_t> skip;
+  bool skip_valid;
+  // graphs, keyed by (use_skip, logits, next_token, cos_out)
+  std::map<std::tuple<int, float*, int32_t*, float*>, cudaGraphExec_t> graphs;
+};
+
+size_t engine_carve(const ntx_model_config* c, uint8_t* base, ntx_engine* e) {
+  Carve k{base};
+  const int64_t Q = (int64_t)c->n_heads * c->head_dim;
+  const int P = max_parts();
+  const int ns = ntx::attn_splits(c->n_kv_heads, c->max_ctx);
+  const int L = c->n_layers > 0 ? c->n_layers : 1;
+  float* hidden = k.take<float>(c->hidden);
+  float* q = k.take<float>(Q);
+  float* ao = k.take<float>(Q);
+  float* ap = k.take<float>((uint64_t)c->n_heads * ns * (c->head_dim + 2));
+  float* h1 = k.take<float>(c->hidden);
+  float* u = k.take<float>(c->ffn);
+  float* se = k.take<float>((uint64_t)P * 4);
+  float* so = k.take<float>((uint64_t)P * 4);
+  float* sd = k.take<float>((uint64_t)L * P * 4);
+  float* apart = k.take<float>((uint64_t)P * 4);
+  float* ci = k.take<float>(L);
+  float* li = k.take<float>(c->vocab > 0 ? c->vocab : 1);
+  int* params = k.take<int>(4);
+  int* ts = k.take<int>(4);
+  int* ll = k.take<int>(L);
+  if (e) {
+    e->hidden = hidden; e->q = q; e->attn_out = ao; e->attn_part = ap; e->h1 = h1; e->u = u;
+    e->stats_embed = se; e->stats_o = so; e->stats_down = sd; e->arg_parts = apart; e->cos_int = ci;
+    e->logits_int = li; e->params = params; e->token_state = ts; e->layer_list = ll;
+    e->stats_stride = (int64_t)P * 4; e->n_split = ns;
+  }
+  return k.off;
+}
+
+extern "C" size_t ntx_engine_workspace_bytes(const ntx_model_config* cfg) {
+  if (!cfg || cfg->n_kv_heads <= 0 || cfg->max_ctx <= 0 || cfg->n_layers < 0) return 0;
+  return engine_carve(cfg, nullptr, nullptr);
+}
+
+namespace {
+
+constexpr int kEmbedParts = 16;
+
+void engine_free(ntx_engine* e) {
+  if (!e) return;
+  for (auto& kv : e->graphs) cudaGraphExecDestroy(kv.second);
+  e->graphs.clear();
+  for (int i = 0; i < 64; ++i)
+    if (e->ring_ev[i]) cudaEventDestroy(e->ring_ev[i]);
+  for (int i = 0; i < 2; ++i) {
+    if (e->copy_done[i]) cudaEventDestroy(e->copy_done[i]);
+    if (e->slot_free[i]) cudaEventDestroy(e->slot_free[i]);
+  }
+  if (e->fork_ev) cudaEventDestroy(e->fork_ev);
+  if (e->join_ev) cudaEventDestroy(e->join_ev);
+  if (e->pinned) cudaFreeHost(e->pinned);
+  delete e;
+}
+
+// Enqueue the per-token launch sequence (everything after the parameter copy).
+cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t* next_token, float* cos_out,
+                           bool calibrate) {
+  const ntx_model_config& c = e->cfg;
+  cudaStream_t s = e->cs;
+  const bool pdl = true;
+  cudaError_t err = ntx::launch_embed(e->embed, c.hidden, c.vocab, e->params + 1, e->token_state, e->hidden,
+                                      e->stats_embed, kEmbedParts, s, pdl);
+  if (err != cudaSuccess) return err;
+  const float* stats_in = e->stats_embed;
+  int n_in = kEmbedParts;
+  const int nparts = ntx::layer_stats_parts(c.hidden);
+
+  // host-tier layers in execution order
+  std::vector<int> host_layers;
+  for (int l = 0; l < c.n_layers; ++l)
+    if (e->tier[l] == 1 && !(use_skip && e->skip[l])) host_layers.push_back(l);
+  auto issue_copy = [&](int k) -> cudaError_t {
+    const int l = host_layers[k], sl = k & 1;
+    cudaError_t r = cudaStreamWaitEvent(e->xs, e->slot_free[sl], 0);
+    if (r == cudaSuccess)
+      r = cudaMemcpyAsync(e->slot[sl], e->layers[l].base, e->extent[l], cudaMemcpyHostToDevice, e->xs);
+    if (r == cudaSuccess) r = cudaEventRecord(e->copy_done[sl], e->xs);
+    return r;
+  };
+  if (!host_layers.empty()) {
+    // fork the copy stream from the compute stream; both slots start free
+    err = cudaEventRecord(e->fork_ev, s);
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(e->xs, e->fork_ev, 0);
+    if (err == cudaSuccess) err = cudaEventRecord(e->slot_free[0], s);
+    if (err == cudaSuccess) err = cudaEventRecord(e->slot_free[1], s);
+    for (int k = 0; k < (int)host_layers.size() && k < 2 && err == cudaSuccess; ++k) err = issue_copy(k);
+    if (err != cudaSuccess) return err;
+  }
+  int hk = 0;  // index into host_layers
+  std::vector<int> computed;
+  for (int l = 0; l < c.n_layers; ++l) {
+    if (use_skip && e->skip[l]) continue;
+    const uint8_t* base = static_cast<const uint8_t*>(e->layers[l].base);
+    bool on_host = e->tier[l] == 1;
+    if (on_host) {
+      const int sl = hk & 1;
+      err = cudaStreamWaitEvent(s, e->copy_done[sl], 0);
+      if (err != cudaSuccess) return err;
+      base = e->slot[sl];
+    }
+    ntx::LayerArgs a = layer_args(&c, base, e->layers[l].qtype, &e->layers[l]);
+    a.k_cache = e->kc[l]; a.v_cache = e->vc[l]; a.hidden = e->hidden;
+    a.stats_in = stats_in; a.n_stats_in = n_in;
+    a.stats_o = e->stats_o;
+    a.stats_down = e->stats_down + l * e->stats_stride;
+    a.q = e->q; a.attn_out = e->attn_out; a.attn_part = e->attn_part; a.h1 = e->h1; a.u = e->u;
+    a.pos = 0; a.pos_dev = e->params; a.n_split = e->n_split;
+    err = ntx::launch_layer(a, s, pdl);
+    if (err != cudaSuccess) return err;
+    stats_in = a.stats_down;
+    n_in = nparts;
+    computed.push_back(l);
+    if (on_host) {
+      err = cudaEventRecord(e->slot_free[hk & 1], s);
+      if (err == cudaSuccess && hk + 2 < (int)host_layers.size()) err = issue_copy(hk + 2);
+      if (err != cudaSuccess) return err;
+      ++hk;
+    }
+  }
+  if (!host_layers.empty()) {
+    err = cudaEventRecord(e->join_ev, e->xs);
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(s, e->join_ev, 0);
+    if (err != cudaSuccess) return err;
+  }
+  err = ntx::launch_head(e->head_qtype, e->head, c.vocab, c.hidden, e->hidden, e->final_norm, stats_in, n_in, c.eps,
+                         logits ? logits : e->logits_int, e->arg_parts, s, pdl);
+  if (err != cudaSuccess) return err;
+  err = ntx::launch_argmax_finalize(e->arg_parts, ntx::head_parts(c.vocab), e->token_state, next_token, s, pdl);
+  if (err != cudaSuccess) return err;
+  float* cdst = calibrate ? e->cos_int : cos_out;
+  if (cdst && !computed.empty()) {
+    // the layer list is the identity when nothing is skipped
+    const int* list = (use_skip && e->skip_valid) ? e->layer_list : nullptr;
+    err = ntx::launch_cos_finalize(e->stats_down, nparts, list, (int)computed.size(), e->stats_stride, cdst, s, pdl);
+    if (err == cudaSuccess && calibrate && cos_out)
+      err = cudaMemcpyAsync(cos_out, e->cos_int, sizeof(float) * c.n_layers, cudaMemcpyDeviceToDevice, s);
+  }
+  return err;
+}
+
+}  // namespace
+
+extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_weights* layers, const int8_t* tier_map,
+                                 void* slot0, void* slot1, size_t slot_bytes, const uint16_t* embed,
+                                 const float* final_norm, const void* head, int head_qtype,
+                                 uint16_t* const* k_caches, uint16_t* const* v_caches, void* workspace,
+                                 size_t ws_bytes, void* compute_stream, void* copy_stream, ntx_engine** out) {
+  if (!out) return fail(NTX_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!cfg || (cfg->n_layers > 0 && (!layers || !k_caches || !v_caches)))
+    return fail(NTX_ERR_INVALID_ARG, "NULL config, layers or caches");
+  int rc = check_config(cfg, cfg->n_layers > 0 ? layers[0].qtype : head_qtype);
+  if (rc) return rc;
+  if (!qtype_ok(head_qtype) || !k_ok_fused(head_qtype, cfg->hidden))
+    return fail(NTX_ERR_QTYPE, "unsupported head type %d for hidden %d", head_qtype, cfg->hidden);
+  if (cfg->vocab <= 0) return fail(NTX_ERR_SHAPE, "vocab must be > 0");
+  if (!embed || !final_norm || !head || !workspace) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  if (!compute_stream) return fail(NTX_ERR_INVALID_ARG, "compute_stream must be a created (non-default) stream");
+  if (!aligned(workspace, 256) || !aligned(head, 16) || !aligned(final_norm, 16))
+    return fail(NTX_ERR_ALIGN, "workspace 256-byte, head and final_norm 16-byte aligned");
+  if (ws_bytes < ntx_engine_workspace_bytes(cfg)) return fail(NTX_ERR_NOMEM, "workspace too small");
+  bool any_host = false;
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    if ((rc = check_config(cfg, layers[l].qtype))) return rc;
+    if ((rc = check_offsets(&layers[l]))) return rc;
+    if (!layers[l].base || !k_caches[l] || !v_caches[l]) return fail(NTX_ERR_INVALID_ARG, "layer %d: NULL pointer", l);
+    const int t = tier_map ? tier_map[l] : 0;
+    if (t != 0 && t != 1) return fail(NTX_ERR_INVALID_ARG, "tier_map[%d] = %d (0 or 1)", l, t);
+    if (t == 1) any_host = true;
+    if (!aligned(layers[l].base, 16)) return fail(NTX_ERR_ALIGN, "layer %d base not 16-byte aligned", l);
+  }
+  if (any_host && (!slot0 || !slot1 || !copy_stream || copy_stream == compute_stream || !aligned(slot0, 256) ||
+                   !aligned(slot1, 256)))
+    return fail(NTX_ERR_INVALID_ARG, "host-tier layers need two 256-byte aligned slots and a separate copy stream");
+  ntx_engine* e = new (std::nothrow) ntx_engine();
+  if (!e) return fail(NTX_ERR_NOMEM, "engine allocation");
+  e->cfg = *cfg;
+  e->layers.assign(layers, layers + cfg->n_layers);
+  e->tier.resize(cfg->n_layers);
+  e->extent.resize(cfg->n_layers);
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    e->tier[l] = tier_map ? tier_map[l] : 0;
+    e->extent[l] = layer_extent(cfg, &layers[l]);
+    if (e->tier[l] == 1 && e->extent[l] > slot_bytes) {
+      engine_free(e);
+      return fail(NTX_ERR_NOMEM, "layer %d (%llu bytes) does not fit a slot of %zu bytes", l,
+                  (unsigned long long)e->extent[l], slot_bytes);
+    }
+  }
+  e->slot[0] = static_cast<uint8_t*>(slot0);
+  e->slot[1] = static_cast<uint8_t*>(slot1);
+  e->slot_bytes = slot_bytes;
+  e->embed = embed; e->final_norm = final_norm; e->head = head; e->head_qtype = head_qtype;
+  e->kc.assign(k_caches, k_caches + cfg->n_layers);
+  e->vc.assign(v_caches, v_caches + cfg->n_layers);
+  e->cs = S(compute_stream);
+  e->xs = S(copy_stream);
+  cudaGetDevice(&e->dev);
+  engine_carve(cfg, static_cast<uint8_t*>(workspace), e);
+  e->skip.assign(cfg->n_layers, 0);
+  e->skip_valid = false;
+  cudaError_t err = cudaHostAlloc(reinterpret_cast<void**>(&e->pinned), 64 * 4 * sizeof(int), cudaHostAllocDefault);
+  for (int i = 0; i < 64 && err == cudaSuccess; ++i) err = cudaEventCreateWithFlags(&e->ring_ev[i], cudaEventDisableTiming);
+  for (int i = 0; i < 2 && err == cudaSuccess; ++i) {
+    err = cudaEventCreateWithFlags(&e->copy_done[i], cudaEventDisableTiming);
+    if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->slot_free[i], cudaEventDisableTiming);
+  }
+  if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->fork_ev, cudaEventDisableTiming);
+  if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->join_ev, cudaEventDisableTiming);
+  // token state starts at 0
+  if (err == cudaSuccess) err = cudaMemsetAsync(e->token_state, 0, 4 * sizeof(int), e->cs);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(e->cs);
+  if (err != cudaSuccess) {
+    engine_free(e);
+    return cuda_fail(err, "ntx_engine_create");
+  }
+  *out = e;
+  return NTX_OK;
+}
+
+extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* logits, int32_t* next_token, int flags,
+                               float* cos_out) {
+  if (!e) return fail(NTX_ERR_INVALID_ARG, "engine is NULL");
+  const ntx_model_config& c = e->cfg;
+  if (pos < 0 || pos >= c.max_ctx) return fail(NTX_ERR_SHAPE, "pos %d outside [0, max_ctx=%d)", pos, c.max_ctx);
+  if (token < -1 || token >= c.vocab) return fail(NTX_ERR_INVALID_ARG, "token %d outside [-1, vocab)", token);
+  if (flags & ~(NTX_CALIBRATE_SKIP | NTX_USE_SKIP | NTX_NO_GRAPH)) return fail(NTX_ERR_INVALID_ARG, "unknown flags");
+  const bool calibrate = flags & NTX_CALIBRATE_SKIP;
+  const bool use_skip = !calibrate && (flags & NTX_USE_SKIP) && e->skip_valid;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != e->dev) return fail(NTX_ERR_INVALID_ARG, "engine was created on device %d, current is %d", e->dev, cur);
+
+  // step parameters: pinned ring slot -> device
+  const int slot = e->ring_pos;
+  e->ring_pos = (e->ring_pos + 1) % 64;
+  cudaError_t err = cudaEventSynchronize(e->ring_ev[slot]);
+  if (err != cudaSuccess) return cuda_fail(err, "param ring");
+  e->pinned[slot * 4 + 0] = pos;
+  e->pinned[slot * 4 + 1] = token;
+  err = cudaMemcpyAsync(e->params, e->pinned + slot * 4, 2 * sizeof(int), cudaMemcpyHostToDevice, e->cs);
+  if (err == cudaSuccess) err = cudaEventRecord(e->ring_ev[slot], e->cs);
+  if (err != cudaSuccess) return cuda_fail(err, "param copy");
+
+  if ((flags & NTX_NO_GRAPH) || calibrate) {
+    err = engine_enqueue(e, use_skip, logits, next_token, cos_out, calibrate);
+    if (err != cudaSuccess) return cuda_fail(err, "ntx_decode_step");
+  } else {
+    const auto key = std::make_tuple(use_skip ? 1 : 0, logits, next_token, cos_out);
+    auto it = e->graphs.find(key);
+    if (it == e->graphs.end()) {
+      cudaGraph_t g = nullptr;
+      err = cudaStreamBeginCapture(e->cs, cudaStreamCaptureModeThreadLocal);
+      if (err != cudaSuccess) return cuda_fail(err, "begin capture");
+      const cudaError_t err_enq = engine_enqueue(e, use_skip, logits, next_token, cos_out, false);
+      err = cudaStreamEndCapture(e->cs, &g);
+      if (err_enq != cudaSuccess || err != cudaSuccess) {
+        if (g) cudaGraphDestroy(g);
+        return cuda_fail(err_enq != cudaSuccess ? err_enq : err, "capture of the decode step");
+      }
+      cudaGraphExec_t ge = nullptr;
+      err = cudaGraphInstantiate(&ge, g, 0);
+      cudaGraphDestroy(g);
+      if (err != cudaSuccess) return cuda_fail(err, "graph instantiate");
+      it = e->graphs.emplace(key, ge).first;
+    }
+    err = cudaGraphLaunch(it->second, e->cs);
+    if (err != cudaSuccess) return cuda_fail(err, "graph launch");
+  }
+
+  if (calibrate) {
+    std::vector<float> cs(c.n_layers);
+    err = cudaMemcpyAsync(cs.data(), e->cos_int, sizeof(float) * c.n_layers, cudaMemcpyDeviceToHost, e->cs);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(e->cs);
+    if (err != cudaSuccess) return cuda_fail(err, "calibration read-back");
+    std::vector<int> list;
+    for (int l = 0; l < c.n_layers; ++l) {
+      e->skip[l] = cs[l] >= c.skip_threshold ? 1 : 0;
+      if (!e->skip[l]) list.push_back(l);
+    }
+    if (!list.empty()) {
+      err = cudaMemcpy(e->layer_list, list.data(), sizeof(int) * list.size(), cudaMemcpyHostToDevice);
+      if (err != cudaSuccess) return cuda_fail(err, "layer list");
+    }
+    e->skip_valid = true;
+    // graphs built with an older skip set are stale
+    for (auto itg = e->graphs.begin(); itg != e->graphs.end();) {
+      if (std::get<0>(itg->first) == 1) {
+        cudaGraphExecDestroy(itg->second);
+        itg = e->graphs.erase(itg);
+      } else {
+        ++itg;
+      }
+    }
+  }
+  return NTX_OK;
+}
+
+extern "C" int ntx_engine_skip_mask(ntx_engine* e, uint8_t* mask_host) {
+  if (!e || !mask_host) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  int n = 0;
+  for (int l = 0; l < e->cfg.n_layers; ++l) {
+    mask_host[l] = e->skip_valid ? e->skip[l] : 0;
+    n += mask_host[l];
+  }
+  return n;
+}
+
+extern "C" void ntx_engine_destroy(ntx_engine* e) {
+  if (!e) return;
+  cudaStreamSynchronize(e->cs);
+  if (e->xs) cudaStreamSynchronize(e->xs);
+  engine_free(e);
+}

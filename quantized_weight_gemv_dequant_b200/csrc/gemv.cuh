@@ -1,0 +1,662 @@
+// gemv.cuh -- fused dequantize + GEMV for GGUF Q8_0 / Q4_0 / Q6_K on sm_100a.
+//
+// y = W_deq x with fp32 accumulation ("NTransformer" -- アーキテクチャ概要: the
+// GEMV kernel; decode time is weight bytes over memory bandwidth, "RTX 3090
+// 1枚でLlama 70B" -- VRAMの壁).  Batch-1 GEMV is not a dense contraction: it is
+// bound by HBM bandwidth, so the design is about moving the packed blocks at
+// full bandwidth and decoding them with few instructions, not tensor cores.
+//
+// Work decomposition (one persistent CTA per SM)
+//  * Output rows are split evenly over the CTAs (in units of 1 or 2 rows so
+//    that paired epilogues see both rows of a pair).  A CTA streams its rows in
+//    stages of TR whole rows: one 1-D bulk copy (TMA, cp.async.bulk) per row
+//    into a ring of S shared-memory stages guarded by full/empty mbarriers.
+//  * K is split into slices of 2048 columns.  Consumer warp (c, g) owns slice
+//    c and row group g: its lanes hold their 64 columns of x (fp32, or
+//    RMSNorm(h) w formed on the fly) in registers for the whole kernel, so the
+//    only shared-memory traffic is the weight bytes themselves.  Each warp
+//    reduces a row's partial with shuffles and leaves it in shared memory.
+//  * The producer warp issues the copies (weights never depend on the previous
+//    kernel, so the first S stages go out before the programmatic-launch wait),
+//    sums the slice partials of each finished stage in a fixed order, runs the
+//    epilogue (store, + residual, RoPE + KV append, SwiGLU pairs, residual +
+//    cosine statistics, argmax) and refills the stage.
+//  * Decode is exact: a byte u becomes the float 2^23 + u with one byte
+//    permute (PRMT) and the offset is removed by one exact subtract; products
+//    and sums use packed fp32x2 FMA (FFMA2).  Block scales multiply the block's
+//    inner sum.
+#pragma once
+
+#include "common.cuh"
+
+namespace ntx {
+
+constexpr int QT_Q4_0 = 2, QT_Q8_0 = 8, QT_Q6_K = 14;
+
+constexpr int kSliceCols = 2048;      // columns per K slice (64 per lane)
+constexpr int kMaxConsumers = 15;     // consumer warps per CTA
+constexpr int kMaxTR = 32;            // rows per stage
+constexpr int kGemvThreads = (kMaxConsumers + 1) * 32;
+
+template <int QT>
+struct QTraits;
+template <>
+struct QTraits<QT_Q8_0> {
+  static constexpr int BE = 32, BB = 34, SEG = kSliceCols / 32 * 34;
+};
+template <>
+struct QTraits<QT_Q4_0> {
+  static constexpr int BE = 32, BB = 18, SEG = kSliceCols / 32 * 18;
+};
+template <>
+struct QTraits<QT_Q6_K> {
+  static constexpr int BE = 256, BB = 210, SEG = kSliceCols / 256 * 210;
+};
+
+// Launch plan, computed on the host.
+struct GemvPlan {
+  int TR;        // rows per stage
+  int S;         // stages in the ring
+  int n_slices;  // ceil(K / 2048)
+  int n_rg;      // row groups (consumer warps per slice)
+  int NW;        // consumer warps = n_slices * n_rg
+  int row_bytes;
+  int stage_bytes;
+};
+
+// ------------------------------------------------------------- row maps
+struct MapSingle {
+  const uint8_t* W;
+  int64_t row_bytes;
+  __device__ __forceinline__ const uint8_t* row(int64_t r) const { return W + r * row_bytes; }
+};
+
+// Rows [0, nq) from Wq, [nq, nq+nkv) from Wk, [nq+nkv, nq+2nkv) from Wv.
+struct MapQKV {
+  const uint8_t *Wq, *Wk, *Wv;
+  int64_t row_bytes, nq, nkv;
+  __device__ __forceinline__ const uint8_t* row(int64_t r) const {
+    if (r < nq) return Wq + r * row_bytes;
+    if (r < nq + nkv) return Wk + (r - nq) * row_bytes;
+    return Wv + (r - nq - nkv) * row_bytes;
+  }
+};
+
+// Logical row 2i is row i of Wa, 2i+1 is row i of Wb (gate/up pairs).
+struct MapPair {
+  const uint8_t *Wa, *Wb;
+  int64_t row_bytes;
+  __device__ __forceinline__ const uint8_t* row(int64_t r) const { return ((r & 1) ? Wb : Wa) + (r >> 1) * row_bytes; }
+};
+
+// ------------------------------------------------------------- x loaders
+struct ProPlain {
+  const float* x;
+  __device__ __forceinline__ void setup(int) {}
+  __device__ __forceinline__ float4 ld(int64_t j) const { return ldg4(x + j); }
+};
+
+// x_j = w_j * (h_j * r),  r = 1 / sqrt(sum(h^2)/n + eps), sum(h^2) from the
+// producer's per-CTA partials (slot 0 of 4 floats per CTA).
+struct ProRms {
+  const float* h;
+  const float* w;
+  const float* parts;
+  int nparts;
+  int n;
+  float eps;
+  float r;
+  __device__ __forceinline__ void setup(int lane) {
+    const float ss = warp_sum_array(parts, nparts, 4, lane);
+    r = 1.0f / sqrtf(ss / (float)n + eps);
+  }
+  __device__ __forceinline__ float4 ld(int64_t j) const {
+    const float4 a = ldg4(h + j), b = ldg4(w + j);
+    return make_float4(b.x * (a.x * r), b.y * (a.y * r), b.z * (a.z * r), b.w * (a.w * r));
+  }
+};
+
+// ------------------------------------------------------------- decoders
+__device__ __forceinline__ float byte_f(uint32_t w, int b) { return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | b)); }
+
+// (2^23 + byte ba of wa, 2^23 + byte bb of wb) as one packed pair.
+__device__ __forceinline__ f32x2 bytes_pair(uint32_t wa, int ba, uint32_t wb, int bb) {
+  f32x2 r;
+  asm("{\n\t.reg .b32 lo, hi;\n\t"
+      "prmt.b32 lo, %1, 0x4B000000, %2;\n\t"
+      "prmt.b32 hi, %3, 0x4B000000, %4;\n\t"
+      "mov.b64 %0, {lo, hi};\n\t}"
+      : "=l"(r)
+      : "r"(wa), "r"(0x7440u | (uint32_t)ba), "r"(wb), "r"(0x7440u | (uint32_t)bb));
+  return r;
+}
+
+// Q8_0: lane l owns blocks 2l, 2l+1 of the slice (68 bytes = 17 words at the
+// 4-byte aligned offset 68 l).  Block 0: scale = low half of word 0, q_i =
+// byte 2+i.  Block 1: scale = high half of word 8, q_i = byte 36+i.
+// x2: the lane's 64 columns of x as 32 packed pairs.
+__device__ __forceinline__ float row_q8_0(const uint8_t* seg, int lane, const f32x2* x2) {
+  const uint32_t* wp = reinterpret_cast<const uint32_t*>(seg + lane * 68);
+  uint32_t w[17], xw[17];
+#pragma unroll
+  for (int i = 0; i < 17; ++i) {
+    w[i] = wp[i];
+    xw[i] = w[i] ^ 0x80808080u;
+  }
+  const f32x2 off = pack2(-8388736.0f, -8388736.0f);  // 2^23 + 128
+  float r = 0.f;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    const float d = half_bits_to_float(b == 0 ? w[0] : (w[8] >> 16));
+    const int o = (b == 0) ? 2 : 36;
+    f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i0 = o + 2 * k, i1 = o + 2 * k + 1;
+      const f32x2 v = add2(bytes_pair(xw[i0 >> 2], i0 & 3, xw[i1 >> 2], i1 & 3), off);
+      acc[k & 3] = fma2(v, x2[16 * b + k], acc[k & 3]);
+    }
+    r = fmaf(d, (hsum2(acc[0]) + hsum2(acc[1])) + (hsum2(acc[2]) + hsum2(acc[3])), r);
+  }
+  return r;
+}
+
+// Q4_0: lane l owns blocks 2l, 2l+1 (36 bytes = 9 words at offset 36 l).
+// Block b: scale at byte 18b; nibble byte j at byte 18b + 2 + j (low nibble
+// = element j, high nibble = element j + 16).  Low nibbles decode as
+// 2^23 + n, high nibbles as 2^23 + 16 n (no shift); the high sum is scaled by
+// 1/16, which is exact.
+__device__ __forceinline__ float row_q4_0(const uint8_t* seg, int lane, const f32x2* x2) {
+  const uint32_t* wp = reinterpret_cast<const uint32_t*>(seg + lane * 36);
+  uint32_t w[9];
+#pragma unroll
+  for (int i = 0; i < 9; ++i) w[i] = wp[i];
+  const f32x2 off_lo = pack2(-8388616.0f, -8388616.0f);  // 2^23 + 8
+  const f32x2 off_hi = pack2(-8388736.0f, -8388736.0f);  // 2^23 + 128
+  float r = 0.f;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    const float d = half_bits_to_float(b == 0 ? w[0] : (w[4] >> 16));
+    const int o = (b == 0) ? 2 : 20;
+    f32x2 lo_acc[2] = {0ull, 0ull}, hi_acc[2] = {0ull, 0ull};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int j0 = o + 2 * k, j1 = o + 2 * k + 1;
+      const uint32_t wa = w[j0 >> 2], wb = w[j1 >> 2];
+      const f32x2 lo = add2(bytes_pair(wa & 0x0F0F0F0Fu, j0 & 3, wb & 0x0F0F0F0Fu, j1 & 3), off_lo);
+      const f32x2 hi = add2(bytes_pair(wa & 0xF0F0F0F0u, j0 & 3, wb & 0xF0F0F0F0u, j1 & 3), off_hi);
+      lo_acc[k & 1] = fma2(lo, x2[16 * b + k], lo_acc[k & 1]);
+      hi_acc[k & 1] = fma2(hi, x2[16 * b + 8 + k], hi_acc[k & 1]);
+    }
+    r = fmaf(d, fmaf(0.0625f, hsum2(hi_acc[0]) + hsum2(hi_acc[1]), hsum2(lo_acc[0]) + hsum2(lo_acc[1])), r);
+  }
+  return r;
+}
+
+// Q6_K: a slice is 8 super-blocks (1680 bytes).  Lane (pp = l>>4, h =
+// (l>>3)&1, j = l&7) owns elements 128h + 32g + 4j + t (g, t < 4) of both
+// super-blocks of pairs P = pp and P = pp + 2.  The even super-block of a pair
+// starts 4-byte aligned (pair stride 420 = 4 x 105), the odd one 2 bytes off;
+// its words are re-aligned with a funnel shift.
+__device__ __forceinline__ uint32_t ld_u32_shift2(const uint8_t* p_aligned) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(p_aligned);
+  return __funnelshift_r(w[0], w[1], 16);
+}
+
+__device__ __forceinline__ float i8_to_f(uint32_t w, int b) { return byte_f(w ^ 0x80808080u, b) - 8388736.0f; }
+
+// sb_aligned: the even super-block's first byte, or for the odd one the
+// 4-byte aligned address 2 bytes before its first byte.  x2: 8 pairs,
+// x2[2g + t/2] = columns 128h + 32g + 4j + t (t even, odd) of the super-block.
+template <bool ODD>
+__device__ __forceinline__ float q6k_sb(const uint8_t* sb_aligned, int h, int j, const f32x2* x2) {
+  uint32_t ql0, ql1, qh, sA, sB, sC;
+  float d;
+  const int jj = j >> 2;
+  if (!ODD) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(sb_aligned);
+    ql0 = w[(64 * h + 4 * j) >> 2];
+    ql1 = w[(64 * h + 32 + 4 * j) >> 2];
+    qh = w[(128 + 32 * h + 4 * j) >> 2];
+    sA = w[(192 + 8 * h) >> 2];
+    sB = w[(196 + 8 * h) >> 2];
+    sC = 0;
+    d = half_bits_to_float(w[208 >> 2]);
+  } else {
+    ql0 = ld_u32_shift2(sb_aligned + 64 * h + 4 * j);
+    ql1 = ld_u32_shift2(sb_aligned + 64 * h + 32 + 4 * j);
+    qh = ld_u32_shift2(sb_aligned + 128 + 32 * h + 4 * j);
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(sb_aligned + 192 + 8 * h);
+    sA = w[0]; sB = w[1]; sC = w[2];
+    d = half_bits_to_float(reinterpret_cast<const uint32_t*>(sb_aligned)[208 >> 2] >> 16);
+  }
+  // scales of sub-blocks 8h + jj + 2g, g = 0..3
+  float sc[4];
+  if (!ODD) {
+    sc[0] = i8_to_f(sA, jj); sc[1] = i8_to_f(sA, jj + 2); sc[2] = i8_to_f(sB, jj); sc[3] = i8_to_f(sB, jj + 2);
+  } else {
+    sc[0] = i8_to_f(sA, jj + 2); sc[1] = i8_to_f(sB, jj); sc[2] = i8_to_f(sB, jj + 2); sc[3] = i8_to_f(sC, jj);
+  }
+  const f32x2 off = pack2(-8388640.0f, -8388640.0f);  // 2^23 + 32
+  float acc = 0.f;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const uint32_t lo = ((g & 2) ? ((g & 1) ? ql1 : ql0) >> 4 : ((g & 1) ? ql1 : ql0)) & 0x0F0F0F0Fu;
+    const uint32_t q = lo | (((qh >> (2 * g)) & 0x03030303u) << 4);
+    const f32x2 v01 = add2(bytes_pair(q, 0, q, 1), off);
+    const f32x2 v23 = add2(bytes_pair(q, 2, q, 3), off);
+    const f32x2 s = fma2(v23, x2[2 * g + 1], mul2(v01, x2[2 * g]));
+    acc = fmaf(sc[g], hsum2(s), acc);
+  }
+  return d * acc;
+}
+
+// x2 layout for Q6_K: x2[16 pass + 8 odd + 2g + t/2].
+__device__ __forceinline__ float row_q6_k(const uint8_t* seg, int lane, const f32x2* x2) {
+  const int pp = lane >> 4, h = (lane >> 3) & 1, j = lane & 7;
+  float r = 0.f;
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const uint8_t* base = seg + 420 * (pp + 2 * pass);
+    r += q6k_sb<false>(base, h, j, x2 + 16 * pass) + q6k_sb<true>(base + 208, h, j, x2 + 16 * pass + 8);
+  }
+  return r;
+}
+
+// Columns of x a lane owns within its slice (relative to the slice start):
+// Q8_0/Q4_0: 64 l + i;  Q6_K: 512 P + 256 odd + 128 h + 32 g + 4 j + t.
+template <int QT>
+__device__ __forceinline__ bool lane_active(int lane, int ucols) {
+  if constexpr (QT == QT_Q6_K) return ucols == kSliceCols;  // Q6_K slices are always whole
+  else return 2 * lane < ucols / 32;
+}
+
+template <int QT, class Pro>
+__device__ __forceinline__ void load_x_slice(const Pro& pro, int64_t c0, int lane, f32x2* x2) {
+  if constexpr (QT == QT_Q6_K) {
+    const int pp = lane >> 4, h = (lane >> 3) & 1, j = lane & 7;
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+      for (int odd = 0; odd < 2; ++odd)
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float4 v = pro.ld(c0 + 512 * (pp + 2 * pass) + 256 * odd + 128 * h + 32 * g + 4 * j);
+          f32x2* o = x2 + 16 * pass + 8 * odd + 2 * g;
+          o[0] = pack2(v.x, v.y);
+          o[1] = pack2(v.z, v.w);
+        }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float4 v = pro.ld(c0 + 64 * lane + 4 * i);
+      x2[2 * i] = pack2(v.x, v.y);
+      x2[2 * i + 1] = pack2(v.z, v.w);
+    }
+  }
+}
+
+template <int QT>
+__device__ __forceinline__ float row_dot(const uint8_t* seg, int lane, const f32x2* xr) {
+  if constexpr (QT == QT_Q8_0) return row_q8_0(seg, lane, xr);
+  else if constexpr (QT == QT_Q4_0) return row_q4_0(seg, lane, xr);
+  else return row_q6_k(seg, lane, xr);
+}
+
+// ------------------------------------------------------------- epilogues
+// Run by the producer warp.  apply(r, a, b): kAlign == 1 -> row r has value
+// a; kAlign == 2 -> rows r (even) and r + 1 have values a and b.  Per-lane
+// statistics are reduced over the warp in finish() into
+// parts[blockIdx.x * 4 + k].
+struct EpiStore {
+  float* y;
+  const float* resid;
+  static constexpr int kAlign = 1;
+  __device__ __forceinline__ void init() {}
+  __device__ __forceinline__ void apply(int64_t r, float a, float) { y[r] = resid ? a + resid[r] : a; }
+  __device__ __forceinline__ void finish(int) {}
+};
+
+// QKV with RoPE (adjacent pairs, angle pos * theta^(-2i/D) formed in fp64)
+// and the k, v store into the fp16 caches at row pos.
+struct EpiQKV {
+  float* q_out;
+  uint16_t* k_cache;
+  uint16_t* v_cache;
+  const int* pos_dev;  // if non-null, pos = *pos_dev
+  int pos;
+  int64_t nq, nkv;
+  int head_dim, max_ctx;
+  float theta;
+  static constexpr int kAlign = 2;
+  __device__ __forceinline__ void init() {
+    if (pos_dev) pos = *pos_dev;
+  }
+  __device__ __forceinline__ void apply(int64_t r, float a, float b) {
+    const int64_t i2 = r % head_dim;  // even index within the head
+    if (r < nq + nkv) {
+      const double inv_freq = pow((double)theta, -(double)i2 / (double)head_dim);
+      double s, c;
+      sincos((double)pos * inv_freq, &s, &c);
+      const float cf = (float)c, sf = (float)s;
+      const float ra = a * cf - b * sf, rb = a * sf + b * cf;
+      a = ra;
+      b = rb;
+    }
+    if (r < nq) {
+      q_out[r] = a;
+      q_out[r + 1] = b;
+    } else {
+      const bool is_k = r < nq + nkv;
+      const int64_t kr = is_k ? r - nq : r - nq - nkv;
+      const int64_t head = kr / head_dim;
+      uint16_t* cache = is_k ? k_cache : v_cache;
+      const uint32_t packed = (uint32_t)float_to_half_bits(a) | ((uint32_t)float_to_half_bits(b) << 16);
+      *reinterpret_cast<uint32_t*>(cache + (head * max_ctx + pos) * head_dim + i2) = packed;
+    }
+  }
+  __device__ __forceinline__ void finish(int) {}
+};
+
+// SwiGLU over interleaved (gate, up) rows: out[i] = silu(g_i) u_i.
+struct EpiSwiGLU {
+  float* out;
+  static constexpr int kAlign = 2;
+  __device__ __forceinline__ void init() {}
+  __device__ __forceinline__ void apply(int64_t r, float g, float u) { out[r >> 1] = (g / (1.0f + expf(-g))) * u; }
+  __device__ __forceinline__ void finish(int) {}
+};
+
+// out = v + resid; statistics sum(out^2), sum(hc out), sum(hc^2) where hc is
+// the layer input (read before `out` overwrites it when they alias).
+struct EpiResid {
+  float* out;
+  const float* resid;
+  const float* hc;  // nullable
+  float* parts;     // [gridDim.x][4]
+  float st0, st1, st2;
+  static constexpr int kAlign = 1;
+  __device__ __forceinline__ void init() { st0 = st1 = st2 = 0.f; }
+  __device__ __forceinline__ void apply(int64_t r, float a, float) {
+    const float o = a + resid[r];
+    if (hc) {
+      const float h = hc[r];
+      st1 = fmaf(h, o, st1);
+      st2 = fmaf(h, h, st2);
+    }
+    st0 = fmaf(o, o, st0);
+    out[r] = o;
+  }
+  __device__ __forceinline__ void finish(int lane) {
+    const float a = warp_sum(st0), b = warp_sum(st1), c = warp_sum(st2);
+    if (lane == 0) {
+      parts[blockIdx.x * 4 + 0] = a;
+      parts[blockIdx.x * 4 + 1] = b;
+      parts[blockIdx.x * 4 + 2] = c;
+    }
+  }
+};
+
+// Logits store + argmax (ties -> lowest index) into parts[cta*4] (value) and
+// parts[cta*4 + 1] (index bits, -1 if the CTA had no rows).
+struct EpiArgmax {
+  float* y;
+  float* parts;
+  float best;
+  int64_t besti;
+  static constexpr int kAlign = 1;
+  __device__ __forceinline__ void init() {
+    best = -INFINITY;
+    besti = INT64_MAX;
+  }
+  __device__ __forceinline__ void apply(int64_t r, float a, float) {
+    if (y) y[r] = a;
+    if (a > best || (a == best && r < besti)) { best = a; besti = r; }
+  }
+  __device__ __forceinline__ void finish(int lane) {
+    float b = best;
+    int64_t bi = besti;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, b, o);
+      const int64_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > b || (ob == b && oi < bi)) { b = ob; bi = oi; }
+    }
+    if (lane == 0) {
+      parts[blockIdx.x * 4] = b;
+      reinterpret_cast<int*>(parts)[blockIdx.x * 4 + 1] = (int)(bi == INT64_MAX ? -1 : bi);
+    }
+  }
+};
+
+// ------------------------------------------------------------- kernel
+// Warp-uniform bounded wait on an mbarrier phase: each lane sleeps in the
+// hardware try_wait; the warp agrees on the outcome.  False on timeout.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  bool done = mbar_try_wait(bar, parity);
+  if (__all_sync(0xffffffffu, done)) return true;
+  const uint64_t t0 = global_ns();
+  while (!__all_sync(0xffffffffu, done)) {
+    if (!done) done = mbar_try_wait_sleep(bar, parity);
+    if (__any_sync(0xffffffffu, !done && global_ns() - t0 > kWaitLimitNs)) break;
+  }
+  return __all_sync(0xffffffffu, done);
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+template <int QT, class Map, class Pro, class Epi>
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    gemv_tma_kernel(Map map, Pro pro, Epi epi, int64_t M, int64_t K, GemvPlan p, int* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.S * p.stage_bytes);
+  uint64_t* empty = full + p.S;
+  float* red = reinterpret_cast<float*>(empty + p.S);  // [S][TR][n_slices]
+  int* abort_flag = reinterpret_cast<int*>(red + p.S * p.TR * p.n_slices);
+
+  // rows of this CTA, in units of Epi::kAlign rows
+  const int64_t A = Epi::kAlign;
+  const int64_t units = (M + A - 1) / A;
+  const int64_t r0 = units * blockIdx.x / gridDim.x * A;
+  const int64_t r1 = min64(M, units * (blockIdx.x + 1) / gridDim.x * A);
+  const int64_t nrows = r1 > r0 ? r1 - r0 : 0;
+  const int n_stages = (int)((nrows + p.TR - 1) / p.TR);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], p.NW);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == p.NW) {
+    // ---------------------------------------------------------- producer
+    const uint64_t policy = l2_evict_first_policy();
+    auto issue = [&](int i, int s) {
+      const int64_t rs = r0 + (int64_t)i * p.TR;
+      const int nr = (int)min64(p.TR, r1 - rs);
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(nr * p.row_bytes));
+      __syncwarp();
+      for (int r = lane; r < nr; r += 32)
+        bulk_g2s(ring + (size_t)s * p.stage_bytes + (size_t)r * p.row_bytes, map.row(rs + r), (uint32_t)p.row_bytes,
+                 &full[s], policy);
+    };
+    // Weights do not depend on the previous kernel: start streaming them first.
+    const int pre = min(p.S, n_stages);
+    for (int i = 0; i < pre; ++i) issue(i, i);
+    pdl_launch_dependents();
+    pdl_wait();
+    epi.init();
+    int i = 0, s = 0;
+    uint32_t ph = 0;
+    for (; i < n_stages; ++i) {
+      if (!warp_wait(&empty[s], ph)) break;
+      const int64_t rs = r0 + (int64_t)i * p.TR;
+      const int nr = (int)min64(p.TR, r1 - rs);
+      const float* rd = red + (size_t)s * p.TR * p.n_slices;
+      if constexpr (Epi::kAlign == 1) {
+        if (lane < nr) {
+          float v = 0.f;
+          for (int c = 0; c < p.n_slices; ++c) v += rd[lane * p.n_slices + c];
+          epi.apply(rs + lane, v, 0.f);
+        }
+      } else {
+        if (2 * lane < nr) {
+          float a = 0.f, b = 0.f;
+          for (int c = 0; c < p.n_slices; ++c) {
+            a += rd[(2 * lane) * p.n_slices + c];
+            b += rd[(2 * lane + 1) * p.n_slices + c];
+          }
+          epi.apply(rs + 2 * lane, a, b);
+        }
+      }
+      __syncwarp();
+      if (i + p.S < n_stages) issue(i + p.S, s);
+      if (++s == p.S) { s = 0; ph ^= 1u; }
+    }
+    if (i < n_stages) {
+      // A wait ran out: record it, stop the consumers, and let the copies
+      // already issued land before the CTA's shared memory is released.
+      if (lane == 0) {
+        atomicExch(status, (int)kStatusTmaTimeout);
+        atomicExch(abort_flag, 1);
+        const uint64_t t0 = global_ns();
+        for (int k = i; k < min(i + p.S, n_stages); ++k)
+          while (!mbar_try_wait(&full[k % p.S], (uint32_t)((k / p.S) & 1)))
+            if (global_ns() - t0 > kWaitLimitNs) { atomicExch(status, (int)kStatusDrainTimeout); break; }
+      }
+      __syncwarp();
+    }
+    epi.finish(lane);
+  } else {
+    // ---------------------------------------------------------- consumers
+    pdl_launch_dependents();
+    pdl_wait();
+    const int c = warp % p.n_slices, g = warp / p.n_slices;
+    const int64_t c0 = (int64_t)c * kSliceCols;
+    const int ucols = (int)min64(kSliceCols, K - c0);
+    const bool active = lane_active<QT>(lane, ucols);
+    pro.setup(lane);
+    f32x2 xr[32];
+    if (active) load_x_slice<QT>(pro, c0, lane, xr);
+    int s = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < n_stages; ++i) {
+      if (!warp_wait(&full[s], ph)) {
+        if (lane == 0) atomicExch(abort_flag, 1);
+        break;
+      }
+      const int64_t rs = r0 + (int64_t)i * p.TR;
+      const int nr = (int)min64(p.TR, r1 - rs);
+      const uint8_t* st = ring + (size_t)s * p.stage_bytes + (size_t)c * QTraits<QT>::SEG;
+      float* rd = red + (size_t)s * p.TR * p.n_slices;
+      for (int r = g; r < nr; r += p.n_rg) {
+        float v = active ? row_dot<QT>(st + (size_t)r * p.row_bytes, lane, xr) : 0.f;
+        v = warp_sum(v);
+        if (lane == 0) rd[r * p.n_slices + c] = v;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == p.S) { s = 0; ph ^= 1u; }
+      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
+    }
+  }
+}
+
+// Host-side plan for a GEMV over rows of row_bytes bytes.  smem budget in
+// bytes for the ring; align: 1 or 2 (rows per epilogue unit).
+inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget) {
+  GemvPlan p;
+  const int be = qtype == QT_Q6_K ? 256 : 32, bb = qtype == QT_Q6_K ? 210 : (qtype == QT_Q8_0 ? 34 : 18);
+  p.row_bytes = (int)(K / be * bb);
+  p.n_slices = (int)((K + kSliceCols - 1) / kSliceCols);
+  int trmax = 34816 / p.row_bytes;
+  if (trmax < 1) trmax = 1;
+  if (trmax > kMaxTR) trmax = kMaxTR;
+  int n_rg = kMaxConsumers / p.n_slices;
+  if (n_rg < 1) n_rg = 1;
+  if (n_rg > trmax) n_rg = trmax;
+  int tr = trmax / n_rg * n_rg;
+  if (align == 2 && (tr & 1)) {
+    if (tr > 1) tr -= 1;
+    else tr = 2;
+    if (n_rg > tr) n_rg = tr;
+    tr = tr / n_rg * n_rg;
+    if (tr & 1) { tr = 2; n_rg = n_rg > 2 ? 2 : n_rg; }
+  }
+  p.TR = tr;
+  p.n_rg = n_rg;
+  p.NW = p.n_slices * n_rg;
+  p.stage_bytes = p.TR * p.row_bytes;
+  int S = smem_budget / p.stage_bytes;
+  if (S > 8) S = 8;
+  if (S < 2) S = 2;
+  p.S = S;
+  return p;
+}
+
+inline size_t gemv_smem_bytes(const GemvPlan& p) {
+  return (size_t)p.S * p.stage_bytes + (size_t)p.S * 16 + (size_t)p.S * p.TR * p.n_slices * 4 + 16;
+}
+
+// ------------------------------------------------------------- generic path
+// Any K that is a multiple of the block length, any alignment >= 2 bytes:
+// one warp per row, lanes stride over blocks, byte loads.  Used only for shapes
+// the bulk-copy path cannot take.
+template <int QT>
+__device__ __forceinline__ float block_dot_generic(const uint8_t* blk, const float* x) {
+  if constexpr (QT == QT_Q8_0) {
+    const float d = half_bits_to_float(blk[0] | (blk[1] << 8));
+    float s = 0.f;
+    for (int i = 0; i < 32; ++i) s = fmaf((float)(int8_t)blk[2 + i], x[i], s);
+    return d * s;
+  } else if constexpr (QT == QT_Q4_0) {
+    const float d = half_bits_to_float(blk[0] | (blk[1] << 8));
+    float s = 0.f;
+    for (int j = 0; j < 16; ++j) {
+      s = fmaf((float)((blk[2 + j] & 15) - 8), x[j], s);
+      s = fmaf((float)((blk[2 + j] >> 4) - 8), x[j + 16], s);
+    }
+    return d * s;
+  } else {
+    const float d = half_bits_to_float(blk[208] | (blk[209] << 8));
+    float s = 0.f;
+    for (int sub = 0; sub < 16; ++sub) {
+      float t = 0.f;
+      for (int e = 0; e < 16; ++e) {
+        const int n = 16 * sub + e, h = n >> 7, rr = n & 127, g = rr >> 5, l = rr & 31;
+        const int byte = blk[64 * h + 32 * (g & 1) + l];
+        const int lo = (g < 2) ? (byte & 15) : (byte >> 4);
+        const int hi = (blk[128 + 32 * h + l] >> (2 * g)) & 3;
+        t = fmaf((float)((lo | (hi << 4)) - 32), x[n], t);
+      }
+      s = fmaf((float)(int8_t)blk[192 + sub], t, s);
+    }
+    return d * s;
+  }
+}
+
+template <int QT>
+__global__ void gemv_generic_kernel(const uint8_t* W, int64_t M, int64_t K, const float* x, float* y,
+                                    const float* resid) {
+  using T = QTraits<QT>;
+  const int lane = threadIdx.x & 31;
+  const int64_t nb = K / T::BE;
+  const int64_t row_bytes = nb * T::BB;
+  for (int64_t r = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); r < M;
+       r += (int64_t)gridDim.x * (blockDim.x / 32)) {
+    float s = 0.f;
+    for (int64_t b = lane; b < nb; b += 32) s += block_dot_generic<QT>(W + r * row_bytes + b * T::BB, x + b * T::BE);
+    s = warp_sum(s);
+    if (lane == 0) y[r] = resid ? s + resid[r] : s;
+  }
+}
+
+}  // namespace ntx

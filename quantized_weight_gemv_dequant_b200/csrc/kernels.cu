@@ -1,0 +1,303 @@
+// kernels.cu -- instantiation and launch of every libntx kernel (sm_100a).
+#include <mutex>
+#include <utility>
+
+#include "attn.cuh"
+#include "common.cuh"
+#include "gemv.cuh"
+#include "launch.h"
+#include "ops.cuh"
+
+namespace ntx {
+
+__device__ int g_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices];
+int g_cps = 1;
+std::mutex g_mu;
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+int* status_ptr() {
+  static int* ptrs[kMaxDevices];
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  if (!ptrs[d]) {
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!ptrs[d]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_status) == cudaSuccess) ptrs[d] = static_cast<int*>(p);
+    }
+  }
+  return ptrs[d];
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device; `done`
+// is a per-kernel bit set (one bit per device).
+template <class K>
+cudaError_t ensure_smem(K kern, size_t bytes, unsigned long long& done) {
+  const int d = current_device();
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  if (done & (1ull << d)) return cudaSuccess;
+  std::lock_guard<std::mutex> g(g_mu);
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done |= 1ull << d;
+  return e;
+}
+
+template <class... KArgs, class... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+int grid_1d(int64_t n, int threads, int cap) {
+  int64_t g = (n + threads - 1) / threads;
+  if (g > cap) g = cap;
+  return g < 1 ? 1 : (int)g;
+}
+
+constexpr int kRingBudget = 150 * 1024;   // shared memory for the weight ring
+constexpr int kSmemMax = 200 * 1024;      // attribute ceiling for every GEMV instantiation
+
+template <int QT, class Map, class Pro, class Epi>
+cudaError_t gemv_tma(Map map, Pro pro, Epi epi, int64_t M, int64_t K, int grid, cudaStream_t s, bool pdl) {
+  static unsigned long long done = 0;  // unique per <QT, Map, Pro, Epi>
+  auto kern = gemv_tma_kernel<QT, Map, Pro, Epi>;
+  const GemvPlan plan = make_gemv_plan(QT, K, Epi::kAlign, kRingBudget);
+  const size_t smem = gemv_smem_bytes(plan);
+  cudaError_t e = ensure_smem(kern, kSmemMax, done);
+  if (e != cudaSuccess) return e;
+  return launch_k(kern, dim3(grid), dim3((plan.NW + 1) * 32), smem, s, pdl, map, pro, epi, M, K, plan, status_ptr());
+}
+
+}  // namespace
+
+int sm_count() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  if (!g_sms[d]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || v <= 0) v = 148;
+    g_sms[d] = v;
+  }
+  return g_sms[d];
+}
+
+void set_gemv_ctas_per_sm(int cps) { g_cps = cps < 1 ? 1 : (cps > 4 ? 4 : cps); }
+int gemv_ctas_per_sm() { return g_cps; }
+
+int gemv_grid(int64_t M, int align) {
+  const int64_t units = (M + align - 1) / align;
+  const int64_t cap = (int64_t)sm_count() * g_cps;
+  return (int)(units < cap ? (units < 1 ? 1 : units) : cap);
+}
+
+int attn_splits(int n_kv_heads, int n_ctx) {
+  if (n_ctx < 1) n_ctx = 1;
+  int s = (2 * sm_count() + n_kv_heads - 1) / n_kv_heads;
+  const int need = (n_ctx + kAttnMaxChunk - 1) / kAttnMaxChunk;
+  if (s < need) s = need;
+  if (s > n_ctx) s = n_ctx;
+  return s < 1 ? 1 : s;
+}
+
+bool gemv_tma_ok(int qtype, const void* W, int64_t K) {
+  if ((reinterpret_cast<uintptr_t>(W) & 15) != 0) return false;
+  if (qtype == QT_Q8_0 || qtype == QT_Q4_0) return K % 256 == 0 && K <= (int64_t)kMaxConsumers * kSliceCols;
+  if (qtype == QT_Q6_K) return K % 2048 == 0 && K <= (int64_t)kMaxConsumers * kSliceCols;
+  return false;
+}
+
+cudaError_t launch_dequant(int qtype, const void* blocks, float* out, int64_t nblocks, cudaStream_t s) {
+  if (nblocks <= 0) return cudaSuccess;
+  const int g = grid_1d(nblocks, 128, sm_count() * 16);
+  const uint8_t* b = static_cast<const uint8_t*>(blocks);
+  if (qtype == QT_Q8_0) dequant_kernel<QT_Q8_0><<<g, 128, 0, s>>>(b, out, nblocks);
+  else if (qtype == QT_Q4_0) dequant_kernel<QT_Q4_0><<<g, 128, 0, s>>>(b, out, nblocks);
+  else dequant_kernel<QT_Q6_K><<<g, 128, 0, s>>>(b, out, nblocks);
+  return cudaGetLastError();
+}
+
+template <int QT>
+static cudaError_t gemv_plain_qt(const void* W, int64_t M, int64_t K, const float* x, float* y, const float* resid,
+                                 cudaStream_t s, bool pdl) {
+  const uint8_t* w = static_cast<const uint8_t*>(W);
+  const int64_t rb = K / QTraits<QT>::BE * QTraits<QT>::BB;
+  if (gemv_tma_ok(QT, W, K)) {
+    EpiStore epi{y, resid};
+    return gemv_tma<QT>(MapSingle{w, rb}, ProPlain{x}, epi, M, K, gemv_grid(M, 1), s, pdl);
+  }
+  const int g = grid_1d(M, 8, sm_count() * 8);
+  gemv_generic_kernel<QT><<<g, 256, 0, s>>>(w, M, K, x, y, resid);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemv(int qtype, const void* W, int64_t M, int64_t K, const float* x, float* y, const float* resid,
+                        cudaStream_t s, bool pdl) {
+  if (qtype == QT_Q8_0) return gemv_plain_qt<QT_Q8_0>(W, M, K, x, y, resid, s, pdl);
+  if (qtype == QT_Q4_0) return gemv_plain_qt<QT_Q4_0>(W, M, K, x, y, resid, s, pdl);
+  return gemv_plain_qt<QT_Q6_K>(W, M, K, x, y, resid, s, pdl);
+}
+
+cudaError_t launch_rmsnorm(const float* x, const float* w, float* y, int64_t n, float eps, cudaStream_t s) {
+  rmsnorm_kernel<<<1, 1024, 0, s>>>(x, w, y, n, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope(float* q, float* k, int nq, int nkv, int head_dim, int pos, float theta, cudaStream_t s) {
+  const int64_t total = (int64_t)(nq + nkv) * (head_dim / 2);
+  if (total <= 0) return cudaSuccess;
+  rope_kernel<<<grid_1d(total, 256, 4096), 256, 0, s>>>(q, k, nq, nkv, head_dim, pos, theta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu(const float* g, const float* u, float* out, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  swiglu_kernel<<<grid_1d(n, 256, sm_count() * 8), 256, 0, s>>>(g, u, out, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn(const float* q, const uint16_t* kc, const uint16_t* vc, float* out, float* part, int Hq,
+                        int Hkv, int n_ctx, const int* pos_dev, int max_ctx, int n_split, cudaStream_t s, bool pdl) {
+  const int G = Hq / Hkv;
+  const dim3 grid(n_split, Hkv);
+  const dim3 block(kAttnWarps * 32);
+  cudaError_t e;
+  switch (G) {
+    case 1: e = launch_k(attn_split_kernel<1>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split); break;
+    case 2: e = launch_k(attn_split_kernel<2>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split); break;
+    case 4: e = launch_k(attn_split_kernel<4>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split); break;
+    case 8: e = launch_k(attn_split_kernel<8>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  return launch_k(attn_combine_kernel, dim3(Hq), dim3(kAttnD), 0, s, pdl, (const float*)part, out, n_split);
+}
+
+int layer_stats_parts(int64_t H) { return gemv_grid(H, 1); }
+
+template <int QT>
+static cudaError_t layer_qt(const LayerArgs& a, cudaStream_t s, bool pdl) {
+  using T = QTraits<QT>;
+  const int64_t rbH = a.H / T::BE * T::BB;  // rows with K = H
+  const int64_t rbQ = a.Hq * a.D / T::BE * T::BB;  // K = Hq*D
+  const int64_t rbF = a.F / T::BE * T::BB;  // K = F
+  const int64_t nq = a.Hq * a.D, nkv = a.Hkv * a.D;
+  cudaError_t e;
+
+  // 1. RMSNorm prologue + Q/K/V GEMV + RoPE + KV append
+  {
+    ProRms pro{a.hidden, a.attn_norm, a.stats_in, a.n_stats_in, (int)a.H, a.eps, 0.f};
+    EpiQKV epi{a.q, a.k_cache, a.v_cache, a.pos_dev, a.pos, nq, nkv, (int)a.D, a.max_ctx, a.theta};
+    const int64_t M = nq + 2 * nkv;
+    e = gemv_tma<QT>(MapQKV{a.wq, a.wk, a.wv, rbH, nq, nkv}, pro, epi, M, a.H, gemv_grid(M, 2), s, pdl);
+    if (e != cudaSuccess) return e;
+  }
+  // 2. split-KV attention + combine
+  e = launch_attn(a.q, a.k_cache, a.v_cache, a.attn_out, a.attn_part, (int)a.Hq, (int)a.Hkv, a.pos + 1, a.pos_dev,
+                  a.max_ctx, a.n_split, s, pdl);
+  if (e != cudaSuccess) return e;
+  // 3. O projection + residual: h1 = h + Wo a   (statistics: sum h1^2)
+  {
+    EpiResid epi{a.h1, a.hidden, nullptr, a.stats_o, 0.f, 0.f, 0.f};
+    e = gemv_tma<QT>(MapSingle{a.wo, rbQ}, ProPlain{a.attn_out}, epi, a.H, nq, gemv_grid(a.H, 1), s, pdl);
+    if (e != cudaSuccess) return e;
+  }
+  // 4. RMSNorm prologue + gate/up GEMV + SwiGLU
+  {
+    ProRms pro{a.h1, a.ffn_norm, a.stats_o, gemv_grid(a.H, 1), (int)a.H, a.eps, 0.f};
+    EpiSwiGLU epi{a.u};
+    e = gemv_tma<QT>(MapPair{a.wg, a.wu, rbH}, pro, epi, 2 * a.F, a.H, gemv_grid(2 * a.F, 2), s, pdl);
+    if (e != cudaSuccess) return e;
+  }
+  // 5. down projection + residual + cosine statistics: h = h1 + Wd u
+  {
+    EpiResid epi{a.hidden, a.h1, a.hidden, a.stats_down, 0.f, 0.f, 0.f};
+    e = gemv_tma<QT>(MapSingle{a.wd, rbF}, ProPlain{a.u}, epi, a.H, a.F, gemv_grid(a.H, 1), s, pdl);
+  }
+  return e;
+}
+
+cudaError_t launch_layer(const LayerArgs& a, cudaStream_t s, bool pdl) {
+  if (a.qtype == QT_Q8_0) return layer_qt<QT_Q8_0>(a, s, pdl);
+  if (a.qtype == QT_Q4_0) return layer_qt<QT_Q4_0>(a, s, pdl);
+  return layer_qt<QT_Q6_K>(a, s, pdl);
+}
+
+cudaError_t launch_sumsq(const float* h, int64_t n, float* parts, int nparts, cudaStream_t s, bool pdl) {
+  return launch_k(sumsq_kernel, dim3(nparts), dim3(256), 0, s, pdl, h, n, parts);
+}
+
+cudaError_t launch_embed(const uint16_t* table, int64_t H, int64_t V, const int* tok_param, const int* tok_state,
+                         float* h, float* parts, int nparts, cudaStream_t s, bool pdl) {
+  return launch_k(embed_kernel, dim3(nparts), dim3(256), 0, s, pdl, table, H, V, tok_param, tok_state, h, parts,
+                  status_ptr());
+}
+
+int head_parts(int64_t V) { return gemv_grid(V, 1); }
+
+template <int QT>
+static cudaError_t head_qt(const void* W, int64_t V, int64_t H, const float* h, const float* final_norm,
+                           const float* stats_in, int n_stats_in, float eps, float* logits, float* arg_parts,
+                           cudaStream_t s, bool pdl) {
+  using T = QTraits<QT>;
+  ProRms pro{h, final_norm, stats_in, n_stats_in, (int)H, eps, 0.f};
+  EpiArgmax epi{logits, arg_parts, 0.f, 0};
+  return gemv_tma<QT>(MapSingle{static_cast<const uint8_t*>(W), H / T::BE * T::BB}, pro, epi, V, H, gemv_grid(V, 1),
+                      s, pdl);
+}
+
+cudaError_t launch_head(int qtype, const void* W, int64_t V, int64_t H, const float* h, const float* final_norm,
+                        const float* stats_in, int n_stats_in, float eps, float* logits, float* arg_parts,
+                        cudaStream_t s, bool pdl) {
+  if (qtype == QT_Q8_0) return head_qt<QT_Q8_0>(W, V, H, h, final_norm, stats_in, n_stats_in, eps, logits, arg_parts, s, pdl);
+  if (qtype == QT_Q4_0) return head_qt<QT_Q4_0>(W, V, H, h, final_norm, stats_in, n_stats_in, eps, logits, arg_parts, s, pdl);
+  return head_qt<QT_Q6_K>(W, V, H, h, final_norm, stats_in, n_stats_in, eps, logits, arg_parts, s, pdl);
+}
+
+cudaError_t launch_argmax_finalize(const float* parts, int nparts, int* token_state, int* next_token, cudaStream_t s,
+                                   bool pdl) {
+  return launch_k(argmax_finalize_kernel, dim3(1), dim3(32), 0, s, pdl, parts, nparts, token_state, next_token);
+}
+
+cudaError_t launch_cos_finalize(const float* stats, int nparts, const int* layers, int nlayers, int64_t layer_stride,
+                                float* cos_out, cudaStream_t s, bool pdl) {
+  if (nlayers <= 0) return cudaSuccess;
+  return launch_k(cos_finalize_kernel, dim3(1), dim3(256), 0, s, pdl, stats, nparts, layers, nlayers, layer_stride,
+                  cos_out);
+}
+
+int read_device_status(int* code) {
+  const cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return (int)e;
+  int v = 0;
+  cudaError_t e2 = cudaMemcpyFromSymbol(&v, g_status, sizeof(int));
+  if (e2 != cudaSuccess) return (int)e2;
+  const int zero = 0;
+  e2 = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+  if (e2 != cudaSuccess) return (int)e2;
+  *code = v;
+  return 0;
+}
+
+}  // namespace ntx
