@@ -236,6 +236,18 @@ NTX_API int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_weigh
 NTX_API int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* logits, int32_t* next_token, int flags,
                     float* cos_out);
 
+/* Profiling: while set, every ntx_decode_step made with NTX_NO_GRAPH records
+ * begin_events[k] and end_events[k] (caller-created cudaEvent_t, passed as
+ * void*) on the compute stream immediately before and after the gate/up GEMV
+ * of the k-th computed layer of the step -- the largest kernel of a layer.
+ * n is the capacity of both arrays (layers past it are not probed); n == 0
+ * clears the probe.  Graph replays never record probe events. */
+NTX_API int ntx_engine_set_probe(ntx_engine* e, void* const* begin_events, void* const* end_events, int n);
+
+/* Number of libntx kernels one decode step launched (the last step enqueued
+ * or captured by this engine), or a negative error. */
+NTX_API int ntx_engine_launches_per_step(ntx_engine* e);
+
 /* Copies the recorded skip set (1 = skipped) into mask_host[L]; returns the
  * number of skipped layers, or a negative error. */
 NTX_API int ntx_engine_skip_mask(ntx_engine* e, uint8_t* mask_host);

@@ -36,7 +36,8 @@ EXPORTS = (
     "ntx_last_error", "ntx_version", "ntx_device_status", "ntx_sm_count", "ntx_set_gemv_ctas_per_sm",
     "ntx_dequant", "ntx_gemv_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_workspace_bytes", "ntx_attn_decode",
     "ntx_swiglu", "ntx_layer_layout", "ntx_layer_workspace_bytes", "ntx_decode_layer", "ntx_engine_workspace_bytes",
-    "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy",
+    "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
+    "ntx_engine_launches_per_step",
 )
 
 
@@ -94,6 +95,8 @@ def lib():
             "ntx_decode_step": ([vp, ctypes.c_int32, i32, vp, vp, i32, vp], i32),
             "ntx_engine_skip_mask": ([vp, vp], i32),
             "ntx_engine_destroy": ([vp], None),
+            "ntx_engine_set_probe": ([vp, vp, vp, i32], i32),
+            "ntx_engine_launches_per_step": ([vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -242,3 +245,18 @@ def ntx_engine_skip_mask(engine, n_layers):
 
 def ntx_engine_destroy(engine):
     lib().ntx_engine_destroy(engine)
+
+
+def ntx_engine_set_probe(engine, begin_events, end_events):
+    """begin_events / end_events: sequences of raw cudaEvent_t handles (ints)."""
+    n = len(begin_events)
+    b = (ctypes.c_void_p * max(n, 1))(*begin_events)
+    e = (ctypes.c_void_p * max(n, 1))(*end_events)
+    _check(lib().ntx_engine_set_probe(engine, b, e, n))
+
+
+def ntx_engine_launches_per_step(engine) -> int:
+    rc = lib().ntx_engine_launches_per_step(engine)
+    if rc < 0:
+        _check(rc)
+    return rc

@@ -346,6 +346,9 @@ struct ntx_engine {
   bool skip_valid;
   // graphs, keyed by (use_skip, logits, next_token, cos_out)
   std::map<std::tuple<int, float*, int32_t*, float*>, cudaGraphExec_t> graphs;
+  // profiling probe (kernel-by-kernel steps only) and launch count
+  std::vector<cudaEvent_t> probe_b, probe_e;
+  int launches;
 };
 
 size_t engine_carve(const ntx_model_config* c, uint8_t* base, ntx_engine* e) {
@@ -405,7 +408,7 @@ void engine_free(ntx_engine* e) {
 
 // Enqueue the per-token launch sequence (everything after the parameter copy).
 cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t* next_token, float* cos_out,
-                           bool calibrate) {
+                           bool calibrate, bool probe) {
   const ntx_model_config& c = e->cfg;
   cudaStream_t s = e->cs;
   const bool pdl = true;
@@ -456,6 +459,11 @@ cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t*
     a.stats_down = e->stats_down + l * e->stats_stride;
     a.q = e->q; a.attn_out = e->attn_out; a.attn_part = e->attn_part; a.h1 = e->h1; a.u = e->u;
     a.pos = 0; a.pos_dev = e->params; a.n_split = e->n_split;
+    const size_t k = computed.size();
+    if (probe && k < e->probe_b.size()) {
+      a.probe_begin = e->probe_b[k];
+      a.probe_end = e->probe_e[k];
+    }
     err = ntx::launch_layer(a, s, pdl);
     if (err != cudaSuccess) return err;
     stats_in = a.stats_down;
@@ -478,8 +486,10 @@ cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t*
   if (err != cudaSuccess) return err;
   err = ntx::launch_argmax_finalize(e->arg_parts, ntx::head_parts(c.vocab), e->token_state, next_token, s, pdl);
   if (err != cudaSuccess) return err;
+  e->launches = 1 + ntx::kLayerLaunches * (int)computed.size() + 2;
   float* cdst = calibrate ? e->cos_int : cos_out;
   if (cdst && !computed.empty()) {
+    e->launches += 1;
     // the layer list is the identity when nothing is skipped
     const int* list = (use_skip && e->skip_valid) ? e->layer_list : nullptr;
     err = ntx::launch_cos_finalize(e->stats_down, nparts, list, (int)computed.size(), e->stats_stride, cdst, s, pdl);
@@ -594,7 +604,7 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
   if (err != cudaSuccess) return cuda_fail(err, "param copy");
 
   if ((flags & NTX_NO_GRAPH) || calibrate) {
-    err = engine_enqueue(e, use_skip, logits, next_token, cos_out, calibrate);
+    err = engine_enqueue(e, use_skip, logits, next_token, cos_out, calibrate, (flags & NTX_NO_GRAPH) != 0);
     if (err != cudaSuccess) return cuda_fail(err, "ntx_decode_step");
   } else {
     const auto key = std::make_tuple(use_skip ? 1 : 0, logits, next_token, cos_out);
@@ -603,7 +613,7 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
       cudaGraph_t g = nullptr;
       err = cudaStreamBeginCapture(e->cs, cudaStreamCaptureModeThreadLocal);
       if (err != cudaSuccess) return cuda_fail(err, "begin capture");
-      const cudaError_t err_enq = engine_enqueue(e, use_skip, logits, next_token, cos_out, false);
+      const cudaError_t err_enq = engine_enqueue(e, use_skip, logits, next_token, cos_out, false, false);
       err = cudaStreamEndCapture(e->cs, &g);
       if (err_enq != cudaSuccess || err != cudaSuccess) {
         if (g) cudaGraphDestroy(g);
@@ -655,6 +665,24 @@ extern "C" int ntx_engine_skip_mask(ntx_engine* e, uint8_t* mask_host) {
     n += mask_host[l];
   }
   return n;
+}
+
+extern "C" int ntx_engine_set_probe(ntx_engine* e, void* const* begin_events, void* const* end_events, int n) {
+  if (!e) return fail(NTX_ERR_INVALID_ARG, "engine is NULL");
+  if (n < 0 || (n > 0 && (!begin_events || !end_events))) return fail(NTX_ERR_INVALID_ARG, "bad probe arrays");
+  e->probe_b.clear();
+  e->probe_e.clear();
+  for (int k = 0; k < n; ++k) {
+    if (!begin_events[k] || !end_events[k]) return fail(NTX_ERR_INVALID_ARG, "probe event %d is NULL", k);
+    e->probe_b.push_back(static_cast<cudaEvent_t>(begin_events[k]));
+    e->probe_e.push_back(static_cast<cudaEvent_t>(end_events[k]));
+  }
+  return NTX_OK;
+}
+
+extern "C" int ntx_engine_launches_per_step(ntx_engine* e) {
+  if (!e) return fail(NTX_ERR_INVALID_ARG, "engine is NULL");
+  return e->launches;
 }
 
 extern "C" void ntx_engine_destroy(ntx_engine* e) {

@@ -227,8 +227,10 @@ static cudaError_t layer_qt(const LayerArgs& a, cudaStream_t s, bool pdl) {
   {
     ProRms pro{a.h1, a.ffn_norm, a.stats_o, gemv_grid(a.H, 1), (int)a.H, a.eps, 0.f};
     EpiSwiGLU epi{a.u};
+    if (a.probe_begin && (e = cudaEventRecord(a.probe_begin, s)) != cudaSuccess) return e;
     e = gemv_tma<QT>(MapPair{a.wg, a.wu, rbH}, pro, epi, 2 * a.F, a.H, gemv_grid(2 * a.F, 2), s, pdl);
     if (e != cudaSuccess) return e;
+    if (a.probe_end && (e = cudaEventRecord(a.probe_end, s)) != cudaSuccess) return e;
   }
   // 5. down projection + residual + cosine statistics: h = h1 + Wd u
   {

@@ -44,7 +44,9 @@ struct LayerArgs {
   int pos;             // used when pos_dev is null
   const int* pos_dev;  // device position word (engine)
   int n_split;
+  cudaEvent_t probe_begin, probe_end;  // recorded around the gate/up GEMV when set
 };
+constexpr int kLayerLaunches = 6;  // kernels one launch_layer() enqueues
 cudaError_t launch_layer(const LayerArgs& a, cudaStream_t s, bool pdl);
 // Number of statistics partials the down projection of a layer writes.
 int layer_stats_parts(int64_t H);
