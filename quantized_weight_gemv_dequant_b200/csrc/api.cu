@@ -306,6 +306,7 @@ extern "C" int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_wei
   a.stats_o = ws.stats_o; a.stats_down = ws.stats_down;
   a.q = ws.q; a.attn_out = ws.attn_out; a.attn_part = ws.attn_part; a.h1 = ws.h1; a.u = ws.u;
   a.pos = pos; a.pos_dev = nullptr; a.n_split = n_split;
+  a.attn_cluster = ntx::attn_cluster_size(cfg->n_heads, cfg->n_kv_heads, cfg->max_ctx);
   cudaStream_t s = S(stream);
   cudaError_t e = ntx::launch_sumsq(hidden, cfg->hidden, ws.stats_in, nin, s, false);
   if (e == cudaSuccess) e = ntx::launch_layer(a, s, true);
@@ -459,6 +460,7 @@ cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t*
     a.stats_down = e->stats_down + l * e->stats_stride;
     a.q = e->q; a.attn_out = e->attn_out; a.attn_part = e->attn_part; a.h1 = e->h1; a.u = e->u;
     a.pos = 0; a.pos_dev = e->params; a.n_split = e->n_split;
+    a.attn_cluster = ntx::attn_cluster_size(c.n_heads, c.n_kv_heads, c.max_ctx);
     const size_t k = computed.size();
     if (probe && k < e->probe_b.size()) {
       a.probe_begin = e->probe_b[k];
@@ -486,7 +488,10 @@ cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t*
   if (err != cudaSuccess) return err;
   err = ntx::launch_argmax_finalize(e->arg_parts, ntx::head_parts(c.vocab), e->token_state, next_token, s, pdl);
   if (err != cudaSuccess) return err;
-  e->launches = 1 + ntx::kLayerLaunches * (int)computed.size() + 2;
+  ntx::LayerArgs probe_args;
+  memset(&probe_args, 0, sizeof probe_args);
+  probe_args.attn_cluster = ntx::attn_cluster_size(c.n_heads, c.n_kv_heads, c.max_ctx);
+  e->launches = 1 + ntx::layer_launches(probe_args) * (int)computed.size() + 2;
   float* cdst = calibrate ? e->cos_int : cos_out;
   if (cdst && !computed.empty()) {
     e->launches += 1;

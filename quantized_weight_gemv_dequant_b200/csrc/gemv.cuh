@@ -37,6 +37,7 @@ constexpr int kSliceCols = 2048;      // columns per K slice (64 per lane)
 constexpr int kMaxConsumers = 15;     // consumer warps per CTA
 constexpr int kMaxTR = 32;            // rows per stage
 constexpr int kGemvThreads = (kMaxConsumers + 1) * 32;
+constexpr int kEpiTable = 128;        // float2 entries of the epilogue table (RoPE: head_dim/2)
 
 template <int QT>
 struct QTraits;
@@ -263,6 +264,148 @@ __device__ __forceinline__ float row_q6_k(const uint8_t* seg, int lane, const f3
   return r;
 }
 
+// ---------------------------------------------------------------------------
+// Q8_0 / Q4_0: exact integer block dot products.
+//
+// A lane owns two whole 32-column blocks of x.  Once per kernel it stores each
+// block in 22-bit block fixed point: X_i = rint(x_i * 2^(22-e)) with 2^e >
+// max|x| over the block (|X_i| <= 2^22; the representation error of each x_i
+// is at most 2^-23 of the block's largest |x|), split into byte limbs
+// X = L0 + 2^8 L1 + 2^16 L2 (L0, L1 unsigned, L2 signed), four columns per
+// 32-bit register.  A block's sum_i q_i X_i is then three sums of 4-way byte
+// dot products (dp4a), exact in int32, combined and scaled once in fp32:
+// d * 2^(e-22) * (2^16 A2 + 2^8 A1 + A0).  Q8_0 codes are int8 as stored;
+// Q4_0 nibbles are unsigned and the -8 offset is folded into the starting
+// value of each limb's accumulator (-8 times the block's limb sum).
+struct XFix {
+  uint32_t l0[16], l1[16], l2[16];  // block b, word k (columns 4k..4k+3) at [8b + k]
+  float xs[2];                      // 2^(e_b - 22)
+  int c0[2], c1[2], c2[2];          // -8 * sum of the block's limb bytes (Q4_0)
+};
+
+__device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
+  uint32_t d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return (int)d;
+}
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+template <class Pro>
+__device__ __forceinline__ void prep_fix(const Pro& pro, int64_t col, XFix& x) {
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 t = pro.ld(col + 32 * b + 4 * i);
+      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+    int e = m > 0.f ? ilogbf(m) + 1 : 0;
+    if (e < -100) e = -100;
+    const float up = ldexpf(1.0f, 22 - e);
+    x.xs[b] = ldexpf(1.0f, e - 22);
+    int s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t a0 = 0, a1 = 0, a2 = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int X = __float2int_rn(v[4 * k + j] * up);
+        const uint32_t b0 = (uint32_t)X & 0xFFu, b1 = ((uint32_t)X >> 8) & 0xFFu;
+        const int hi = X >> 16;  // arithmetic: in [-64, 64]
+        a0 |= b0 << (8 * j);
+        a1 |= b1 << (8 * j);
+        a2 |= ((uint32_t)hi & 0xFFu) << (8 * j);
+        s0 += (int)b0;
+        s1 += (int)b1;
+        s2 += hi;
+      }
+      x.l0[8 * b + k] = a0;
+      x.l1[8 * b + k] = a1;
+      x.l2[8 * b + k] = a2;
+    }
+    x.c0[b] = -8 * s0;
+    x.c1[b] = -8 * s1;
+    x.c2[b] = -8 * s2;
+  }
+}
+
+__device__ __forceinline__ float limbs_to_f(int a0, int a1, int a2) {
+  return fmaf((float)a2, 65536.0f, (float)a1 * 256.0f) + (float)a0;
+}
+
+// Q8_0 rows: lane l owns blocks 2l, 2l+1 (68 bytes = 17 words at offset 68 l).
+// Block 0: scale = low half of word 0, codes at bytes 2..33 (re-aligned by a
+// funnel shift); block 1: scale = high half of word 8, codes = words 9..16.
+__device__ __forceinline__ float rowfix_q8_0(const uint8_t* seg, int lane, const XFix& x) {
+  const uint32_t* wp = reinterpret_cast<const uint32_t*>(seg + lane * 68);
+  uint32_t w[17];
+#pragma unroll
+  for (int i = 0; i < 17; ++i) w[i] = wp[i];
+  float r = 0.f;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    int a0 = 0, a1 = 0, a2 = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t q = b == 0 ? __funnelshift_r(w[k], w[k + 1], 16) : w[9 + k];
+      a0 = dp4a_su(q, x.l0[8 * b + k], a0);
+      a1 = dp4a_su(q, x.l1[8 * b + k], a1);
+      a2 = dp4a_ss(q, x.l2[8 * b + k], a2);
+    }
+    const float d = half_bits_to_float(b == 0 ? w[0] : (w[8] >> 16));
+    r = fmaf(d * x.xs[b], limbs_to_f(a0, a1, a2), r);
+  }
+  return r;
+}
+
+// Q4_0 rows: lane l owns blocks 2l, 2l+1 (36 bytes = 9 words at offset 36 l).
+// Block 0: scale = low half of word 0, nibble bytes 2..17 (re-aligned);
+// block 1: scale = high half of word 4, nibble bytes = words 5..8.  Nibble
+// word k: low nibbles are elements 4k..4k+3, high nibbles 16+4k..16+4k+3.
+__device__ __forceinline__ float rowfix_q4_0(const uint8_t* seg, int lane, const XFix& x) {
+  const uint32_t* wp = reinterpret_cast<const uint32_t*>(seg + lane * 36);
+  uint32_t w[9];
+#pragma unroll
+  for (int i = 0; i < 9; ++i) w[i] = wp[i];
+  float r = 0.f;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    int a0 = x.c0[b], a1 = x.c1[b], a2 = x.c2[b];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t n = b == 0 ? __funnelshift_r(w[k], w[k + 1], 16) : w[5 + k];
+      const uint32_t lo = n & 0x0F0F0F0Fu, hi = (n >> 4) & 0x0F0F0F0Fu;
+      a0 = dp4a_uu(lo, x.l0[8 * b + k], a0);
+      a0 = dp4a_uu(hi, x.l0[8 * b + 4 + k], a0);
+      a1 = dp4a_uu(lo, x.l1[8 * b + k], a1);
+      a1 = dp4a_uu(hi, x.l1[8 * b + 4 + k], a1);
+      a2 = dp4a_us(lo, x.l2[8 * b + k], a2);
+      a2 = dp4a_us(hi, x.l2[8 * b + 4 + k], a2);
+    }
+    const float d = half_bits_to_float(b == 0 ? w[0] : (w[4] >> 16));
+    r = fmaf(d * x.xs[b], limbs_to_f(a0, a1, a2), r);
+  }
+  return r;
+}
+
 // Columns of x a lane owns within its slice (relative to the slice start):
 // Q8_0/Q4_0: 64 l + i;  Q6_K: 512 P + 256 odd + 128 h + 32 g + 4 j + t.
 template <int QT>
@@ -296,29 +439,57 @@ __device__ __forceinline__ void load_x_slice(const Pro& pro, int64_t c0, int lan
   }
 }
 
+// The x registers a consumer lane keeps for the whole kernel, per format.
 template <int QT>
-__device__ __forceinline__ float row_dot(const uint8_t* seg, int lane, const f32x2* xr) {
-  if constexpr (QT == QT_Q8_0) return row_q8_0(seg, lane, xr);
-  else if constexpr (QT == QT_Q4_0) return row_q4_0(seg, lane, xr);
-  else return row_q6_k(seg, lane, xr);
-}
+struct XRegs {
+  XFix x;
+  template <class Pro>
+  __device__ __forceinline__ void load(const Pro& pro, int64_t c0, int lane) {
+    prep_fix(pro, c0 + 64 * lane, x);
+  }
+  __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const {
+    if constexpr (QT == QT_Q8_0) return rowfix_q8_0(seg, lane, x);
+    else return rowfix_q4_0(seg, lane, x);
+  }
+};
+template <>
+struct XRegs<QT_Q6_K> {
+  f32x2 x2[32];
+  template <class Pro>
+  __device__ __forceinline__ void load(const Pro& pro, int64_t c0, int lane) {
+    load_x_slice<QT_Q6_K>(pro, c0, lane, x2);
+  }
+  __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const { return row_q6_k(seg, lane, x2); }
+};
 
 // ------------------------------------------------------------- epilogues
-// Run by the producer warp.  apply(r, a, b): kAlign == 1 -> row r has value
-// a; kAlign == 2 -> rows r (even) and r + 1 have values a and b.  Per-lane
-// statistics are reduced over the warp in finish() into
-// parts[blockIdx.x * 4 + k].
+// Run by the producer warp, off the ring-refill path:
+//   init(esm, lane)        once, after the programmatic-launch wait (tables);
+//   preload(rs, nr, lane)  loads the global inputs of the next stage's rows
+//                          into registers (latency hidden by the next wait);
+//   rotate()               makes the preloaded values current;
+//   apply(r, a, b)         kAlign == 1: row r has value a; kAlign == 2: rows r
+//                          (even) and r + 1 have values a and b;  lane k of
+//                          the producer handles row (pair) k of the stage;
+//   finish(lane)           per-lane statistics reduced over the warp into
+//                          parts[blockIdx.x * 4 + k].
 struct EpiStore {
   float* y;
   const float* resid;
+  float nres, cres;
   static constexpr int kAlign = 1;
-  __device__ __forceinline__ void init() {}
-  __device__ __forceinline__ void apply(int64_t r, float a, float) { y[r] = resid ? a + resid[r] : a; }
+  __device__ __forceinline__ void init(float2*, int) {}
+  __device__ __forceinline__ void preload(int64_t rs, int nr, int lane) {
+    if (resid && lane < nr) nres = resid[rs + lane];
+  }
+  __device__ __forceinline__ void rotate() { cres = nres; }
+  __device__ __forceinline__ void apply(int64_t r, float a, float) { y[r] = resid ? a + cres : a; }
   __device__ __forceinline__ void finish(int) {}
 };
 
-// QKV with RoPE (adjacent pairs, angle pos * theta^(-2i/D) formed in fp64)
-// and the k, v store into the fp16 caches at row pos.
+// QKV with RoPE (adjacent pairs, angle pos * theta^(-2i/D), cos and sin formed
+// in fp64 once per kernel into a shared table) and the k, v store into the
+// fp16 caches at row pos.
 struct EpiQKV {
   float* q_out;
   uint16_t* k_cache;
@@ -328,24 +499,31 @@ struct EpiQKV {
   int64_t nq, nkv;
   int head_dim, max_ctx;
   float theta;
+  const float2* cs;  // shared: (cos, sin) of pair i
   static constexpr int kAlign = 2;
-  __device__ __forceinline__ void init() {
+  __device__ __forceinline__ void init(float2* esm, int lane) {
     if (pos_dev) pos = *pos_dev;
+    for (int i = lane; i < head_dim / 2; i += 32) {
+      const double inv_freq = pow((double)theta, -2.0 * (double)i / (double)head_dim);
+      double sn, cn;
+      sincos((double)pos * inv_freq, &sn, &cn);
+      esm[i] = make_float2((float)cn, (float)sn);
+    }
+    cs = esm;
+    __syncwarp();
   }
+  __device__ __forceinline__ void preload(int64_t, int, int) {}
+  __device__ __forceinline__ void rotate() {}
   __device__ __forceinline__ void apply(int64_t r, float a, float b) {
     const int64_t i2 = r % head_dim;  // even index within the head
     if (r < nq + nkv) {
-      const double inv_freq = pow((double)theta, -(double)i2 / (double)head_dim);
-      double s, c;
-      sincos((double)pos * inv_freq, &s, &c);
-      const float cf = (float)c, sf = (float)s;
-      const float ra = a * cf - b * sf, rb = a * sf + b * cf;
+      const float2 t = cs[i2 >> 1];
+      const float ra = a * t.x - b * t.y, rb = a * t.y + b * t.x;
       a = ra;
       b = rb;
     }
     if (r < nq) {
-      q_out[r] = a;
-      q_out[r + 1] = b;
+      *reinterpret_cast<float2*>(q_out + r) = make_float2(a, b);
     } else {
       const bool is_k = r < nq + nkv;
       const int64_t kr = is_k ? r - nq : r - nq - nkv;
@@ -362,27 +540,40 @@ struct EpiQKV {
 struct EpiSwiGLU {
   float* out;
   static constexpr int kAlign = 2;
-  __device__ __forceinline__ void init() {}
+  __device__ __forceinline__ void init(float2*, int) {}
+  __device__ __forceinline__ void preload(int64_t, int, int) {}
+  __device__ __forceinline__ void rotate() {}
   __device__ __forceinline__ void apply(int64_t r, float g, float u) { out[r >> 1] = (g / (1.0f + expf(-g))) * u; }
   __device__ __forceinline__ void finish(int) {}
 };
 
 // out = v + resid; statistics sum(out^2), sum(hc out), sum(hc^2) where hc is
-// the layer input (read before `out` overwrites it when they alias).
+// the layer input.  hc is read one stage ahead of the store to out, so `out`
+// may alias hc (each row is read before it is overwritten).
 struct EpiResid {
   float* out;
   const float* resid;
   const float* hc;  // nullable
   float* parts;     // [gridDim.x][4]
   float st0, st1, st2;
+  float nres, nhc, cres, chc;
   static constexpr int kAlign = 1;
-  __device__ __forceinline__ void init() { st0 = st1 = st2 = 0.f; }
+  __device__ __forceinline__ void init(float2*, int) { st0 = st1 = st2 = 0.f; }
+  __device__ __forceinline__ void preload(int64_t rs, int nr, int lane) {
+    if (lane < nr) {
+      nres = resid[rs + lane];
+      nhc = hc ? hc[rs + lane] : 0.f;
+    }
+  }
+  __device__ __forceinline__ void rotate() {
+    cres = nres;
+    chc = nhc;
+  }
   __device__ __forceinline__ void apply(int64_t r, float a, float) {
-    const float o = a + resid[r];
+    const float o = a + cres;
     if (hc) {
-      const float h = hc[r];
-      st1 = fmaf(h, o, st1);
-      st2 = fmaf(h, h, st2);
+      st1 = fmaf(chc, o, st1);
+      st2 = fmaf(chc, chc, st2);
     }
     st0 = fmaf(o, o, st0);
     out[r] = o;
@@ -405,10 +596,12 @@ struct EpiArgmax {
   float best;
   int64_t besti;
   static constexpr int kAlign = 1;
-  __device__ __forceinline__ void init() {
+  __device__ __forceinline__ void init(float2*, int) {
     best = -INFINITY;
     besti = INT64_MAX;
   }
+  __device__ __forceinline__ void preload(int64_t, int, int) {}
+  __device__ __forceinline__ void rotate() {}
   __device__ __forceinline__ void apply(int64_t r, float a, float) {
     if (y) y[r] = a;
     if (a > best || (a == best && r < besti)) { best = a; besti = r; }
@@ -456,7 +649,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.S * p.stage_bytes);
   uint64_t* empty = full + p.S;
   float* red = reinterpret_cast<float*>(empty + p.S);  // [S][TR][n_slices]
-  int* abort_flag = reinterpret_cast<int*>(red + p.S * p.TR * p.n_slices);
+  float2* esm = reinterpret_cast<float2*>(red + p.S * p.TR * p.n_slices);  // epilogue table, 128 entries
+  int* abort_flag = reinterpret_cast<int*>(esm + kEpiTable);
 
   // rows of this CTA, in units of Epi::kAlign rows
   const int64_t A = Epi::kAlign;
@@ -493,33 +687,33 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     for (int i = 0; i < pre; ++i) issue(i, i);
     pdl_launch_dependents();
     pdl_wait();
-    epi.init();
+    epi.init(esm, lane);
+    if (n_stages > 0) epi.preload(r0, (int)min64(p.TR, r1 - r0), lane);
     int i = 0, s = 0;
     uint32_t ph = 0;
     for (; i < n_stages; ++i) {
       if (!warp_wait(&empty[s], ph)) break;
       const int64_t rs = r0 + (int64_t)i * p.TR;
       const int nr = (int)min64(p.TR, r1 - rs);
+      // 1. this stage's row totals (fixed slice order) into registers
       const float* rd = red + (size_t)s * p.TR * p.n_slices;
-      if constexpr (Epi::kAlign == 1) {
-        if (lane < nr) {
-          float v = 0.f;
-          for (int c = 0; c < p.n_slices; ++c) v += rd[lane * p.n_slices + c];
-          epi.apply(rs + lane, v, 0.f);
-        }
-      } else {
-        if (2 * lane < nr) {
-          float a = 0.f, b = 0.f;
-          for (int c = 0; c < p.n_slices; ++c) {
-            a += rd[(2 * lane) * p.n_slices + c];
-            b += rd[(2 * lane + 1) * p.n_slices + c];
-          }
-          epi.apply(rs + 2 * lane, a, b);
+      float a = 0.f, b = 0.f;
+      const int row_a = Epi::kAlign == 1 ? lane : 2 * lane;
+      const bool mine = row_a < nr;
+      if (mine) {
+        for (int c = 0; c < p.n_slices; ++c) {
+          a += rd[row_a * p.n_slices + c];
+          if (Epi::kAlign == 2) b += rd[(row_a + 1) * p.n_slices + c];
         }
       }
       __syncwarp();
+      // 2. refill the slot before any global-memory epilogue work
       if (i + p.S < n_stages) issue(i + p.S, s);
       if (++s == p.S) { s = 0; ph ^= 1u; }
+      // 3. epilogue; the next stage's inputs are requested first
+      epi.rotate();
+      if (i + 1 < n_stages) epi.preload(rs + p.TR, (int)min64(p.TR, r1 - rs - p.TR), lane);
+      if (mine) epi.apply(rs + row_a, a, b);
     }
     if (i < n_stages) {
       // A wait ran out: record it, stop the consumers, and let the copies
@@ -544,8 +738,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     const int ucols = (int)min64(kSliceCols, K - c0);
     const bool active = lane_active<QT>(lane, ucols);
     pro.setup(lane);
-    f32x2 xr[32];
-    if (active) load_x_slice<QT>(pro, c0, lane, xr);
+    XRegs<QT> xr;
+    if (active) xr.load(pro, c0, lane);
     int s = 0;
     uint32_t ph = 0;
     for (int i = 0; i < n_stages; ++i) {
@@ -558,7 +752,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       const uint8_t* st = ring + (size_t)s * p.stage_bytes + (size_t)c * QTraits<QT>::SEG;
       float* rd = red + (size_t)s * p.TR * p.n_slices;
       for (int r = g; r < nr; r += p.n_rg) {
-        float v = active ? row_dot<QT>(st + (size_t)r * p.row_bytes, lane, xr) : 0.f;
+        float v = active ? xr.dot(st + (size_t)r * p.row_bytes, lane) : 0.f;
         v = warp_sum(v);
         if (lane == 0) rd[r * p.n_slices + c] = v;
       }
@@ -603,7 +797,7 @@ inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget)
 }
 
 inline size_t gemv_smem_bytes(const GemvPlan& p) {
-  return (size_t)p.S * p.stage_bytes + (size_t)p.S * 16 + (size_t)p.S * p.TR * p.n_slices * 4 + 16;
+  return (size_t)p.S * p.stage_bytes + (size_t)p.S * 16 + (size_t)p.S * p.TR * p.n_slices * 4 + kEpiTable * 8 + 16;
 }
 
 // ------------------------------------------------------------- generic path

@@ -194,6 +194,72 @@ cudaError_t launch_attn(const float* q, const uint16_t* kc, const uint16_t* vc, 
   return launch_k(attn_combine_kernel, dim3(Hq), dim3(kAttnD), 0, s, pdl, (const float*)part, out, n_split);
 }
 
+template <int G>
+static cudaError_t attn_cluster_g(const float* q, const uint16_t* kc, const uint16_t* vc, float* out, int Hkv,
+                                  int n_ctx, const int* pos_dev, int max_ctx, int cs, cudaStream_t s, bool pdl) {
+  static unsigned long long done = 0;
+  auto kern = attn_cluster_kernel<G>;
+  const int d = current_device();
+  if (!(done & (1ull << d))) {
+    std::lock_guard<std::mutex> g(g_mu);
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    done |= 1ull << d;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, Hkv);
+  cfg.blockDim = dim3(kAttnWarps * 32);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  int na = 1;
+  if (pdl) {
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    na = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, q, kc, vc, out, n_ctx, pos_dev, max_ctx);
+}
+
+int attn_cluster_size(int Hq, int Hkv, int n_ctx_max) {
+  const int need = (n_ctx_max + kAttnMaxChunk - 1) / kAttnMaxChunk;
+  if (need > 16 || Hkv <= 0 || Hq % Hkv) return 0;
+  int cs = need > 8 ? 16 : 8;
+  // largest cluster the device can co-schedule for this kernel shape
+  static int cap[kMaxDevices];
+  const int d = current_device();
+  if (d >= 0 && d < kMaxDevices && cap[d] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, Hkv);
+    cfg.blockDim = dim3(kAttnWarps * 32);
+    int v = 0;
+    cudaFuncSetAttribute(attn_cluster_kernel<8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (cudaOccupancyMaxPotentialClusterSize(&v, attn_cluster_kernel<8>, &cfg) != cudaSuccess || v < 1) v = 8;
+    cudaGetLastError();
+    cap[d] = v;
+  }
+  const int c = (d >= 0 && d < kMaxDevices) ? cap[d] : 8;
+  if (cs > c) cs = c >= 8 ? 8 : c;
+  if ((int64_t)cs * kAttnMaxChunk < n_ctx_max) return 0;
+  return cs;
+}
+
+cudaError_t launch_attn_cluster(const float* q, const uint16_t* kc, const uint16_t* vc, float* out, int Hq, int Hkv,
+                                int n_ctx, const int* pos_dev, int max_ctx, int cs, cudaStream_t s, bool pdl) {
+  switch (Hq / Hkv) {
+    case 1: return attn_cluster_g<1>(q, kc, vc, out, Hkv, n_ctx, pos_dev, max_ctx, cs, s, pdl);
+    case 2: return attn_cluster_g<2>(q, kc, vc, out, Hkv, n_ctx, pos_dev, max_ctx, cs, s, pdl);
+    case 4: return attn_cluster_g<4>(q, kc, vc, out, Hkv, n_ctx, pos_dev, max_ctx, cs, s, pdl);
+    case 8: return attn_cluster_g<8>(q, kc, vc, out, Hkv, n_ctx, pos_dev, max_ctx, cs, s, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 int layer_stats_parts(int64_t H) { return gemv_grid(H, 1); }
 
 template <int QT>
@@ -213,9 +279,14 @@ static cudaError_t layer_qt(const LayerArgs& a, cudaStream_t s, bool pdl) {
     e = gemv_tma<QT>(MapQKV{a.wq, a.wk, a.wv, rbH, nq, nkv}, pro, epi, M, a.H, gemv_grid(M, 2), s, pdl);
     if (e != cudaSuccess) return e;
   }
-  // 2. split-KV attention + combine
-  e = launch_attn(a.q, a.k_cache, a.v_cache, a.attn_out, a.attn_part, (int)a.Hq, (int)a.Hkv, a.pos + 1, a.pos_dev,
-                  a.max_ctx, a.n_split, s, pdl);
+  // 2. split-KV attention: one cluster per KV head (partials merged through
+  //    distributed shared memory), or split + combine kernels for long contexts
+  if (a.attn_cluster > 0)
+    e = launch_attn_cluster(a.q, a.k_cache, a.v_cache, a.attn_out, (int)a.Hq, (int)a.Hkv, a.pos + 1, a.pos_dev,
+                            a.max_ctx, a.attn_cluster, s, pdl);
+  else
+    e = launch_attn(a.q, a.k_cache, a.v_cache, a.attn_out, a.attn_part, (int)a.Hq, (int)a.Hkv, a.pos + 1, a.pos_dev,
+                    a.max_ctx, a.n_split, s, pdl);
   if (e != cudaSuccess) return e;
   // 3. O projection + residual: h1 = h + Wo a   (statistics: sum h1^2)
   {

@@ -43,10 +43,16 @@ struct LayerArgs {
   float *q, *attn_out, *attn_part, *h1, *u;
   int pos;             // used when pos_dev is null
   const int* pos_dev;  // device position word (engine)
-  int n_split;
+  int n_split;       // split + combine attention (when attn_cluster == 0)
+  int attn_cluster;  // CTAs per KV-head cluster of the fused attention, 0 = split + combine
   cudaEvent_t probe_begin, probe_end;  // recorded around the gate/up GEMV when set
 };
-constexpr int kLayerLaunches = 6;  // kernels one launch_layer() enqueues
+// Kernels one launch_layer() enqueues.
+inline int layer_launches(const LayerArgs& a) { return a.attn_cluster > 0 ? 5 : 6; }
+// Cluster size for the fused attention over contexts up to n_ctx_max (0: use split + combine).
+int attn_cluster_size(int Hq, int Hkv, int n_ctx_max);
+cudaError_t launch_attn_cluster(const float* q, const uint16_t* kc, const uint16_t* vc, float* out, int Hq, int Hkv,
+                                int n_ctx, const int* pos_dev, int max_ctx, int cs, cudaStream_t s, bool pdl);
 cudaError_t launch_layer(const LayerArgs& a, cudaStream_t s, bool pdl);
 // Number of statistics partials the down projection of a layer writes.
 int layer_stats_parts(int64_t H);

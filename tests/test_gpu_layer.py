@@ -99,6 +99,13 @@ def test_layer_small_q6_k(pos):
     run_layer_case(SMALL_Q6K, ntx.NTX_Q6_K, 3000 + pos, pos, 512)
 
 
+@pytest.mark.parametrize("pos", [7, 4100, 4499])
+def test_layer_long_context_split_combine_path(pos):
+    """A cache longer than 16 clusters x 256 positions takes the split +
+    combine attention kernels instead of the cluster-fused one."""
+    run_layer_case(SMALL, ntx.NTX_Q8_0, 4000 + pos, pos, 4500)
+
+
 def test_layer_config_3_llama8b_q8_0():
     """Config 3: the 8B-shaped Q8_0 layer, 1024 prior positions, token at 1024.
     Also checks that the device generator writes this layer bit-identically."""
