@@ -21,14 +21,16 @@ def _newest_input():
     return max(os.path.getmtime(f) for f in files)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(SO) and os.path.getmtime(SO) >= _newest_input():
-        return SO
+def build(force: bool = False, verbose: bool = False, out: str = SO, defines=()) -> str:
+    """Compile libntx.so (or a variant at `out` with extra -D definitions)."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= _newest_input():
+        return out
     objs = []
     procs = []
     for src in SOURCES:
-        obj = os.path.join(CSRC, src.replace(".cu", ".o"))
-        cmd = [NVCC, *ARCH, *FLAGS, "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o", obj]
+        obj = out + "." + src.replace(".cu", ".o")
+        cmd = [NVCC, *ARCH, *FLAGS, *["-D" + d for d in defines], "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o",
+               obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         procs.append(subprocess.Popen(cmd))
@@ -36,12 +38,12 @@ def build(force: bool = False, verbose: bool = False) -> str:
     for p in procs:
         if p.wait() != 0:
             raise RuntimeError("nvcc failed")
-    tmp = SO + ".tmp"
+    tmp = out + ".tmp"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs])
-    os.replace(tmp, SO)
+    os.replace(tmp, out)
     for o in objs:
         os.remove(o)
-    return SO
+    return out
 
 
 if __name__ == "__main__":

@@ -33,9 +33,16 @@ namespace ntx {
 
 constexpr int QT_Q4_0 = 2, QT_Q8_0 = 8, QT_Q6_K = 14;
 
-constexpr int kSliceCols = 2048;      // columns per K slice (64 per lane)
-constexpr int kMaxConsumers = 15;     // consumer warps per CTA
-constexpr int kMaxTR = 32;            // rows per stage
+#ifndef NTX_GEMV_MAX_CONSUMERS
+#define NTX_GEMV_MAX_CONSUMERS 15
+#endif
+#ifndef NTX_GEMV_STAGE_BYTES
+#define NTX_GEMV_STAGE_BYTES 34816
+#endif
+constexpr int kSliceCols = 2048;                         // columns per K slice (64 per lane)
+constexpr int kMaxConsumers = NTX_GEMV_MAX_CONSUMERS;    // consumer warps per CTA
+constexpr int kMaxTR = 32;                               // rows per stage
+constexpr int kStageTarget = NTX_GEMV_STAGE_BYTES;       // bytes a stage aims at
 constexpr int kGemvThreads = (kMaxConsumers + 1) * 32;
 constexpr int kEpiTable = 128;        // float2 entries of the epilogue table (RoPE: head_dim/2)
 
@@ -771,7 +778,7 @@ inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget)
   const int be = qtype == QT_Q6_K ? 256 : 32, bb = qtype == QT_Q6_K ? 210 : (qtype == QT_Q8_0 ? 34 : 18);
   p.row_bytes = (int)(K / be * bb);
   p.n_slices = (int)((K + kSliceCols - 1) / kSliceCols);
-  int trmax = 34816 / p.row_bytes;
+  int trmax = kStageTarget / p.row_bytes;
   if (trmax < 1) trmax = 1;
   if (trmax > kMaxTR) trmax = kMaxTR;
   int n_rg = kMaxConsumers / p.n_slices;

@@ -76,7 +76,10 @@ int grid_1d(int64_t n, int threads, int cap) {
   return g < 1 ? 1 : (int)g;
 }
 
-constexpr int kRingBudget = 150 * 1024;   // shared memory for the weight ring
+#ifndef NTX_GEMV_RING_BYTES
+#define NTX_GEMV_RING_BYTES (150 * 1024)
+#endif
+constexpr int kRingBudget = NTX_GEMV_RING_BYTES;  // shared memory for the weight ring
 constexpr int kSmemMax = 200 * 1024;      // attribute ceiling for every GEMV instantiation
 
 template <int QT, class Map, class Pro, class Epi>
