@@ -138,6 +138,23 @@ NTX_API int ntx_attn_decode(const float* q, const uint16_t* k_cache, const uint1
                     int n_kv_heads, int head_dim, int n_ctx, int max_ctx, void* workspace, size_t ws_bytes,
                     void* stream);
 
+/* ntx_attn_decode without a workspace (the pages have no counterpart: this is
+ * a convenience of this library).  Same computation, arguments, limits and
+ * results as ntx_attn_decode, but the per-split partials live in a 2 MiB
+ * static device array inside libntx, so the call allocates nothing and takes
+ * no scratch buffer -- for callers that cannot provide one: hosts whose device
+ * memory is owned by another allocator with a fixed budget, C programs with no
+ * allocator on that path, latency-critical threads that must not take an
+ * allocator's lock.  Limit: n_q_heads x (attention splits) x 130 floats <=
+ * 524288, NTX_ERR_NOMEM beyond it (on a 148-SM B200 with 8 KV heads: up to
+ * 32256 positions at 32 query heads, 16128 at 64).  The first call on
+ * a device looks up the array's address (cudaGetSymbolAddress); make that
+ * first call before any stream capture.  Every GPU that loads libntx holds the
+ * array until exit, all calls share it and it keeps the last call's contents:
+ * calls that overlap on the GPU (e.g. on two streams) race. */
+NTX_API int ntx_attn_decode_static(const float* q, const uint16_t* k_cache, const uint16_t* v_cache, float* out,
+                                   int n_q_heads, int n_kv_heads, int head_dim, int n_ctx, int max_ctx, void* stream);
+
 /* SwiGLU out_i = silu(gate_i) up_i, silu(z) = z / (1 + e^-z) ([README]
  * 主な機能: SwiGLU).  Device fp32[n] each; out may alias either input. */
 NTX_API int ntx_swiglu(const float* gate, const float* up, float* out, int64_t n, void* stream);

@@ -37,7 +37,7 @@ EXPORTS = (
     "ntx_dequant", "ntx_gemv_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_workspace_bytes", "ntx_attn_decode",
     "ntx_swiglu", "ntx_layer_layout", "ntx_layer_workspace_bytes", "ntx_decode_layer", "ntx_engine_workspace_bytes",
     "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
-    "ntx_engine_launches_per_step",
+    "ntx_engine_launches_per_step", "ntx_attn_decode_static",
 )
 
 
@@ -97,6 +97,7 @@ def lib():
             "ntx_engine_destroy": ([vp], None),
             "ntx_engine_set_probe": ([vp, vp, vp, i32], i32),
             "ntx_engine_launches_per_step": ([vp], i32),
+            "ntx_attn_decode_static": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -179,6 +180,12 @@ def ntx_attn_decode(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, n
                     stream=None):
     _check(lib().ntx_attn_decode(_p(q), _p(k_cache), _p(v_cache), _p(out), n_q_heads, n_kv_heads, head_dim, n_ctx,
                                  max_ctx, _p(workspace), ws_bytes, _s(stream)))
+
+
+def ntx_attn_decode_static(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, n_ctx, max_ctx, stream=None):
+    """ntx_attn_decode without a workspace (partials in libntx's static device array)."""
+    _check(lib().ntx_attn_decode_static(_p(q), _p(k_cache), _p(v_cache), _p(out), n_q_heads, n_kv_heads, head_dim,
+                                        n_ctx, max_ctx, _s(stream)))
 
 
 def ntx_swiglu(gate, up, out, n, stream=None):

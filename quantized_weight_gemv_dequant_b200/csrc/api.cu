@@ -108,6 +108,11 @@ uint64_t carve_layer(const ntx_model_config* c, int n_split, uint8_t* base, Laye
 
 }  // namespace
 
+namespace ntx {
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+int record_cuda_error(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+}  // namespace ntx
+
 // ======================================================================
 extern "C" {
 

@@ -75,4 +75,8 @@ cudaError_t launch_cos_finalize(const float* stats, int nparts, const int* layer
 
 int read_device_status(int* code);
 
+// Record a failure for ntx_last_error() on the calling thread; returns code.
+int record_error(int code, const char* msg);
+int record_cuda_error(cudaError_t e, const char* what);
+
 }  // namespace ntx
