@@ -70,6 +70,7 @@ struct GemvPlan {
   int NW;        // consumer warps = n_slices * n_rg
   int row_bytes;
   int stage_bytes;
+  int xstage_bytes;  // shared memory holding x for the lanes (16-byte multiple)
 };
 
 // ------------------------------------------------------------- row maps
@@ -122,6 +123,12 @@ struct ProRms {
     const float4 a = ldg4(h + j), b = ldg4(w + j);
     return make_float4(b.x * (a.x * r), b.y * (a.y * r), b.z * (a.z * r), b.w * (a.w * r));
   }
+};
+
+// x already staged in shared memory (fp32).
+struct ProSmem {
+  const float* x;
+  __device__ __forceinline__ float4 ld(int64_t j) const { return *reinterpret_cast<const float4*>(x + j); }
 };
 
 // ------------------------------------------------------------- decoders
@@ -311,49 +318,6 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
   return d;
 }
 
-template <class Pro>
-__device__ __forceinline__ void prep_fix(const Pro& pro, int64_t col, XFix& x) {
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 t = pro.ld(col + 32 * b + 4 * i);
-      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
-    }
-    float m = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
-    int e = m > 0.f ? ilogbf(m) + 1 : 0;
-    if (e < -100) e = -100;
-    const float up = ldexpf(1.0f, 22 - e);
-    x.xs[b] = ldexpf(1.0f, e - 22);
-    int s0 = 0, s1 = 0, s2 = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      uint32_t a0 = 0, a1 = 0, a2 = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int X = __float2int_rn(v[4 * k + j] * up);
-        const uint32_t b0 = (uint32_t)X & 0xFFu, b1 = ((uint32_t)X >> 8) & 0xFFu;
-        const int hi = X >> 16;  // arithmetic: in [-64, 64]
-        a0 |= b0 << (8 * j);
-        a1 |= b1 << (8 * j);
-        a2 |= ((uint32_t)hi & 0xFFu) << (8 * j);
-        s0 += (int)b0;
-        s1 += (int)b1;
-        s2 += hi;
-      }
-      x.l0[8 * b + k] = a0;
-      x.l1[8 * b + k] = a1;
-      x.l2[8 * b + k] = a2;
-    }
-    x.c0[b] = -8 * s0;
-    x.c1[b] = -8 * s1;
-    x.c2[b] = -8 * s2;
-  }
-}
-
 __device__ __forceinline__ float limbs_to_f(int a0, int a1, int a2) {
   return fmaf((float)a2, 65536.0f, (float)a1 * 256.0f) + (float)a0;
 }
@@ -421,27 +385,131 @@ __device__ __forceinline__ bool lane_active(int lane, int ucols) {
   else return 2 * lane < ucols / 32;
 }
 
+// The 64 columns of a Q6_K slice a lane keeps, as fp32 pairs.
+template <class Pro>
+__device__ __forceinline__ void load_x_slice_q6_k(const Pro& pro, int64_t c0, int lane, f32x2* x2) {
+  const int pp = lane >> 4, h = (lane >> 3) & 1, j = lane & 7;
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+    for (int odd = 0; odd < 2; ++odd)
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float4 v = pro.ld(c0 + 512 * (pp + 2 * pass) + 256 * odd + 128 * h + 32 * g + 4 * j);
+        f32x2* o = x2 + 16 * pass + 8 * odd + 2 * g;
+        o[0] = pack2(v.x, v.y);
+        o[1] = pack2(v.z, v.w);
+      }
+}
+
+// ---------------------------------------------------------------------------
+// x staging: once per CTA, after the producer of x has finished, the consumer
+// warps read x with coalesced float4 loads (128 columns per warp and load,
+// eight loads in flight per lane) and leave it in shared memory in the form
+// the lanes need; after a named barrier among the consumer warps each lane
+// copies its own part into registers.
+//   Q8_0 / Q4_0 (fixed point, see XFix): the 8 lanes holding a 32-column
+//     block take its max|x| with shuffles; each lane turns its 4 columns into
+//     one 32-bit word per limb, stored at wd[(j*16 + k) * NP + c*32 + l]
+//     (limb j, word k of lane l of slice c; NP = 32 * slices + 2, the pad
+//     making the stores of a warp hit 32 distinct banks); the block scale
+//     2^(e-22) goes to sc[B] and the Q4_0 offsets -8 * sum(limb j) to
+//     cr[3B + j].
+//   Q6_K: x as fp32 in xf[K].
+struct XStage {
+  uint32_t* wd;
+  float* sc;
+  int* cr;
+  float* xf;
+  int np;
+};
+
+__host__ __device__ inline size_t xstage_bytes(int qtype, int64_t K) {
+  const int64_t nslices = (K + kSliceCols - 1) / kSliceCols;
+  if (qtype == QT_Q6_K) return (size_t)K * 4;
+  return (size_t)3 * 16 * (32 * nslices + 2) * 4 + (size_t)(K / 32) * 4 + (size_t)(K / 32) * 12;
+}
+
+__device__ __forceinline__ XStage xstage_at(uint8_t* base, int64_t K) {
+  XStage x;
+  const int64_t nslices = (K + kSliceCols - 1) / kSliceCols;
+  x.np = (int)(32 * nslices + 2);
+  x.wd = reinterpret_cast<uint32_t*>(base);
+  x.sc = reinterpret_cast<float*>(base + (size_t)3 * 16 * x.np * 4);
+  x.cr = reinterpret_cast<int*>(x.sc + K / 32);
+  x.xf = reinterpret_cast<float*>(base);
+  return x;
+}
+
+__device__ __forceinline__ float group8_max(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+}
+__device__ __forceinline__ int group8_sum(int v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  return v + __shfl_xor_sync(0xffffffffu, v, 4);
+}
+
+// K is a multiple of 256 on every path that stages x.
 template <int QT, class Pro>
-__device__ __forceinline__ void load_x_slice(const Pro& pro, int64_t c0, int lane, f32x2* x2) {
-  if constexpr (QT == QT_Q6_K) {
-    const int pp = lane >> 4, h = (lane >> 3) & 1, j = lane & 7;
+__device__ __forceinline__ void stage_x(const Pro& pro, int64_t K, const XStage& xs, int cw, int NW, int lane) {
+  constexpr int kBatch = 8;
+  const int nchunk = (int)(K / 128);
+  for (int ch0 = cw; ch0 < nchunk; ch0 += kBatch * NW) {
+    float4 v[kBatch];
 #pragma unroll
-    for (int pass = 0; pass < 2; ++pass)
+    for (int b = 0; b < kBatch; ++b) {
+      const int ch = ch0 + b * NW;
+      v[b] = ch < nchunk ? pro.ld((int64_t)ch * 128 + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
-      for (int odd = 0; odd < 2; ++odd)
+    for (int b = 0; b < kBatch; ++b) {
+      const int ch = ch0 + b * NW;
+      if (ch >= nchunk) break;  // uniform across the warp
+      const int64_t col = (int64_t)ch * 128 + 4 * lane;
+      if constexpr (QT == QT_Q6_K) {
+        *reinterpret_cast<float4*>(xs.xf + col) = v[b];
+      } else {
+        const float m = group8_max(fmaxf(fmaxf(fabsf(v[b].x), fabsf(v[b].y)), fmaxf(fabsf(v[b].z), fabsf(v[b].w))));
+        int e = m > 0.f ? ilogbf(m) + 1 : 0;
+        if (e < -100) e = -100;
+        const float up = ldexpf(1.0f, 22 - e);
+        const int X[4] = {__float2int_rn(v[b].x * up), __float2int_rn(v[b].y * up), __float2int_rn(v[b].z * up),
+                          __float2int_rn(v[b].w * up)};
+        uint32_t w0 = 0, w1 = 0, w2 = 0;
+        int s0 = 0, s1 = 0, s2 = 0;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float4 v = pro.ld(c0 + 512 * (pp + 2 * pass) + 256 * odd + 128 * h + 32 * g + 4 * j);
-          f32x2* o = x2 + 16 * pass + 8 * odd + 2 * g;
-          o[0] = pack2(v.x, v.y);
-          o[1] = pack2(v.z, v.w);
+        for (int t = 0; t < 4; ++t) {
+          const uint32_t b0 = (uint32_t)X[t] & 0xFFu, b1 = ((uint32_t)X[t] >> 8) & 0xFFu;
+          const int hi = X[t] >> 16;  // arithmetic: in [-64, 64]
+          w0 |= b0 << (8 * t);
+          w1 |= b1 << (8 * t);
+          w2 |= ((uint32_t)hi & 0xFFu) << (8 * t);
+          s0 += (int)b0;
+          s1 += (int)b1;
+          s2 += hi;
         }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float4 v = pro.ld(c0 + 64 * lane + 4 * i);
-      x2[2 * i] = pack2(v.x, v.y);
-      x2[2 * i + 1] = pack2(v.z, v.w);
+        const int c = (int)(col / kSliceCols), u = (int)(col % kSliceCols);
+        const int l = u / 64, k = (u % 64) / 4;
+        const int wi = k * xs.np + c * 32 + l;
+        xs.wd[wi] = w0;
+        xs.wd[16 * xs.np + wi] = w1;
+        xs.wd[32 * xs.np + wi] = w2;
+        const int64_t B = col / 32;
+        if constexpr (QT == QT_Q4_0) {
+          s0 = group8_sum(s0);
+          s1 = group8_sum(s1);
+          s2 = group8_sum(s2);
+          if ((lane & 7) == 0) {
+            xs.cr[3 * B + 0] = -8 * s0;
+            xs.cr[3 * B + 1] = -8 * s1;
+            xs.cr[3 * B + 2] = -8 * s2;
+          }
+        }
+        if ((lane & 7) == 0) xs.sc[B] = ldexpf(1.0f, e - 22);
+      }
     }
   }
 }
@@ -450,9 +518,24 @@ __device__ __forceinline__ void load_x_slice(const Pro& pro, int64_t c0, int lan
 template <int QT>
 struct XRegs {
   XFix x;
-  template <class Pro>
-  __device__ __forceinline__ void load(const Pro& pro, int64_t c0, int lane) {
-    prep_fix(pro, c0 + 64 * lane, x);
+  __device__ __forceinline__ void load(const XStage& xs, int c, int lane) {
+    const int idx = c * 32 + lane;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      x.l0[k] = xs.wd[(0 * 16 + k) * xs.np + idx];
+      x.l1[k] = xs.wd[(1 * 16 + k) * xs.np + idx];
+      x.l2[k] = xs.wd[(2 * 16 + k) * xs.np + idx];
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const int B = c * 64 + 2 * lane + b;
+      x.xs[b] = xs.sc[B];
+      if constexpr (QT == QT_Q4_0) {
+        x.c0[b] = xs.cr[3 * B + 0];
+        x.c1[b] = xs.cr[3 * B + 1];
+        x.c2[b] = xs.cr[3 * B + 2];
+      }
+    }
   }
   __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const {
     if constexpr (QT == QT_Q8_0) return rowfix_q8_0(seg, lane, x);
@@ -462,9 +545,8 @@ struct XRegs {
 template <>
 struct XRegs<QT_Q6_K> {
   f32x2 x2[32];
-  template <class Pro>
-  __device__ __forceinline__ void load(const Pro& pro, int64_t c0, int lane) {
-    load_x_slice<QT_Q6_K>(pro, c0, lane, x2);
+  __device__ __forceinline__ void load(const XStage& xs, int c, int lane) {
+    load_x_slice_q6_k(ProSmem{xs.xf}, (int64_t)c * kSliceCols, lane, x2);
   }
   __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const { return row_q6_k(seg, lane, x2); }
 };
@@ -647,13 +729,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-template <int QT, class Map, class Pro, class Epi>
-__global__ void __launch_bounds__(kGemvThreads, 1)
+// MAXC: consumer warps the CTA is built for.  With MAXC <= 8 two CTAs fit on
+// one SM (registers and shared memory), so the next kernel of a
+// programmatic-launch chain can start streaming its weights while this one
+// drains.
+template <int QT, class Map, class Pro, class Epi, int MAXC>
+__global__ void __launch_bounds__((MAXC + 1) * 32, MAXC <= 8 ? 2 : 1)
     gemv_tma_kernel(Map map, Pro pro, Epi epi, int64_t M, int64_t K, GemvPlan p, int* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.S * p.stage_bytes);
+  uint8_t* xstage_base = smem + (size_t)p.S * p.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(xstage_base + p.xstage_bytes);
   uint64_t* empty = full + p.S;
   float* red = reinterpret_cast<float*>(empty + p.S);  // [S][TR][n_slices]
   float2* esm = reinterpret_cast<float2*>(red + p.S * p.TR * p.n_slices);  // epilogue table, 128 entries
@@ -745,8 +832,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     const int ucols = (int)min64(kSliceCols, K - c0);
     const bool active = lane_active<QT>(lane, ucols);
     pro.setup(lane);
+    const XStage xs = xstage_at(xstage_base, K);
+    stage_x<QT>(pro, K, xs, warp, p.NW, lane);
+    asm volatile("bar.sync 1, %0;" ::"r"(p.NW * 32) : "memory");  // consumer warps only
     XRegs<QT> xr;
-    if (active) xr.load(pro, c0, lane);
+    if (active) xr.load(xs, c, lane);
     int s = 0;
     uint32_t ph = 0;
     for (int i = 0; i < n_stages; ++i) {
@@ -773,7 +863,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 
 // Host-side plan for a GEMV over rows of row_bytes bytes.  smem budget in
 // bytes for the ring; align: 1 or 2 (rows per epilogue unit).
-inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget) {
+inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget, int max_consumers) {
   GemvPlan p;
   const int be = qtype == QT_Q6_K ? 256 : 32, bb = qtype == QT_Q6_K ? 210 : (qtype == QT_Q8_0 ? 34 : 18);
   p.row_bytes = (int)(K / be * bb);
@@ -781,7 +871,7 @@ inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget)
   int trmax = kStageTarget / p.row_bytes;
   if (trmax < 1) trmax = 1;
   if (trmax > kMaxTR) trmax = kMaxTR;
-  int n_rg = kMaxConsumers / p.n_slices;
+  int n_rg = max_consumers / p.n_slices;
   if (n_rg < 1) n_rg = 1;
   if (n_rg > trmax) n_rg = trmax;
   int tr = trmax / n_rg * n_rg;
@@ -796,6 +886,7 @@ inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget)
   p.n_rg = n_rg;
   p.NW = p.n_slices * n_rg;
   p.stage_bytes = p.TR * p.row_bytes;
+  p.xstage_bytes = (int)((xstage_bytes(qtype, K) + 15) / 16 * 16);
   int S = smem_budget / p.stage_bytes;
   if (S > 8) S = 8;
   if (S < 2) S = 2;
@@ -804,7 +895,8 @@ inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget)
 }
 
 inline size_t gemv_smem_bytes(const GemvPlan& p) {
-  return (size_t)p.S * p.stage_bytes + (size_t)p.S * 16 + (size_t)p.S * p.TR * p.n_slices * 4 + kEpiTable * 8 + 16;
+  return (size_t)p.S * p.stage_bytes + p.xstage_bytes + (size_t)p.S * 16 + (size_t)p.S * p.TR * p.n_slices * 4 +
+         kEpiTable * 8 + 16;
 }
 
 // ------------------------------------------------------------- generic path

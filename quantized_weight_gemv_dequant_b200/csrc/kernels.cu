@@ -79,18 +79,42 @@ int grid_1d(int64_t n, int threads, int cap) {
 #ifndef NTX_GEMV_RING_BYTES
 #define NTX_GEMV_RING_BYTES (150 * 1024)
 #endif
-constexpr int kRingBudget = NTX_GEMV_RING_BYTES;  // shared memory for the weight ring
-constexpr int kSmemMax = 200 * 1024;      // attribute ceiling for every GEMV instantiation
+#ifndef NTX_GEMV_RING_BYTES_PAIRED
+#define NTX_GEMV_RING_BYTES_PAIRED (100 * 1024)
+#endif
+#ifndef NTX_GEMV_PAIRED
+#define NTX_GEMV_PAIRED 0
+#endif
+constexpr int kRingBudget = NTX_GEMV_RING_BYTES;           // one CTA per SM
+constexpr int kRingBudgetPaired = NTX_GEMV_RING_BYTES_PAIRED;  // two CTAs per SM
+constexpr int kPairedConsumers = 8;
+constexpr int kSmemMax = 227 * 1024;  // attribute ceiling for every GEMV instantiation
 
-template <int QT, class Map, class Pro, class Epi>
-cudaError_t gemv_tma(Map map, Pro pro, Epi epi, int64_t M, int64_t K, int grid, cudaStream_t s, bool pdl) {
-  static unsigned long long done = 0;  // unique per <QT, Map, Pro, Epi>
-  auto kern = gemv_tma_kernel<QT, Map, Pro, Epi>;
-  const GemvPlan plan = make_gemv_plan(QT, K, Epi::kAlign, kRingBudget);
+template <int QT, int MAXC, class Map, class Pro, class Epi>
+cudaError_t gemv_tma_v(Map map, Pro pro, Epi epi, int64_t M, int64_t K, int grid, cudaStream_t s, bool pdl,
+                       int ring) {
+  static unsigned long long done = 0;  // unique per instantiation
+  auto kern = gemv_tma_kernel<QT, Map, Pro, Epi, MAXC>;
+  // the ring gives up what x staging needs beyond the per-CTA ceiling
+  const int xst = (int)((xstage_bytes(QT, K) + 15) / 16 * 16);
+  if (ring > kSmemMax - 8192 - xst) ring = kSmemMax - 8192 - xst;
+  const GemvPlan plan = make_gemv_plan(QT, K, Epi::kAlign, ring, MAXC);
   const size_t smem = gemv_smem_bytes(plan);
   cudaError_t e = ensure_smem(kern, kSmemMax, done);
   if (e != cudaSuccess) return e;
   return launch_k(kern, dim3(grid), dim3((plan.NW + 1) * 32), smem, s, pdl, map, pro, epi, M, K, plan, status_ptr());
+}
+
+// Two co-resident CTAs per SM when the K slices fit 8 consumer warps (Q8_0 and
+// Q4_0, K <= 16384); one wide CTA per SM otherwise.
+template <int QT, class Map, class Pro, class Epi>
+cudaError_t gemv_tma(Map map, Pro pro, Epi epi, int64_t M, int64_t K, int grid, cudaStream_t s, bool pdl) {
+  if constexpr (QT != QT_Q6_K && NTX_GEMV_PAIRED) {
+    const int n_slices = (int)((K + kSliceCols - 1) / kSliceCols);
+    if (n_slices <= kPairedConsumers)
+      return gemv_tma_v<QT, kPairedConsumers>(map, pro, epi, M, K, grid, s, pdl, kRingBudgetPaired);
+  }
+  return gemv_tma_v<QT, kMaxConsumers>(map, pro, epi, M, K, grid, s, pdl, kRingBudget);
 }
 
 }  // namespace
