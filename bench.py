@@ -224,31 +224,83 @@ def run_ntx(args, dist: Dist):
     ms_step = ms_total / args.steps
     value = dist.world * args.steps / (ms_total / 1e3)
 
+    persistent = launches <= 2  # one persistent kernel (+ cosine finalisation when asked)
+
+    def probe(flags, n_ev, n_steps, pos_base):
+        """Kernel-by-kernel steps with probe events; returns (durations ms, ms/step)."""
+        ev_b = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(n_steps)]
+        ev_e = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(n_steps)]
+        with torch.cuda.stream(cs):
+            for row in ev_b + ev_e:
+                for ev in row:
+                    ev.record(cs)  # creates the CUDA events
+        cs.synchronize()
+        p0_, p1_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(cs):
+            p0_.record(cs)
+            for i in range(n_steps):
+                ntx.ntx_engine_set_probe(eng, [e.cuda_event for e in ev_b[i]], [e.cuda_event for e in ev_e[i]])
+                ntx.ntx_decode_step(eng, -1, pos_of(pos_base + i), None, next_tok, flags | ntx.NTX_NO_GRAPH, None)
+            p1_.record(cs)
+            ntx.ntx_engine_set_probe(eng, [], [])
+        cs.synchronize()
+        durs = [ev_b[i][k].elapsed_time(ev_e[i][k]) for i in range(n_steps) for k in range(n_ev)]
+        return durs, p0_.elapsed_time(p1_) / n_steps
+
     # ------------------------------------------------ dominant kernel (probe)
     n_probe = min(args.steps, 24)
-    ev_b = [[torch.cuda.Event(enable_timing=True) for _ in range(L)] for _ in range(n_probe)]
-    ev_e = [[torch.cuda.Event(enable_timing=True) for _ in range(L)] for _ in range(n_probe)]
-    with torch.cuda.stream(cs):
-        for row in ev_b + ev_e:
-            for ev in row:
-                ev.record(cs)  # creates the CUDA events
-    cs.synchronize()
-    step_probe0, step_probe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(cs):
-        step_probe0.record(cs)
-        for i in range(n_probe):
-            ntx.ntx_engine_set_probe(eng, [e.cuda_event for e in ev_b[i]], [e.cuda_event for e in ev_e[i]])
-            ntx.ntx_decode_step(eng, -1, pos_of(args.warmup + args.steps + i), None, next_tok, ntx.NTX_NO_GRAPH,
-                                None)
-        step_probe1.record(cs)
-        ntx.ntx_engine_set_probe(eng, [], [])
-    cs.synchronize()
-    durs = [ev_b[i][l].elapsed_time(ev_e[i][l]) for i in range(n_probe) for l in range(L)]
-    gu_ms = statistics.mean(durs)
+    pos_base = args.warmup + args.steps
     H, F = d["hidden"], d["ffn"]
-    gu_bytes = 2 * wl.mat_bytes(qt, F, H) + 2 * 4 * H + 4 * F + 4 * 4 * 148  # weights, h1 + norm, u out, stats in
-    gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
-    probe_ms_step = step_probe0.elapsed_time(step_probe1) / n_probe
+    peak, peak_kind = measured_peaks()
+    if persistent:
+        durs, probe_ms_step = probe(0, 1, n_probe, pos_base)
+        k_ms = statistics.mean(durs)
+        n_ctx_mean = statistics.mean(pos_of(pos_base + i) + 1 for i in range(n_probe))
+        k_bytes = wl.bytes_per_token(d, qt, hqt, int(round(n_ctx_mean)))
+        roof = {"bound": "hbm", "kernel": "persistent decode-step kernel (one launch per token)",
+                "achieved": round(k_bytes / (k_ms * 1e-3) / 1e9, 1), "peak": peak, "peak_kind": peak_kind,
+                "unit": "GB/s", "frac": round(k_bytes / (k_ms * 1e-3) / 1e9 / peak, 4), "traffic": args.traffic,
+                "bytes_per_launch": k_bytes, "avg_launch_us": round(k_ms * 1e3, 3),
+                "timing": f"CUDA events on the compute stream around each of {n_probe} kernel launches "
+                          f"(uncaptured steps right after the timed region, {round(probe_ms_step, 4)} ms/step there)"}
+    pos_base += n_probe
+
+    # ------------------------------------------- the per-op kernel chain, for comparison
+    chain = None
+    if not args.no_chain:
+        n_chain = min(args.steps, 256)
+        with torch.cuda.stream(cs):
+            for i in range(3):
+                ntx.ntx_decode_step(eng, -1, pos_of(pos_base + i), None, next_tok, ntx.NTX_NO_PERSIST, None)
+        pos_base += 3
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(cs):
+            c0.record(cs)
+            for i in range(n_chain):
+                ntx.ntx_decode_step(eng, -1, pos_of(pos_base + i), None, next_tok, ntx.NTX_NO_PERSIST, None)
+            c1.record(cs)
+        cs.synchronize()
+        pos_base += n_chain
+        chain_launches = ntx.ntx_engine_launches_per_step(eng)
+        gdurs, gprobe_ms = probe(ntx.NTX_NO_PERSIST, L, n_probe, pos_base)
+        pos_base += n_probe
+        gu_ms = statistics.mean(gdurs)
+        gu_bytes = 2 * wl.mat_bytes(qt, F, H) + 2 * 4 * H + 4 * F + 4 * 4 * 148  # weights, h1 + norm, u, stats
+        chain = {"tok_s": round(n_chain / (c0.elapsed_time(c1) / 1e3), 3), "steps": n_chain,
+                 "launches_per_step": chain_launches,
+                 "gate_up_gemv": {"achieved": round(gu_bytes / (gu_ms * 1e-3) / 1e9, 1),
+                                  "frac": round(gu_bytes / (gu_ms * 1e-3) / 1e9 / peak, 4),
+                                  "bytes_per_launch": gu_bytes, "avg_launch_us": round(gu_ms * 1e3, 3),
+                                  "timing": f"CUDA events around every gate/up launch of {n_probe} kernel-by-kernel "
+                                            f"steps ({round(gprobe_ms, 4)} ms/step there)"}}
+        if not persistent:
+            roof = {"bound": "hbm", "kernel": "gate/up GEMV (RMSNorm prologue + SwiGLU epilogue)",
+                    "achieved": chain["gate_up_gemv"]["achieved"], "peak": peak, "peak_kind": peak_kind,
+                    "unit": "GB/s", "frac": chain["gate_up_gemv"]["frac"], "traffic": args.traffic,
+                    "bytes_per_launch": gu_bytes, "avg_launch_us": round(gu_ms * 1e3, 3),
+                    "timing": chain["gate_up_gemv"]["timing"]}
+    elif not persistent:
+        raise SystemExit("--no-chain needs the persistent kernel (all layers resident)")
 
     # ------------------------------------------------------------ e2e
     host_tok = torch.zeros(1, dtype=torch.int32, pin_memory=True)
@@ -259,7 +311,7 @@ def run_ntx(args, dist: Dist):
     t0 = time.perf_counter()
     with torch.cuda.stream(cs):
         for i in range(n_e2e):
-            ntx.ntx_decode_step(eng, tok, pos_of(args.warmup + args.steps + n_probe + i), None, next_tok, 0, None)
+            ntx.ntx_decode_step(eng, tok, pos_of(pos_base + i), None, next_tok, 0, None)
             host_tok.copy_(next_tok, non_blocking=True)
             cs.synchronize()
             tok = int(host_tok[0])
@@ -267,7 +319,6 @@ def run_ntx(args, dist: Dist):
     e2e_value = dist.world * n_e2e / e2e_s
 
     # ------------------------------------------------------------ GEMV sweep
-    peak, peak_kind = measured_peaks()
     gemv = [] if args.no_gemv else gemv_sweep(ntx, sg, wl, torch, peak)
 
     # ------------------------------------------------------------ CPU baseline
@@ -286,13 +337,9 @@ def run_ntx(args, dist: Dist):
                    "hidden": d["hidden"], "ffn": d["ffn"], "vocab": d["vocab"], "batch": 1,
                    "parallelism": f"replicas x{dist.world}" if dist.world > 1 else "single GPU",
                    "l2": "weights per step >> 126 MB L2 (inputs larger than L2; no flush)",
-                   "graph": "one CUDA graph per step, PDL between kernels"},
-        "roofline": {"bound": "hbm", "kernel": "gate/up GEMV (RMSNorm prologue + SwiGLU epilogue)",
-                     "achieved": round(gu_gbs, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(gu_gbs / peak, 4), "traffic": args.traffic,
-                     "bytes_per_launch": gu_bytes, "avg_launch_us": round(gu_ms * 1e3, 3),
-                     "timing": f"CUDA events around every gate/up launch of {n_probe} kernel-by-kernel steps "
-                               f"right after the timed region ({round(probe_ms_step, 4)} ms/step there)"},
+                   "graph": ("one CUDA graph per step: parameter copy, sync-word reset, one persistent kernel"
+                             if persistent else "one CUDA graph per step, PDL between kernels")},
+        "roofline": roof,
         "decode_roofline": {"bytes_per_token": bpt, "peak": peak, "unit": "GB/s",
                             "roofline_tok_s": round(peak * 1e9 / bpt, 2),
                             "frac": round(value / dist.world / (peak * 1e9 / bpt), 4),
@@ -305,6 +352,7 @@ def run_ntx(args, dist: Dist):
         "launches_per_step": launches,
         "clocks": clk,
         "gemv": gemv,
+        "chain": chain,
         "cpu_baseline": cpu,
     }
     return out
@@ -435,6 +483,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama8b-q8_0")
     ap.add_argument("--no-gemv", action="store_true", help="skip the config 1-2 GEMV sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-chain", action="store_true", help="skip timing the per-op kernel chain for comparison")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture (reported as is)")
     args = ap.parse_args()

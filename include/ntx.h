@@ -227,12 +227,18 @@ NTX_API int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_weight
  *     when no layer is on the host.
  * The engine owns only its events, a pinned 16-byte parameter block and the
  * captured CUDA graphs; the caller keeps every buffer alive until
- * ntx_engine_destroy. */
+ * ntx_engine_destroy.
+ * Execution: when every layer is resident (tier 0) and every layer and the
+ * head share one block type, a step runs as ONE persistent kernel (one CTA
+ * per SM, grid-wide phase barriers, the weight stream continuing across
+ * phases); otherwise, or with NTX_NO_PERSIST, as a chain of per-op kernels
+ * (about five per layer) joined by programmatic dependent launch. */
 typedef struct ntx_engine ntx_engine;
 
 #define NTX_CALIBRATE_SKIP 1 /* run every layer, record cosines, fix the skip set {l : cos_l >= tau} */
 #define NTX_USE_SKIP 2       /* skip the layers of the recorded set (not computed, not streamed) */
 #define NTX_NO_GRAPH 4       /* launch kernel by kernel instead of replaying the captured graph */
+#define NTX_NO_PERSIST 8     /* run the step as a chain of per-op kernels even where the persistent kernel applies */
 
 NTX_API size_t ntx_engine_workspace_bytes(const ntx_model_config* cfg);
 NTX_API int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_weights* layers, const int8_t* tier_map,
@@ -255,10 +261,12 @@ NTX_API int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* logits
 
 /* Profiling: while set, every ntx_decode_step made with NTX_NO_GRAPH records
  * begin_events[k] and end_events[k] (caller-created cudaEvent_t, passed as
- * void*) on the compute stream immediately before and after the gate/up GEMV
- * of the k-th computed layer of the step -- the largest kernel of a layer.
- * n is the capacity of both arrays (layers past it are not probed); n == 0
- * clears the probe.  Graph replays never record probe events. */
+ * void*) on the compute stream.  Per-op chain: immediately before and after
+ * the gate/up GEMV of the k-th computed layer of the step -- the largest
+ * kernel of a layer.  Persistent kernel: begin_events[0] / end_events[0]
+ * bracket the kernel.  n is the capacity of both arrays (layers past it are
+ * not probed); n == 0 clears the probe.  Graph replays never record probe
+ * events. */
 NTX_API int ntx_engine_set_probe(ntx_engine* e, void* const* begin_events, void* const* end_events, int n);
 
 /* Number of libntx kernels one decode step launched (the last step enqueued

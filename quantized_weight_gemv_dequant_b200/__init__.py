@@ -26,7 +26,7 @@ NTX_ERR_TIMEOUT = -6
 NTX_ERR_NOMEM = -7
 
 NTX_F32, NTX_F16, NTX_Q4_0, NTX_Q8_0, NTX_Q6_K = 0, 1, 2, 8, 14
-NTX_CALIBRATE_SKIP, NTX_USE_SKIP, NTX_NO_GRAPH = 1, 2, 4
+NTX_CALIBRATE_SKIP, NTX_USE_SKIP, NTX_NO_GRAPH, NTX_NO_PERSIST = 1, 2, 4, 8
 
 BLOCK_ELEMS = {NTX_Q4_0: 32, NTX_Q8_0: 32, NTX_Q6_K: 256}
 BLOCK_BYTES = {NTX_Q4_0: 18, NTX_Q8_0: 34, NTX_Q6_K: 210}

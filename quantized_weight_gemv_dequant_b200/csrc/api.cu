@@ -14,6 +14,7 @@
 
 #include "launch.h"
 #include "ntx.h"
+#include "persist.h"
 
 namespace {
 
@@ -350,11 +351,19 @@ struct ntx_engine {
   // skip set
   std::vector<uint8_t> skip;
   bool skip_valid;
-  // graphs, keyed by (use_skip, logits, next_token, cos_out)
+  // graphs, keyed by (use_skip | no_persist << 1, logits, next_token, cos_out)
   std::map<std::tuple<int, float*, int32_t*, float*>, cudaGraphExec_t> graphs;
   // profiling probe (kernel-by-kernel steps only) and launch count
   std::vector<cudaEvent_t> probe_b, probe_e;
   int launches;
+  // persistent decode kernel (all layers resident, one block type)
+  bool persist;
+  ntx::PStep pst;
+  size_t psmem;
+  int pgrid;
+  ntx::PLayer *pl_all, *pl_skip;
+  int n_skip_run;  // executed layers under the skip set
+  unsigned* psync;
 };
 
 size_t engine_carve(const ntx_model_config* c, uint8_t* base, ntx_engine* e) {
@@ -362,11 +371,12 @@ size_t engine_carve(const ntx_model_config* c, uint8_t* base, ntx_engine* e) {
   const int64_t Q = (int64_t)c->n_heads * c->head_dim;
   const int P = max_parts();
   const int ns = ntx::attn_splits(c->n_kv_heads, c->max_ctx);
+  const int ns_p = ntx::persist_splits(ntx::sm_count(), c->n_kv_heads, c->max_ctx);
   const int L = c->n_layers > 0 ? c->n_layers : 1;
   float* hidden = k.take<float>(c->hidden);
   float* q = k.take<float>(Q);
   float* ao = k.take<float>(Q);
-  float* ap = k.take<float>((uint64_t)c->n_heads * ns * (c->head_dim + 2));
+  float* ap = k.take<float>((uint64_t)c->n_heads * (ns > ns_p ? ns : ns_p) * (c->head_dim + 2));
   float* h1 = k.take<float>(c->hidden);
   float* u = k.take<float>(c->ffn);
   float* se = k.take<float>((uint64_t)P * 4);
@@ -378,7 +388,11 @@ size_t engine_carve(const ntx_model_config* c, uint8_t* base, ntx_engine* e) {
   int* params = k.take<int>(4);
   int* ts = k.take<int>(4);
   int* ll = k.take<int>(L);
+  ntx::PLayer* pla = k.take<ntx::PLayer>(L);
+  ntx::PLayer* pls = k.take<ntx::PLayer>(L);
+  unsigned* psync = k.take<unsigned>(ntx::persist_sync_words(L, c->n_kv_heads));
   if (e) {
+    e->pl_all = pla; e->pl_skip = pls; e->psync = psync;
     e->hidden = hidden; e->q = q; e->attn_out = ao; e->attn_part = ap; e->h1 = h1; e->u = u;
     e->stats_embed = se; e->stats_o = so; e->stats_down = sd; e->arg_parts = apart; e->cos_int = ci;
     e->logits_int = li; e->params = params; e->token_state = ts; e->layer_list = ll;
@@ -412,9 +426,60 @@ void engine_free(ntx_engine* e) {
   delete e;
 }
 
+// Device table of the executed layers for the persistent kernel.
+cudaError_t upload_players(ntx_engine* e, const std::vector<int>& list, ntx::PLayer* dst) {
+  std::vector<ntx::PLayer> t(list.size());
+  for (size_t i = 0; i < list.size(); ++i) {
+    const int l = list[i];
+    const ntx::LayerArgs a = layer_args(&e->cfg, static_cast<const uint8_t*>(e->layers[l].base), e->layers[l].qtype,
+                                        &e->layers[l]);
+    ntx::PLayer& p = t[i];
+    p.wq = a.wq; p.wk = a.wk; p.wv = a.wv; p.wo = a.wo; p.wg = a.wg; p.wu = a.wu; p.wd = a.wd;
+    p.attn_norm = a.attn_norm; p.ffn_norm = a.ffn_norm;
+    p.kc = e->kc[l]; p.vc = e->vc[l];
+    p.stats_down = e->stats_down + l * e->stats_stride;
+  }
+  if (t.empty()) return cudaSuccess;
+  return cudaMemcpy(dst, t.data(), sizeof(ntx::PLayer) * t.size(), cudaMemcpyHostToDevice);
+}
+
+// The whole step as one persistent kernel (plus the cosine finalisation when asked).
+cudaError_t persist_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t* next_token, float* cos_out,
+                            bool calibrate, bool probe) {
+  const ntx_model_config& c = e->cfg;
+  cudaStream_t s = e->cs;
+  const bool sk = use_skip && e->skip_valid;
+  const int nrun = sk ? e->n_skip_run : c.n_layers;
+  ntx::PStep st = e->pst;
+  st.layers = sk ? e->pl_skip : e->pl_all;
+  st.n_layers = nrun;
+  st.logits = logits ? logits : e->logits_int;
+  st.next_token = next_token;
+  st.head_ctr_index = 2 + 5 * nrun;
+  st.abort_index = st.head_ctr_index + nrun * c.n_kv_heads;
+  cudaError_t err =
+      cudaMemsetAsync(e->psync, 0, sizeof(unsigned) * ntx::persist_sync_words(nrun, c.n_kv_heads), s);
+  if (err == cudaSuccess && probe && !e->probe_b.empty()) err = cudaEventRecord(e->probe_b[0], s);
+  if (err == cudaSuccess) err = ntx::launch_persist(e->layers.empty() ? e->head_qtype : e->layers[0].qtype, st,
+                                                    e->psmem, e->pgrid, s);
+  if (err == cudaSuccess && probe && !e->probe_e.empty()) err = cudaEventRecord(e->probe_e[0], s);
+  if (err != cudaSuccess) return err;
+  e->launches = 1;
+  float* cdst = calibrate ? e->cos_int : cos_out;
+  if (cdst && nrun > 0) {
+    e->launches += 1;
+    err = ntx::launch_cos_finalize(e->stats_down, e->pgrid, sk ? e->layer_list : nullptr, nrun, e->stats_stride, cdst,
+                                   s, false);
+    if (err == cudaSuccess && calibrate && cos_out)
+      err = cudaMemcpyAsync(cos_out, e->cos_int, sizeof(float) * c.n_layers, cudaMemcpyDeviceToDevice, s);
+  }
+  return err;
+}
+
 // Enqueue the per-token launch sequence (everything after the parameter copy).
 cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t* next_token, float* cos_out,
-                           bool calibrate, bool probe) {
+                           bool calibrate, bool probe, bool no_persist) {
+  if (e->persist && !no_persist) return persist_enqueue(e, use_skip, logits, next_token, cos_out, calibrate, probe);
   const ntx_model_config& c = e->cfg;
   cudaStream_t s = e->cs;
   const bool pdl = true;
@@ -578,6 +643,50 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   }
   if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->fork_ev, cudaEventDisableTiming);
   if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->join_ev, cudaEventDisableTiming);
+  // persistent kernel: every layer resident and of the head's block type, shapes and alignment it handles
+  e->persist = false;
+  bool one_type = !any_host && (head_qtype == NTX_Q8_0 || head_qtype == NTX_Q4_0 || head_qtype == NTX_Q6_K);
+  for (int l = 0; l < cfg->n_layers && one_type; ++l) one_type = layers[l].qtype == head_qtype;
+  if (err == cudaSuccess && one_type) {
+    ntx::PStep st;
+    memset(&st, 0, sizeof st);
+    size_t psm = 0;
+    const int qt = head_qtype;
+    if (ntx::persist_plan(qt, cfg->hidden, cfg->n_heads, cfg->n_kv_heads, cfg->head_dim, cfg->ffn, cfg->vocab,
+                          cfg->max_ctx, ntx::sm_count(), cfg->n_layers, &st, &psm) == 0) {
+      const int grid = ntx::persist_grid(qt, psm);
+      bool ok = grid > 0 && grid == ntx::sm_count() && ntx::gemv_tma_ok(qt, head, cfg->hidden);
+      for (int l = 0; l < cfg->n_layers && ok; ++l) {
+        const ntx::LayerArgs a = layer_args(cfg, static_cast<const uint8_t*>(layers[l].base), qt, &layers[l]);
+        const int64_t KO = (int64_t)cfg->n_heads * cfg->head_dim;
+        ok = ntx::gemv_tma_ok(qt, a.wq, cfg->hidden) && ntx::gemv_tma_ok(qt, a.wk, cfg->hidden) &&
+             ntx::gemv_tma_ok(qt, a.wv, cfg->hidden) && ntx::gemv_tma_ok(qt, a.wo, KO) &&
+             ntx::gemv_tma_ok(qt, a.wg, cfg->hidden) && ntx::gemv_tma_ok(qt, a.wu, cfg->hidden) &&
+             ntx::gemv_tma_ok(qt, a.wd, cfg->ffn) && aligned(a.attn_norm, 16) && aligned(a.ffn_norm, 16) &&
+             aligned(e->kc[l], 16) && aligned(e->vc[l], 16);
+      }
+      if (ok) {
+        st.H = cfg->hidden; st.Hq = cfg->n_heads; st.Hkv = cfg->n_kv_heads; st.D = cfg->head_dim; st.F = cfg->ffn;
+        st.V = cfg->vocab; st.max_ctx = cfg->max_ctx; st.eps = cfg->eps; st.theta = cfg->theta;
+        st.embed = embed; st.final_norm = final_norm; st.head = static_cast<const uint8_t*>(head);
+        st.hidden = e->hidden; st.q = e->q; st.attn_out = e->attn_out; st.attn_part = e->attn_part;
+        st.h1 = e->h1; st.u = e->u; st.stats_embed = e->stats_embed; st.stats_o = e->stats_o;
+        st.arg_parts = e->arg_parts; st.params = e->params; st.token_state = e->token_state;
+        st.sync = e->psync;
+        st.n_split = ntx::persist_splits(grid, cfg->n_kv_heads, cfg->max_ctx);
+        st.status = ntx::device_status_ptr();
+        std::vector<int> all(cfg->n_layers);
+        for (int l = 0; l < cfg->n_layers; ++l) all[l] = l;
+        err = upload_players(e, all, e->pl_all);
+        if (err == cudaSuccess) {
+          e->pst = st;
+          e->psmem = psm;
+          e->pgrid = grid;
+          e->persist = true;
+        }
+      }
+    }
+  }
   // token state starts at 0
   if (err == cudaSuccess) err = cudaMemsetAsync(e->token_state, 0, 4 * sizeof(int), e->cs);
   if (err == cudaSuccess) err = cudaStreamSynchronize(e->cs);
@@ -595,7 +704,9 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
   const ntx_model_config& c = e->cfg;
   if (pos < 0 || pos >= c.max_ctx) return fail(NTX_ERR_SHAPE, "pos %d outside [0, max_ctx=%d)", pos, c.max_ctx);
   if (token < -1 || token >= c.vocab) return fail(NTX_ERR_INVALID_ARG, "token %d outside [-1, vocab)", token);
-  if (flags & ~(NTX_CALIBRATE_SKIP | NTX_USE_SKIP | NTX_NO_GRAPH)) return fail(NTX_ERR_INVALID_ARG, "unknown flags");
+  if (flags & ~(NTX_CALIBRATE_SKIP | NTX_USE_SKIP | NTX_NO_GRAPH | NTX_NO_PERSIST))
+    return fail(NTX_ERR_INVALID_ARG, "unknown flags");
+  const bool no_persist = (flags & NTX_NO_PERSIST) != 0;
   const bool calibrate = flags & NTX_CALIBRATE_SKIP;
   const bool use_skip = !calibrate && (flags & NTX_USE_SKIP) && e->skip_valid;
   int cur = 0;
@@ -614,16 +725,17 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
   if (err != cudaSuccess) return cuda_fail(err, "param copy");
 
   if ((flags & NTX_NO_GRAPH) || calibrate) {
-    err = engine_enqueue(e, use_skip, logits, next_token, cos_out, calibrate, (flags & NTX_NO_GRAPH) != 0);
+    err = engine_enqueue(e, use_skip, logits, next_token, cos_out, calibrate, (flags & NTX_NO_GRAPH) != 0,
+                         no_persist);
     if (err != cudaSuccess) return cuda_fail(err, "ntx_decode_step");
   } else {
-    const auto key = std::make_tuple(use_skip ? 1 : 0, logits, next_token, cos_out);
+    const auto key = std::make_tuple((use_skip ? 1 : 0) | (no_persist ? 2 : 0), logits, next_token, cos_out);
     auto it = e->graphs.find(key);
     if (it == e->graphs.end()) {
       cudaGraph_t g = nullptr;
       err = cudaStreamBeginCapture(e->cs, cudaStreamCaptureModeThreadLocal);
       if (err != cudaSuccess) return cuda_fail(err, "begin capture");
-      const cudaError_t err_enq = engine_enqueue(e, use_skip, logits, next_token, cos_out, false, false);
+      const cudaError_t err_enq = engine_enqueue(e, use_skip, logits, next_token, cos_out, false, false, no_persist);
       err = cudaStreamEndCapture(e->cs, &g);
       if (err_enq != cudaSuccess || err != cudaSuccess) {
         if (g) cudaGraphDestroy(g);
@@ -651,12 +763,14 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
     }
     if (!list.empty()) {
       err = cudaMemcpy(e->layer_list, list.data(), sizeof(int) * list.size(), cudaMemcpyHostToDevice);
+      if (err == cudaSuccess && e->persist) err = upload_players(e, list, e->pl_skip);
       if (err != cudaSuccess) return cuda_fail(err, "layer list");
     }
+    e->n_skip_run = (int)list.size();
     e->skip_valid = true;
     // graphs built with an older skip set are stale
     for (auto itg = e->graphs.begin(); itg != e->graphs.end();) {
-      if (std::get<0>(itg->first) == 1) {
+      if (std::get<0>(itg->first) & 1) {
         cudaGraphExecDestroy(itg->second);
         itg = e->graphs.erase(itg);
       } else {

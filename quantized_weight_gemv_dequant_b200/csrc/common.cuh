@@ -13,7 +13,13 @@
 namespace ntx {
 
 // Device status word (read and cleared by ntx_device_status()).
-enum : int { kStatusOk = 0, kStatusTmaTimeout = 1, kStatusDrainTimeout = 2, kStatusBadToken = 3 };
+enum : int {
+  kStatusOk = 0,
+  kStatusTmaTimeout = 1,
+  kStatusDrainTimeout = 2,
+  kStatusBadToken = 3,
+  kStatusGridTimeout = 4,  // a grid-wide barrier of the persistent decode kernel ran out
+};
 
 // Limit on any single wait (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

@@ -452,6 +452,56 @@ __device__ __forceinline__ int group8_sum(int v) {
   return v + __shfl_xor_sync(0xffffffffu, v, 4);
 }
 
+// One 128-column chunk of x (4 columns per lane, starting at col = chunk
+// start + 4 lane) into the staged form.
+template <int QT>
+__device__ __forceinline__ void stage_chunk(const float4 v, int64_t col, const XStage& xs, int lane) {
+  if constexpr (QT == QT_Q6_K) {
+    *reinterpret_cast<float4*>(xs.xf + col) = v;
+  } else {
+    const float m = group8_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    // e with 2^(e-1) <= m < 2^e from the exponent field (m = 0 or subnormal: the
+    // clamp at -100 makes every X round to 0, as it must); both scales are
+    // normal powers of two built from their exponent fields.
+    int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 126;
+    if (e < -100) e = -100;
+    const float up = __uint_as_float((uint32_t)(127 + 22 - e) << 23);
+    const int X[4] = {__float2int_rn(v.x * up), __float2int_rn(v.y * up), __float2int_rn(v.z * up),
+                      __float2int_rn(v.w * up)};
+    uint32_t w0 = 0, w1 = 0, w2 = 0;
+    int s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t b0 = (uint32_t)X[t] & 0xFFu, b1 = ((uint32_t)X[t] >> 8) & 0xFFu;
+      const int hi = X[t] >> 16;  // arithmetic: in [-64, 64]
+      w0 |= b0 << (8 * t);
+      w1 |= b1 << (8 * t);
+      w2 |= ((uint32_t)hi & 0xFFu) << (8 * t);
+      s0 += (int)b0;
+      s1 += (int)b1;
+      s2 += hi;
+    }
+    const int c = (int)(col / kSliceCols), u = (int)(col % kSliceCols);
+    const int l = u / 64, k = (u % 64) / 4;
+    const int wi = k * xs.np + c * 32 + l;
+    xs.wd[wi] = w0;
+    xs.wd[16 * xs.np + wi] = w1;
+    xs.wd[32 * xs.np + wi] = w2;
+    const int64_t B = col / 32;
+    if constexpr (QT == QT_Q4_0) {
+      s0 = group8_sum(s0);
+      s1 = group8_sum(s1);
+      s2 = group8_sum(s2);
+      if ((lane & 7) == 0) {
+        xs.cr[3 * B + 0] = -8 * s0;
+        xs.cr[3 * B + 1] = -8 * s1;
+        xs.cr[3 * B + 2] = -8 * s2;
+      }
+    }
+    if ((lane & 7) == 0) xs.sc[B] = __uint_as_float((uint32_t)(127 + e - 22) << 23);
+  }
+}
+
 // K is a multiple of 256 on every path that stages x.
 template <int QT, class Pro>
 __device__ __forceinline__ void stage_x(const Pro& pro, int64_t K, const XStage& xs, int cw, int NW, int lane) {
@@ -468,48 +518,7 @@ __device__ __forceinline__ void stage_x(const Pro& pro, int64_t K, const XStage&
     for (int b = 0; b < kBatch; ++b) {
       const int ch = ch0 + b * NW;
       if (ch >= nchunk) break;  // uniform across the warp
-      const int64_t col = (int64_t)ch * 128 + 4 * lane;
-      if constexpr (QT == QT_Q6_K) {
-        *reinterpret_cast<float4*>(xs.xf + col) = v[b];
-      } else {
-        const float m = group8_max(fmaxf(fmaxf(fabsf(v[b].x), fabsf(v[b].y)), fmaxf(fabsf(v[b].z), fabsf(v[b].w))));
-        int e = m > 0.f ? ilogbf(m) + 1 : 0;
-        if (e < -100) e = -100;
-        const float up = ldexpf(1.0f, 22 - e);
-        const int X[4] = {__float2int_rn(v[b].x * up), __float2int_rn(v[b].y * up), __float2int_rn(v[b].z * up),
-                          __float2int_rn(v[b].w * up)};
-        uint32_t w0 = 0, w1 = 0, w2 = 0;
-        int s0 = 0, s1 = 0, s2 = 0;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const uint32_t b0 = (uint32_t)X[t] & 0xFFu, b1 = ((uint32_t)X[t] >> 8) & 0xFFu;
-          const int hi = X[t] >> 16;  // arithmetic: in [-64, 64]
-          w0 |= b0 << (8 * t);
-          w1 |= b1 << (8 * t);
-          w2 |= ((uint32_t)hi & 0xFFu) << (8 * t);
-          s0 += (int)b0;
-          s1 += (int)b1;
-          s2 += hi;
-        }
-        const int c = (int)(col / kSliceCols), u = (int)(col % kSliceCols);
-        const int l = u / 64, k = (u % 64) / 4;
-        const int wi = k * xs.np + c * 32 + l;
-        xs.wd[wi] = w0;
-        xs.wd[16 * xs.np + wi] = w1;
-        xs.wd[32 * xs.np + wi] = w2;
-        const int64_t B = col / 32;
-        if constexpr (QT == QT_Q4_0) {
-          s0 = group8_sum(s0);
-          s1 = group8_sum(s1);
-          s2 = group8_sum(s2);
-          if ((lane & 7) == 0) {
-            xs.cr[3 * B + 0] = -8 * s0;
-            xs.cr[3 * B + 1] = -8 * s1;
-            xs.cr[3 * B + 2] = -8 * s2;
-          }
-        }
-        if ((lane & 7) == 0) xs.sc[B] = ldexpf(1.0f, e - 22);
-      }
+      stage_chunk<QT>(v[b], (int64_t)ch * 128 + 4 * lane, xs, lane);
     }
   }
 }
@@ -547,6 +556,10 @@ struct XRegs<QT_Q6_K> {
   f32x2 x2[32];
   __device__ __forceinline__ void load(const XStage& xs, int c, int lane) {
     load_x_slice_q6_k(ProSmem{xs.xf}, (int64_t)c * kSliceCols, lane, x2);
+  }
+  template <class Pro>
+  __device__ __forceinline__ void load_direct(const Pro& pro, int c, int lane) {
+    load_x_slice_q6_k(pro, (int64_t)c * kSliceCols, lane, x2);
   }
   __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const { return row_q6_k(seg, lane, x2); }
 };
@@ -648,10 +661,12 @@ struct EpiResid {
   float nres, nhc, cres, chc;
   static constexpr int kAlign = 1;
   __device__ __forceinline__ void init(float2*, int) { st0 = st1 = st2 = 0.f; }
+  // L2 loads: inside the persistent decode kernel these rows were written by
+  // an earlier phase of the same launch.
   __device__ __forceinline__ void preload(int64_t rs, int nr, int lane) {
     if (lane < nr) {
-      nres = resid[rs + lane];
-      nhc = hc ? hc[rs + lane] : 0.f;
+      nres = __ldcg(resid + rs + lane);
+      nhc = hc ? __ldcg(hc + rs + lane) : 0.f;
     }
   }
   __device__ __forceinline__ void rotate() {

@@ -39,6 +39,12 @@ int* status_ptr() {
   return ptrs[d];
 }
 
+}  // namespace
+
+int* device_status_ptr() { return status_ptr(); }
+
+namespace {
+
 // Raise the dynamic shared-memory limit of a kernel once per device; `done`
 // is a per-kernel bit set (one bit per device).
 template <class K>

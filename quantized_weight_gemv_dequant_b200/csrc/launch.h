@@ -74,6 +74,7 @@ cudaError_t launch_cos_finalize(const float* stats, int nparts, const int* layer
                                 float* cos_out, cudaStream_t s, bool pdl);
 
 int read_device_status(int* code);
+int* device_status_ptr();
 
 // Record a failure for ntx_last_error() on the calling thread; returns code.
 int record_error(int code, const char* msg);

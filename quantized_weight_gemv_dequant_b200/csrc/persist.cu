@@ -1,0 +1,1180 @@
+// persist.cu -- one decode step (embed -> L layers -> head -> argmax) as a
+// single persistent kernel: one CTA per SM for the whole step.
+//
+// Why.  Batch-1 decode streams every weight byte once per token ("NTransformer"
+// -- アーキテクチャ概要 and "RTX 3090 1枚でLlama 70B" -- VRAMの壁: the GEMV is
+// memory bound), so the step can only approach the HBM roofline if the weight
+// stream never pauses.  A chain of per-op kernels pauses at every boundary:
+// each kernel's CTAs must drain before the next kernel's CTAs (one per SM, up
+// to 227 KB of shared memory each) can start copying.  Here the producer warp
+// of each CTA walks one continuous list of weight stages across all phases of
+// the step; the weights never depend on activations, so it keeps the copy ring
+// full while the consumer warps wait at a phase boundary or compute attention.
+//
+// Phases (index p; one grid-wide counter each):
+//   0            EMBED  h = fp16 row of the token, sum(h^2) partials
+//   1 + 5k + 0   QKV    RMSNorm(h) prologue, q/k/v rows, RoPE, KV append
+//   1 + 5k + 1   ATTN   split-KV GQA attention, the last CTA of each KV head
+//                       merges the splits (log-sum-exp)
+//   1 + 5k + 2   O      h1 = h + Wo a, sum(h1^2) partials
+//   1 + 5k + 3   GU     RMSNorm(h1) prologue, u = silu(Wg n) * (Wu n)
+//   1 + 5k + 4   DOWN   h = h1 + Wd u, residual and cosine statistics
+//   1 + 5n       HEAD   RMSNorm(h) prologue, logits, argmax (the last CTA to
+//                       finish picks the token)
+// where k runs over the executed layers (a skip set removes layers from the
+// list).  A phase's inputs are complete when every CTA has arrived on the
+// previous phase's counter: GEMV phases arrive from the producer warp after
+// its epilogue stores, EMBED and ATTN from the consumer warps.  Every wait is
+// bounded (%globaltimer) and any CTA that gives up raises a grid-wide abort
+// word, so the other CTAs stop waiting too; the producer lets its copies in
+// flight land before the CTA exits.
+//
+// GEMV work inside a phase is the same as in gemv_tma_kernel: rows are split
+// evenly over the CTAs; consumer warp (c, g) owns K slice c (2048 columns,
+// x in registers) and row group g; partials go through shared memory to the
+// producer warp, which sums them in a fixed order and runs the epilogue.  All
+// phases share one ring of equal-size slots; each phase fits as many whole
+// rows in a slot as it can (an even count where the epilogue pairs rows).
+// Data written by an earlier phase of this launch is read through L2
+// (ld.global.cg), never through the non-coherent or L1 paths.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "gemv.cuh"
+#include "launch.h"
+#include "persist.h"
+
+namespace ntx {
+namespace {
+
+extern __shared__ __align__(128) uint8_t p_smem[];  // the kernel's dynamic shared memory
+
+constexpr int kPWarps = kPConsumers + 2;  // + epilogue warp + copy warp
+constexpr int kPEpiWarp = kPConsumers, kPCopyWarp = kPConsumers + 1;
+constexpr int kPThreads = kPWarps * 32;
+constexpr int kPCThreads = kPConsumers * 32;
+constexpr float kAttnScale = 0.08838834764831845f;  // 1 / sqrt(128)
+
+__device__ __forceinline__ void cons_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kPCThreads) : "memory"); }
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned atom_acq_rel_add(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// One thread: wait until *ctr >= target.  False if the grid-wide abort word is
+// raised or the wait runs out (which raises it).
+__device__ bool grid_wait(const unsigned* ctr, unsigned target, unsigned* gabort, int* status) {
+  if (ld_acquire(ctr) >= target) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    __nanosleep(20);
+    if (ld_acquire(ctr) >= target) return true;
+    if (*reinterpret_cast<volatile unsigned*>(gabort)) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicExch(status, (int)kStatusGridTimeout);
+      atomicExch(gabort, 1u);
+      return false;
+    }
+  }
+}
+
+// Warp-uniform bounded wait on an mbarrier phase that also gives up when this
+// CTA has aborted.
+__device__ bool pwait(uint64_t* bar, uint32_t parity, volatile int* cta_abort) {
+  bool done = mbar_try_wait(bar, parity);
+  if (__all_sync(0xffffffffu, done)) return true;
+  const uint64_t t0 = global_ns();
+  while (!__all_sync(0xffffffffu, done)) {
+    if (!done) done = mbar_try_wait_sleep(bar, parity);
+    const bool give_up = *cta_abort || global_ns() - t0 > kWaitLimitNs;
+    if (__any_sync(0xffffffffu, !done && give_up)) break;
+  }
+  return __all_sync(0xffffffffu, done);
+}
+
+__device__ __forceinline__ int phase_kind(int p, int n) {
+  if (p == 0) return PK_EMBED;
+  if (p == 1 + 5 * n) return PK_HEAD;
+  return PK_QKV + (p - 1) % 5;
+}
+
+struct PRows {
+  int r0, r1;  // rows [r0, r1) of this CTA (every phase has fewer than 2^31 rows)
+  int n;       // stages
+};
+
+__device__ __forceinline__ int64_t phase_M(const PStep& st, int kind) {
+  switch (kind) {
+    case PK_QKV: return (int64_t)(st.Hq + 2 * st.Hkv) * st.D;
+    case PK_O: return st.H;
+    case PK_GU: return 2 * (int64_t)st.F;
+    case PK_DOWN: return st.H;
+    default: return st.V;
+  }
+}
+__device__ __forceinline__ int64_t phase_K(const PStep& st, int kind) {
+  switch (kind) {
+    case PK_O: return (int64_t)st.Hq * st.D;
+    case PK_DOWN: return st.F;
+    default: return st.H;
+  }
+}
+
+__device__ __forceinline__ PRows phase_rows(const PStep& st, int kind) {
+  const PGeom& g = st.g[kind];
+  const int64_t M = phase_M(st, kind), A = g.align;
+  const int64_t units = (M + A - 1) / A;
+  PRows r;
+  r.r0 = (int)(units * blockIdx.x / gridDim.x * A);
+  r.r1 = (int)min64(M, units * (blockIdx.x + 1) / gridDim.x * A);
+  const int nr = r.r1 > r.r0 ? r.r1 - r.r0 : 0;
+  r.n = (nr + g.TR - 1) / g.TR;
+  return r;
+}
+
+__device__ __forceinline__ const PLayer* phase_layer(const PStep& st, int p) {
+  return (p >= 1 && p < 1 + 5 * st.n_layers) ? st.layers + (p - 1) / 5 : nullptr;
+}
+
+// Walks the weight stages of this CTA over all phases, in order.  Entering a
+// phase loads its matrix base pointers once, so that the source address of a
+// row copy is register arithmetic only.
+struct PIssue {
+  int p, j, n, kind;
+  int64_t r0, r1;
+  int TR, rb;
+  const uint8_t *b0, *b1, *b2;  // QKV: wq, wk, wv; GU: wg, wu; otherwise b0
+  int64_t nq, nkv;
+  __device__ void seek(const PStep& st, int from, int np) {
+    for (p = from; p < np; ++p) {
+      kind = phase_kind(p, st.n_layers);
+      if (kind == PK_EMBED || kind == PK_ATTN) continue;
+      const PRows r = phase_rows(st, kind);
+      if (r.n == 0) continue;
+      r0 = r.r0; r1 = r.r1; n = r.n; j = 0;
+      TR = st.g[kind].TR;
+      rb = st.g[kind].row_bytes;
+      const PLayer* L = phase_layer(st, p);
+      nq = (int64_t)st.Hq * st.D;
+      nkv = (int64_t)st.Hkv * st.D;
+      b1 = b2 = nullptr;
+      switch (kind) {
+        case PK_QKV: b0 = L->wq; b1 = L->wk; b2 = L->wv; break;
+        case PK_O: b0 = L->wo; break;
+        case PK_GU: b0 = L->wg; b1 = L->wu; break;
+        case PK_DOWN: b0 = L->wd; break;
+        default: b0 = st.head; break;
+      }
+      return;
+    }
+  }
+  __device__ __forceinline__ const uint8_t* row(int64_t r) const {
+    if (kind == PK_QKV) {
+      if (r < nq) return b0 + r * rb;
+      if (r < nq + nkv) return b1 + (r - nq) * rb;
+      return b2 + (r - nq - nkv) * rb;
+    }
+    if (kind == PK_GU) return ((r & 1) ? b1 : b0) + (r >> 1) * rb;
+    return b0 + r * rb;
+  }
+  __device__ __forceinline__ bool valid(int np) const { return p < np; }
+  __device__ __forceinline__ void advance(const PStep& st, int np) {
+    if (++j >= n) seek(st, p + 1, np);
+  }
+};
+
+// x prologue with L2 loads (x was produced by an earlier phase): RMSNorm(h) w
+// when a norm weight is given, x itself otherwise.
+struct PX {
+  const float* h;
+  const float* w;  // nullable
+  float r;
+  __device__ __forceinline__ float4 ld(int64_t j) const {
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(h + j));
+    if (!w) return a;
+    const float4 b = ldg4(w + j);
+    return make_float4(b.x * (a.x * r), b.y * (a.y * r), b.z * (a.z * r), b.w * (a.w * r));
+  }
+};
+
+// Shared-memory carve, identical on host and device.
+struct PSmem {
+  uint8_t* ring;    // [S][Z] weight slots
+  uint8_t* xst;     // x staging / attention scratch
+  uint64_t* full;   // [S] weight slot landed (copy warp -> consumers)
+  uint64_t* empty;  // [S] weight slot read (consumers -> copy warp)
+  uint64_t* rfull;  // [kPRed] row partials written (consumers -> epilogue warp)
+  uint64_t* rempty; // [kPRed] row partials read (epilogue warp -> consumers)
+  float* red;       // [kPRed][RF] row partials
+  float2* rope;     // [64] RoPE (cos, sin) of this step's position
+  int* misc;        // [0] CTA abort, [1..2] phase go flags, [3] last-CTA flag
+  float* scr;       // [16] reductions
+  struct LRow* lt;  // [n_layers] per-layer pointers the consumer and epilogue warps use
+  struct KGeo* kg;  // [7] geometry and this CTA's rows per phase kind
+};
+// Geometry and row range of one GEMV phase kind for this CTA, computed once.
+struct KGeo {
+  PGeom g;
+  PRows rows;
+};
+// Per-layer pointers copied to shared memory at kernel start, so a phase
+// start does not wait for a global load to learn where its inputs are.
+struct LRow {
+  const float* attn_norm;
+  const float* ffn_norm;
+  float* stats_down;
+  uint16_t* kc;
+  uint16_t* vc;
+};
+__host__ __device__ inline size_t psmem_bytes(int S, int Z, int XB, int RF, int nl) {
+  return (size_t)S * Z + XB + (size_t)S * 16 + (size_t)kPRed * 16 + (size_t)kPRed * RF * 4 + 64 * 8 + 16 * 4 +
+         16 * 4 + (size_t)nl * sizeof(LRow) + 7 * sizeof(KGeo);
+}
+__device__ __forceinline__ PSmem psmem_at(uint8_t* base, int S, int Z, int XB, int RF, int nl) {
+  PSmem m;
+  m.ring = base;
+  m.xst = base + (size_t)S * Z;
+  m.full = reinterpret_cast<uint64_t*>(m.xst + XB);
+  m.empty = m.full + S;
+  m.rfull = m.empty + S;
+  m.rempty = m.rfull + kPRed;
+  m.red = reinterpret_cast<float*>(m.rempty + kPRed);
+  m.rope = reinterpret_cast<float2*>(m.red + (size_t)kPRed * RF);
+  m.misc = reinterpret_cast<int*>(m.rope + 64);
+  m.scr = reinterpret_cast<float*>(m.misc + 16);
+  m.lt = reinterpret_cast<LRow*>(m.scr + 16);
+  m.kg = reinterpret_cast<KGeo*>(m.lt + nl);
+  return m;
+}
+
+// Attention scratch inside the x staging region (consumer warps only).
+struct AttnSmem {
+  uint8_t* k;   // [kPChunk][128] fp16
+  uint8_t* v;   // [kPChunk][128] fp16
+  float* sc;    // [G][kPChunk] scores, then probabilities
+  float* ml;    // [G][2]
+  float* sw;    // [G][ns] merge weights
+};
+__host__ __device__ inline size_t attn_smem_bytes(int G, int ns) {
+  return (size_t)2 * kPChunk * kPD * 2 + (size_t)G * kPChunk * 4 + (size_t)G * 2 * 4 + (size_t)G * ns * 4;
+}
+__device__ __forceinline__ AttnSmem attn_smem(uint8_t* base, int G) {
+  AttnSmem a;
+  a.k = base;
+  a.v = base + kPChunk * kPD * 2;
+  a.sc = reinterpret_cast<float*>(a.v + kPChunk * kPD * 2);
+  a.ml = a.sc + G * kPChunk;
+  a.sw = a.ml + 2 * G;
+  return a;
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Bulk prefetch into L2 (16-byte aligned address, size a multiple of 16).
+__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// mbarrier operations on 32-bit shared-window addresses (keeps loop state small).
+__device__ __forceinline__ bool mbar_test_a(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(ok)
+               : "r"(a), "r"(parity)
+               : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_sleep_a(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(a), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void mbar_arrive_a(uint32_t a) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+// pwait on a 32-bit address; cta_abort is the CTA abort word in shared memory.
+__device__ bool pwait_a(uint32_t bar, uint32_t parity, const volatile int* cta_abort) {
+  bool done = mbar_test_a(bar, parity);
+  if (__all_sync(0xffffffffu, done)) return true;
+  const uint64_t t0 = global_ns();
+  while (!__all_sync(0xffffffffu, done)) {
+    if (!done) done = mbar_sleep_a(bar, parity);
+    const bool give_up = *cta_abort || global_ns() - t0 > kWaitLimitNs;
+    if (__any_sync(0xffffffffu, !done && give_up)) break;
+  }
+  return __all_sync(0xffffffffu, done);
+}
+
+// ------------------------------------------------------------ copy warp
+// Streams every weight stage of this CTA, phase after phase, into the ring.
+// It waits only for slots to be released: weights never depend on
+// activations, so the stream runs ahead across phase boundaries.
+struct Copier {
+  const PStep& st;
+  PSmem sm;
+  int lane, np, n_slots, slot_bytes;
+  uint64_t policy;
+  PIssue it;
+  long issued, done;
+
+  __device__ Copier(const PStep& st_, PSmem sm_, int lane_, int np_)
+      : st(st_), sm(sm_), lane(lane_), np(np_), issued(0), done(0) {
+    n_slots = st.n_slots;
+    slot_bytes = st.slot_bytes;
+    policy = l2_evict_first_policy();
+    it.seek(st, 0, np);
+  }
+
+  __device__ __forceinline__ void issue(int slot) {
+    const int64_t rs = it.r0 + (int64_t)it.j * it.TR;
+    const int nr = (int)min64(it.TR, it.r1 - rs);
+    const int rb = it.rb;
+    uint64_t* bar = sm.full + slot;
+    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(nr * rb));
+    __syncwarp();
+    uint8_t* dst = sm.ring + (size_t)slot * slot_bytes;
+    for (int r = lane; r < nr; r += 32) bulk_g2s(dst + (size_t)r * rb, it.row(rs + r), (uint32_t)rb, bar, policy);
+    it.advance(st, np);
+    ++issued;
+  }
+
+  // Lets every issued copy land (bounded) before the warp exits.
+  __device__ void drain() {
+    if (lane == 0) {
+      const uint64_t t0 = global_ns();
+      for (long k = done; k < issued; ++k) {
+        uint64_t* bar = sm.full + k % n_slots;
+        const uint32_t par = (uint32_t)((k / n_slots) & 1);
+        while (!mbar_try_wait(bar, par))
+          if (global_ns() - t0 > kWaitLimitNs) { atomicExch(st.status, (int)kStatusDrainTimeout); return; }
+      }
+    }
+    __syncwarp();
+  }
+
+  __device__ void run() {
+    for (int k = 0; k < n_slots && it.valid(np); ++k) issue(k);
+    int s = 0;
+    uint32_t ph = 0;
+    while (it.valid(np)) {
+      if (!pwait(sm.empty + s, ph, sm.misc)) {
+        if (lane == 0) {
+          atomicExch(sm.misc, 1);
+          atomicExch(st.sync + st.abort_index, 1u);
+        }
+        break;
+      }
+      issue(s);
+      ++done;
+      if (++s == n_slots) { s = 0; ph ^= 1u; }
+    }
+    drain();
+  }
+};
+
+// Residual epilogue for a CTA row range of at most 64 rows: out = v + resid
+// with statistics sum(out^2), sum(hc out), sum(hc^2).  resid and hc (the layer
+// input) for all of the CTA's rows are loaded once at the phase start, so the
+// epilogue warp does not wait on L2 stage by stage; a stage's values are
+// picked with shuffles (all lanes call apply_stage).
+struct PEpiResid {
+  float* out;
+  const float* resid;
+  const float* hc;  // nullable
+  float* parts;     // [gridDim.x][4]
+  int r0;
+  float rv[2], hv[2];
+  float st0, st1, st2;
+  __device__ __forceinline__ void begin(int r0_, int r1_, int lane) {
+    r0 = r0_;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = r0 + lane + 32 * k;
+      rv[k] = i < r1_ ? __ldcg(resid + i) : 0.f;
+      hv[k] = (hc && i < r1_) ? __ldcg(hc + i) : 0.f;
+    }
+    st0 = st1 = st2 = 0.f;
+  }
+  __device__ __forceinline__ void apply_stage(int rs, bool mine, int lane, float a) {
+    const int idx = rs - r0 + lane;  // this lane's row, relative to r0 (< 64 where mine)
+    const int src = idx & 31;
+    const float ra = __shfl_sync(0xffffffffu, rv[0], src), rb = __shfl_sync(0xffffffffu, rv[1], src);
+    const float ha = __shfl_sync(0xffffffffu, hv[0], src), hb = __shfl_sync(0xffffffffu, hv[1], src);
+    if (mine) {
+      const float res = idx < 32 ? ra : rb, h = idx < 32 ? ha : hb;
+      const float o = a + res;
+      if (hc) {
+        st1 = fmaf(h, o, st1);
+        st2 = fmaf(h, h, st2);
+      }
+      st0 = fmaf(o, o, st0);
+      out[rs + lane] = o;
+    }
+  }
+  __device__ __forceinline__ void finish(int lane) {
+    const float a = warp_sum(st0), b = warp_sum(st1), c = warp_sum(st2);
+    if (lane == 0) {
+      parts[blockIdx.x * 4 + 0] = a;
+      parts[blockIdx.x * 4 + 1] = b;
+      parts[blockIdx.x * 4 + 2] = c;
+    }
+  }
+};
+
+// ------------------------------------------------------------ epilogue warp
+// Sums each stage's row partials in a fixed slice order, runs the phase's
+// epilogue and, at the end of the phase, publishes its outputs to the grid.
+struct Epilogue {
+  const PStep& st;
+  PSmem sm;
+  int lane, red_floats;
+  int q;  // partial-ring position (global stage count)
+
+  __device__ Epilogue(const PStep& st_, PSmem sm_, int lane_) : st(st_), sm(sm_), lane(lane_), q(0) {
+    red_floats = st.red_floats;
+  }
+
+  template <class Epi>
+  __device__ bool run(Epi& epi, const PRows rows, const PGeom g) {
+    constexpr int A = Epi::kAlign;
+    const int TR = g.TR, nsl = g.n_slices, nst = rows.n;
+    const int64_t r0 = rows.r0, r1 = rows.r1;
+    const int row_a = A == 1 ? lane : 2 * lane;
+    if (nst > 0) epi.preload(r0, (int)min64(TR, r1 - r0), lane);
+    for (int i = 0; i < nst; ++i, ++q) {
+      const int slot = q % kPRed;
+      if (!pwait(sm.rfull + slot, (uint32_t)((q / kPRed) & 1), sm.misc)) return false;
+      const int64_t rs = r0 + (int64_t)i * TR;
+      const int nr = (int)min64(TR, r1 - rs);
+      const float* rd = sm.red + (size_t)slot * red_floats;
+      float a = 0.f, b = 0.f;
+      const bool mine = row_a < nr;
+      if (mine) {
+        for (int c = 0; c < nsl; ++c) {
+          a += rd[row_a * nsl + c];
+          if (A == 2) b += rd[(row_a + 1) * nsl + c];
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.rempty + slot);
+      epi.rotate();
+      if (i + 1 < nst) epi.preload(rs + TR, (int)min64(TR, r1 - rs - TR), lane);
+      if (mine) epi.apply(rs + row_a, a, b);
+    }
+    return true;
+  }
+
+  // run() for the residual epilogue (rows of this CTA <= 64).
+  __device__ bool run_resid(PEpiResid& epi, const PRows rows, const PGeom g) {
+    const int TR = g.TR, nsl = g.n_slices, nst = rows.n;
+    const int r0 = rows.r0, r1 = rows.r1;
+    epi.begin(r0, r1, lane);
+    for (int i = 0; i < nst; ++i, ++q) {
+      const int slot = q % kPRed;
+      if (!pwait(sm.rfull + slot, (uint32_t)((q / kPRed) & 1), sm.misc)) return false;
+      const int rs = r0 + i * TR;
+      const int nr = min(TR, r1 - rs);
+      const float* rd = sm.red + (size_t)slot * red_floats;
+      float a = 0.f;
+      const bool mine = lane < nr;
+      if (mine)
+        for (int c = 0; c < nsl; ++c) a += rd[lane * nsl + c];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.rempty + slot);
+      epi.apply_stage(rs, mine, lane, a);
+    }
+    return true;
+  }
+};
+
+// ------------------------------------------------------------ consumers
+template <int QT>
+struct Consumer {
+  const PStep& st;
+  PSmem sm;  // used outside the GEMV stage loop only
+  int warp, lane, ctid;
+  int s;
+  uint32_t ph;
+  int q;  // partial-ring position (global stage count)
+
+  __device__ Consumer(const PStep& st_, PSmem sm_, int warp_, int lane_)
+      : st(st_), sm(sm_), warp(warp_), lane(lane_), ctid(warp_ * 32 + lane_), s(0), ph(0), q(0) {}
+
+  // x of a GEMV phase into shared memory (fixed-point limbs or fp32): x = h, or
+  // RMSNorm(h) w with the scale from the per-CTA sum-of-squares partials.  The
+  // partials and the first batch of h (and w) are requested together, so the
+  // staging costs one round trip to L2 for the shapes used here.  Returns the
+  // RMSNorm scale (1 without a norm).
+  template <bool NORM>
+  __device__ float stage(const float* h, const float* w, const float* parts, int64_t K, bool staged,
+                         const XStage& xs) {
+    constexpr int kBatch = NORM ? 4 : 8;
+    const int nchunk = (int)(K / 128);
+    float pp[kPPartsPerLane];
+    if constexpr (NORM) {
+#pragma unroll
+      for (int k = 0; k < kPPartsPerLane; ++k) {
+        const int i = lane + 32 * k;
+        pp[k] = i < (int)gridDim.x ? __ldcg(parts + (int64_t)i * 4) : 0.f;
+      }
+    }
+    float4 hv[kBatch], wv[NORM ? kBatch : 1];
+    if (staged) {
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int ch = warp + b * kPConsumers;
+        const int64_t col = (int64_t)ch * 128 + 4 * lane;
+        hv[b] = ch < nchunk ? __ldcg(reinterpret_cast<const float4*>(h + col)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if constexpr (NORM) wv[b] = ch < nchunk ? ldg4(w + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float r = 1.f;
+    if constexpr (NORM) {
+      float ss = 0.f;
+#pragma unroll
+      for (int k = 0; k < kPPartsPerLane; ++k) ss += pp[k];
+      ss = warp_sum(ss);
+      r = 1.0f / sqrtf(ss / (float)st.H + st.eps);
+    }
+    if (!staged) return r;
+    const PX pro{h, NORM ? w : nullptr, r};
+    for (int ch0 = warp;; ch0 += kBatch * kPConsumers) {
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int ch = ch0 + b * kPConsumers;
+        if (ch >= nchunk) break;  // uniform across the warp
+        float4 v = hv[b];
+        if constexpr (NORM) {
+          if (ch0 == warp)  // only the first batch still needs the norm applied
+            v = make_float4(wv[b].x * (v.x * r), wv[b].y * (v.y * r), wv[b].z * (v.z * r), wv[b].w * (v.w * r));
+        }
+        stage_chunk<QT>(v, (int64_t)ch * 128 + 4 * lane, xs, lane);
+      }
+      if (ch0 + kBatch * kPConsumers >= nchunk) break;
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int ch = ch0 + (kBatch + b) * kPConsumers;
+        hv[b] = ch < nchunk ? pro.ld((int64_t)ch * 128 + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    return r;
+  }
+
+  __device__ bool gemv(int kind, const float* h, const float* w, const float* parts) {
+    const PGeom g = sm.kg[kind].g;
+    const PRows rows = sm.kg[kind].rows;
+    const int64_t K = phase_K(st, kind);
+    const int nsl = g.n_slices, nrg = g.n_rg, TR = g.TR, rbytes = g.row_bytes, nst = rows.n;
+    const int r0 = rows.r0, r1 = rows.r1;
+    const bool busy = warp < g.NW;
+    const int c = warp % nsl, gr = warp / nsl;
+    const int64_t c0 = (int64_t)c * kSliceCols;
+    const int ucols = (int)min64(kSliceCols, K - c0);
+    const bool active = busy && lane_active<QT>(lane, ucols);
+    XRegs<QT> xr;
+    const XStage xs = xstage_at(sm.xst, K);
+    const float r = w ? stage<true>(h, w, parts, K, g.staged, xs) : stage<false>(h, w, parts, K, g.staged, xs);
+    if (g.staged) {
+      cons_bar();
+      if (active) xr.load(xs, c, lane);
+    } else {
+      if constexpr (QT == QT_Q6_K) {
+        if (active) xr.load_direct(PX{h, w, r}, c, lane);
+      }
+    }
+    // Stage loop.  Shared-memory locations are 32-bit offsets recomputed from
+    // the plan, so the loop keeps few registers beside x and the weights.
+    const uint32_t S = (uint32_t)st.n_slots, Z = (uint32_t)st.slot_bytes, RF = (uint32_t)st.red_floats;
+    const uint32_t o_full = S * Z + (uint32_t)st.xstage_bytes;
+    const uint32_t o_empty = o_full + 8 * S, o_rfull = o_empty + 8 * S, o_rempty = o_rfull + 8 * kPRed;
+    const uint32_t o_red = o_rempty + 8 * kPRed;
+    const volatile int* cta_abort = reinterpret_cast<const volatile int*>(p_smem + o_red + kPRed * RF * 4 + 64 * 8);
+    const uint32_t sb = smem_addr(p_smem);
+    const uint32_t ring_c = (uint32_t)c * QTraits<QT>::SEG;
+    for (int i = 0; i < nst; ++i, ++q) {
+      const uint32_t rslot = (uint32_t)q % kPRed;
+      bool ok = pwait_a(sb + o_full + 8 * s, ph, cta_abort);
+      if (ok && busy) ok = pwait_a(sb + o_rempty + 8 * rslot, (uint32_t)(((q / kPRed) & 1) ^ 1), cta_abort);
+      if (!ok) {
+        if (lane == 0) {
+          atomicExch(sm.misc, 1);
+          atomicExch(st.sync + st.abort_index, 1u);
+        }
+        return false;
+      }
+      if (busy) {
+        const int rs = r0 + i * TR;
+        const int nr = min(TR, r1 - rs);
+        const uint8_t* stg = p_smem + ring_c + (uint32_t)s * Z;
+        float* rd = reinterpret_cast<float*>(p_smem + o_red) + rslot * RF;
+        // the row group that takes the extra rows rotates from stage to stage
+        for (int rr = (gr + nrg - i % nrg) % nrg; rr < nr; rr += nrg) {
+          float v = active ? xr.dot(stg + (uint32_t)rr * (uint32_t)rbytes, lane) : 0.f;
+          v = warp_sum(v);
+          if (lane == 0) rd[rr * nsl + c] = v;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_a(sb + o_empty + 8 * s);
+        mbar_arrive_a(sb + o_rfull + 8 * rslot);
+      }
+      if (++s == (int)S) { s = 0; ph ^= 1u; }
+    }
+    return true;
+  }
+
+  // Block-wide (consumer warps) sum; result valid in every consumer thread.
+  __device__ float csum(float v) {
+    v = warp_sum(v);
+    if (lane == 0) sm.scr[warp] = v;
+    cons_bar();
+    float t = 0.f;
+    for (int w2 = 0; w2 < kPConsumers; ++w2) t += sm.scr[w2];
+    cons_bar();
+    return t;
+  }
+
+  __device__ void embed() {
+    const int tp = st.params[1];
+    int64_t tok = tp >= 0 ? tp : __ldcg(st.token_state);
+    if (tok < 0 || tok >= st.V) {
+      if (blockIdx.x == 0 && ctid == 0) atomicExch(st.status, (int)kStatusBadToken);
+      tok = 0;
+    }
+    const int64_t H = st.H;
+    const int64_t i0 = H * blockIdx.x / gridDim.x, i1 = H * (blockIdx.x + 1) / gridDim.x;
+    float ss = 0.f;
+    for (int64_t i = i0 + ctid; i < i1; i += kPCThreads) {
+      const float v = half_bits_to_float(st.embed[tok * H + i]);
+      st.hidden[i] = v;
+      ss = fmaf(v, v, ss);
+    }
+    ss = csum(ss);
+    if (ctid == 0) st.stats_embed[blockIdx.x * 4] = ss;
+  }
+
+  // Split-KV attention units (kv head, split) of this CTA, then the merge of
+  // every KV head whose last split finished here.  A unit holds at most
+  // kPChunk positions; its K and V rows (contiguous in the cache) come into
+  // shared memory with 16-byte asynchronous copies issued all at once.
+  template <int G>
+  __device__ void attention(const LRow& L, int lk) {
+    const int n_ctx = st.params[0] + 1;
+    const int ns = st.n_split;
+    const int chunk = (n_ctx + ns - 1) / ns;
+    const AttnSmem a = attn_smem(sm.xst, G);
+    const int units = st.Hkv * ns;
+    const int S = kAttnPartStride;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      const int kvh = u / ns, split = u % ns;
+      const int p0 = split * chunk;
+      const int p1 = min(p0 + chunk, n_ctx);
+      const int np = p1 > p0 ? p1 - p0 : 0;
+      // K, V rows p0..p1-1 -> shared memory (np * 256 bytes each)
+      {
+        const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(L.kc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
+        const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(L.vc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
+        const int n16 = np * (kPD * 2 / 16);
+        for (int i = ctid; i < 2 * n16; i += kPCThreads) {
+          const bool isv = i >= n16;
+          const int o = (isv ? i - n16 : i) * 16;
+          cp_async16((isv ? a.v : a.k) + o, (isv ? vsrc : ksrc) + o);
+        }
+        cp_async_commit();
+      }
+      float qr[G][4];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float4 t = __ldcg(reinterpret_cast<const float4*>(st.q + (int64_t)(kvh * G + h) * kPD + 4 * lane));
+        qr[h][0] = t.x; qr[h][1] = t.y; qr[h][2] = t.z; qr[h][3] = t.w;
+      }
+      cp_async_wait_all();
+      cons_bar();
+      // scores: a warp per position, lanes split the head dimension
+      for (int i = warp; i < np; i += kPConsumers) {
+        const uint2 kr = *reinterpret_cast<const uint2*>(a.k + (size_t)i * kPD * 2 + 8 * lane);
+        const float k0 = half_bits_to_float(kr.x), k1 = half_bits_to_float(kr.x >> 16);
+        const float k2 = half_bits_to_float(kr.y), k3 = half_bits_to_float(kr.y >> 16);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float d = qr[h][0] * k0;
+          d = fmaf(qr[h][1], k1, d);
+          d = fmaf(qr[h][2], k2, d);
+          d = fmaf(qr[h][3], k3, d);
+          d = warp_sum(d);
+          if (lane == 0) a.sc[h * kPChunk + i] = d * kAttnScale;
+        }
+      }
+      cons_bar();
+      for (int h = warp; h < G; h += kPConsumers) {
+        float m = -INFINITY;
+        for (int i = lane; i < np; i += 32) m = fmaxf(m, a.sc[h * kPChunk + i]);
+        m = warp_max(m);
+        float l = 0.f;
+        for (int i = lane; i < np; i += 32) {
+          const float e = expf(a.sc[h * kPChunk + i] - m);
+          a.sc[h * kPChunk + i] = e;
+          l += e;
+        }
+        l = warp_sum(l);
+        if (lane == 0) { a.ml[2 * h] = m; a.ml[2 * h + 1] = l; }
+      }
+      cons_bar();
+      // P V: thread (h, d2) accumulates dims 2 d2, 2 d2 + 1 of head h
+      for (int idx = ctid; idx < G * (kPD / 2); idx += kPCThreads) {
+        const int h = idx / (kPD / 2), d2 = idx % (kPD / 2);
+        const float* e = a.sc + h * kPChunk;
+        float o0 = 0.f, o1 = 0.f;
+        for (int i = 0; i < np; ++i) {
+          const uint32_t wv = *reinterpret_cast<const uint32_t*>(a.v + (size_t)i * kPD * 2 + 4 * d2);
+          o0 = fmaf(e[i], half_bits_to_float(wv), o0);
+          o1 = fmaf(e[i], half_bits_to_float(wv >> 16), o1);
+        }
+        float* dst = st.attn_part + ((int64_t)(kvh * G + h) * ns + split) * S;
+        *reinterpret_cast<float2*>(dst + 2 + 2 * d2) = make_float2(o0, o1);
+        if (d2 == 0) {
+          dst[0] = np > 0 ? a.ml[2 * h] : -INFINITY;
+          dst[1] = np > 0 ? a.ml[2 * h + 1] : 0.f;
+        }
+      }
+      // publish this split (release by one thread after the CTA barrier)
+      cons_bar();
+      if (ctid == 0) {
+        const unsigned old = atom_acq_rel_add(st.sync + st.head_ctr_index + lk * st.Hkv + kvh, 1u);
+        sm.misc[3] = old == (unsigned)(ns - 1);
+      }
+      cons_bar();
+      if (sm.misc[3]) {
+        // (m, l) of every split: one warp per query head, 4 loads per lane in flight
+        for (int h = warp; h < G; h += kPConsumers) {
+          const float* ph0 = st.attn_part + (int64_t)(kvh * G + h) * ns * S;
+          float M = -INFINITY;
+          for (int t0 = 0; t0 < ns; t0 += 32 * kPSplitsPerRound) {
+            float mv[kPSplitsPerRound];
+#pragma unroll
+            for (int k = 0; k < kPSplitsPerRound; ++k) {
+              const int t = t0 + lane + 32 * k;
+              mv[k] = t < ns ? __ldcg(ph0 + (int64_t)t * S) : -INFINITY;
+            }
+#pragma unroll
+            for (int k = 0; k < kPSplitsPerRound; ++k) M = fmaxf(M, mv[k]);
+          }
+          M = warp_max(M);
+          float Ls = 0.f;
+          for (int t0 = 0; t0 < ns; t0 += 32 * kPSplitsPerRound) {
+            float mv[kPSplitsPerRound], lv[kPSplitsPerRound];
+#pragma unroll
+            for (int k = 0; k < kPSplitsPerRound; ++k) {
+              const int t = t0 + lane + 32 * k;
+              mv[k] = t < ns ? __ldcg(ph0 + (int64_t)t * S) : -INFINITY;
+              lv[k] = t < ns ? __ldcg(ph0 + (int64_t)t * S + 1) : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < kPSplitsPerRound; ++k) {
+              const int t = t0 + lane + 32 * k;
+              const float wgt = mv[k] == -INFINITY ? 0.f : expf(mv[k] - M);
+              Ls = fmaf(wgt, lv[k], Ls);
+              if (t < ns) a.sw[h * ns + t] = wgt;
+            }
+          }
+          Ls = warp_sum(Ls);
+          if (lane == 0) a.ml[2 * h + 1] = Ls;  // this unit's own (m, l) are already stored
+        }
+        cons_bar();
+        for (int idx = ctid; idx < G * kPD; idx += kPCThreads) {
+          const int h = idx / kPD, d = idx % kPD;
+          const float* ph0 = st.attn_part + (int64_t)(kvh * G + h) * ns * S + 2 + d;
+          const float* wt = a.sw + h * ns;
+          float O = 0.f;
+          for (int t = 0; t < ns; t += 8) {
+            float v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = t + k < ns ? __ldcg(ph0 + (int64_t)(t + k) * S) : 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              if (t + k < ns) O = fmaf(wt[t + k], v[k], O);
+          }
+          st.attn_out[(int64_t)(kvh * G + h) * kPD + d] = O / a.ml[2 * h + 1];
+        }
+      }
+      cons_bar();  // scratch reuse by the next unit
+    }
+  }
+};
+
+template <int QT>
+__global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_constant__ PStep st) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const PSmem sm = psmem_at(p_smem, st.n_slots, st.slot_bytes, st.xstage_bytes, st.red_floats, st.n_layers);
+  const int n = st.n_layers;
+  const int np = 2 + 5 * n;
+  const unsigned G = gridDim.x;
+  unsigned* gabort = st.sync + st.abort_index;
+
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < st.n_slots; ++k) {
+      mbar_init(sm.full + k, 1);
+      mbar_init(sm.empty + k, kPConsumers);
+    }
+    for (int k = 0; k < kPRed; ++k) {
+      mbar_init(sm.rfull + k, kPConsumers);
+      mbar_init(sm.rempty + k, 1);
+    }
+    sm.misc[0] = 0;
+    fence_barrier_init();
+  }
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const PLayer& Lg = st.layers[k];
+    sm.lt[k] = LRow{Lg.attn_norm, Lg.ffn_norm, Lg.stats_down, Lg.kc, Lg.vc};
+  }
+  if (threadIdx.x < 7) {
+    const int kind = threadIdx.x;
+    if (kind == PK_QKV || kind == PK_O || kind == PK_GU || kind == PK_DOWN || kind == PK_HEAD)
+      sm.kg[kind] = KGeo{st.g[kind], phase_rows(st, kind)};
+  }
+  // RMSNorm weights into L2 now, so that a phase start finds them there
+  // (layer k's two vectors by CTA k mod grid, the final norm by the next one).
+  if (warp == kPCopyWarp && lane == 0) {
+    const uint32_t nb = (uint32_t)st.H * 4;
+    for (int k = blockIdx.x; k <= n; k += gridDim.x) {
+      if (k < n) {
+        l2_prefetch(st.layers[k].attn_norm, nb);
+        l2_prefetch(st.layers[k].ffn_norm, nb);
+      } else {
+        l2_prefetch(st.final_norm, nb);
+      }
+    }
+  }
+  // RoPE table of this step's position (the same for every layer)
+  if (warp == kPEpiWarp) {
+    const int pos = st.params[0];
+    for (int i = lane; i < kPD / 2; i += 32) {
+      const double inv_freq = pow((double)st.theta, -2.0 * (double)i / (double)kPD);
+      double sn, cn;
+      sincos((double)pos * inv_freq, &sn, &cn);
+      sm.rope[i] = make_float2((float)cn, (float)sn);
+    }
+  }
+  __syncthreads();
+
+  if (warp == kPCopyWarp) {
+    Copier cp(st, sm, lane, np);
+    cp.run();
+  } else if (warp == kPEpiWarp) {
+    // ---------------------------------------------------------- epilogue
+    Epilogue ep(st, sm, lane);
+    bool ok = true;
+    for (int p = 1; p < np && ok; ++p) {
+      const int kind = phase_kind(p, n);
+      if (kind == PK_ATTN) continue;
+      const LRow* L = (p >= 1 && p < 1 + 5 * n) ? sm.lt + (p - 1) / 5 : nullptr;
+      const PRows rows = sm.kg[kind].rows;
+      const PGeom g = sm.kg[kind].g;
+      // the epilogue reads what earlier phases wrote
+      int wok = 1;
+      if (lane == 0) wok = grid_wait(st.sync + (p - 1), G, gabort, st.status);
+      if (!__shfl_sync(0xffffffffu, wok, 0)) { ok = false; break; }
+      switch (kind) {
+        case PK_QKV: {
+          EpiQKV epi{st.q, L->kc, L->vc, nullptr, st.params[0], (int64_t)st.Hq * st.D, (int64_t)st.Hkv * st.D,
+                     st.D, st.max_ctx, st.theta, sm.rope};
+          ok = ep.run(epi, rows, g);
+          break;
+        }
+        case PK_O: {
+          if (rows.r1 - rows.r0 <= 64) {
+            PEpiResid epi{st.h1, st.hidden, nullptr, st.stats_o};
+            ok = ep.run_resid(epi, rows, g);
+            if (ok) epi.finish(lane);
+          } else {
+            EpiResid epi{st.h1, st.hidden, nullptr, st.stats_o};
+            epi.init(nullptr, lane);
+            ok = ep.run(epi, rows, g);
+            if (ok) epi.finish(lane);
+          }
+          break;
+        }
+        case PK_GU: {
+          EpiSwiGLU epi{st.u};
+          ok = ep.run(epi, rows, g);
+          break;
+        }
+        case PK_DOWN: {
+          if (rows.r1 - rows.r0 <= 64) {
+            PEpiResid epi{st.hidden, st.h1, st.hidden, L->stats_down};
+            ok = ep.run_resid(epi, rows, g);
+            if (ok) epi.finish(lane);
+          } else {
+            EpiResid epi{st.hidden, st.h1, st.hidden, L->stats_down};
+            epi.init(nullptr, lane);
+            ok = ep.run(epi, rows, g);
+            if (ok) epi.finish(lane);
+          }
+          break;
+        }
+        default: {
+          EpiArgmax epi{st.logits, st.arg_parts};
+          epi.init(nullptr, lane);
+          ok = ep.run(epi, rows, g);
+          if (ok) epi.finish(lane);
+          break;
+        }
+      }
+      if (!ok) break;
+      // publish (release by lane 0 after the warp barrier); the last CTA
+      // through the head phase picks the greedy token
+      __syncwarp();
+      unsigned old = 0;
+      if (lane == 0) {
+        if (kind == PK_HEAD) old = atom_acq_rel_add(st.sync + p, 1u);
+        else red_release_add(st.sync + p, 1u);
+      }
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (kind == PK_HEAD && old == G - 1) {
+        float b = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int i = lane; i < (int)G; i += 32) {
+          const float v = __ldcg(st.arg_parts + i * 4);
+          const int vi = __ldcg(reinterpret_cast<const int*>(st.arg_parts) + i * 4 + 1);
+          if (vi < 0) continue;
+          if (v > b || (v == b && vi < bi)) { b = v; bi = vi; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ob = __shfl_xor_sync(0xffffffffu, b, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (ob > b || (ob == b && oi < bi)) { b = ob; bi = oi; }
+        }
+        if (lane == 0) {
+          *st.token_state = bi;
+          if (st.next_token) *st.next_token = bi;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      atomicExch(sm.misc, 1);
+      atomicExch(gabort, 1u);
+    }
+  } else {
+    // ---------------------------------------------------------- consumers
+    Consumer<QT> cs(st, sm, warp, lane);
+    const int ctid = cs.ctid;
+    for (int p = 0; p < np; ++p) {
+      const int kind = phase_kind(p, n);
+      int* go = sm.misc + 1 + (p & 1);
+      if (ctid == 0) {
+        bool ok = !*reinterpret_cast<volatile int*>(sm.misc);
+        if (ok && p > 0) ok = grid_wait(st.sync + (p - 1), G, gabort, st.status);
+        if (!ok) atomicExch(sm.misc, 1);  // the other warps stop waiting for these
+        *go = ok;
+      }
+      cons_bar();
+      if (!*go) break;
+      const LRow* L = (p >= 1 && p < 1 + 5 * n) ? sm.lt + (p - 1) / 5 : nullptr;
+      switch (kind) {
+        case PK_EMBED:
+          cs.embed();
+          break;
+        case PK_ATTN: {
+          const int Gq = st.Hq / st.Hkv, lk = (p - 1) / 5;
+          if (Gq == 8) cs.template attention<8>(*L, lk);
+          else if (Gq == 4) cs.template attention<4>(*L, lk);
+          else if (Gq == 2) cs.template attention<2>(*L, lk);
+          else cs.template attention<1>(*L, lk);
+          break;
+        }
+        default: {  // GEMV phases
+          const bool norm = kind == PK_QKV || kind == PK_GU || kind == PK_HEAD;
+          const float* h = kind == PK_GU ? st.h1 : kind == PK_O ? st.attn_out : kind == PK_DOWN ? st.u : st.hidden;
+          const float* w = nullptr;
+          const float* parts = nullptr;
+          if (norm) {
+            w = kind == PK_QKV ? L->attn_norm : (kind == PK_GU ? L->ffn_norm : st.final_norm);
+            parts = kind == PK_GU ? st.stats_o
+                    : (p == 1 || (kind == PK_HEAD && n == 0)) ? st.stats_embed
+                                                             : sm.lt[(p - 2) / 5].stats_down;
+          }
+          cs.gemv(kind, h, w, parts);  // a failed wait raised the CTA abort flag
+          break;
+        }
+      }
+      if (kind == PK_EMBED || kind == PK_ATTN) {
+        // publish (release by one thread after the CTA barrier)
+        cons_bar();
+        if (ctid == 0) red_release_add(st.sync + p, 1u);
+      }
+    }
+  }
+}
+
+std::mutex g_pmu;
+
+}  // namespace
+
+// Host-side plan: slot size, stages, per-phase geometry.
+int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int max_ctx, int grid, int n_layers,
+                 PStep* st, size_t* smem) {
+  (void)V;
+  if (D != kPD) return -1;
+  if (Hkv <= 0 || Hq % Hkv) return -1;
+  const int Gq = Hq / Hkv;
+  if (Gq != 1 && Gq != 2 && Gq != 4 && Gq != 8) return -1;
+  const int be = qtype == QT_Q6_K ? 256 : 32, bb = qtype == QT_Q6_K ? 210 : (qtype == QT_Q8_0 ? 34 : 18);
+  const int64_t KO = (int64_t)Hq * D;
+  struct KInfo {
+    int kind;
+    int64_t K;
+    int align;
+  } ks[5] = {{PK_QKV, H, 2}, {PK_O, KO, 1}, {PK_GU, H, 2}, {PK_DOWN, F, 1}, {PK_HEAD, H, 1}};
+  for (auto& k : ks) {
+    const bool fixed = qtype != QT_Q6_K;
+    if (fixed ? (k.K % 256) : (k.K % 2048)) return -1;
+    if (k.K > (int64_t)kPConsumers * kSliceCols) return -1;
+    PGeom& g = st->g[k.kind];
+    g.align = k.align;
+    g.row_bytes = (int)(k.K / be * bb);
+    g.n_slices = (int)((k.K + kSliceCols - 1) / kSliceCols);
+  }
+  // attention scratch lives in the x staging region
+  const int ns = persist_splits(grid, Hkv, max_ctx);
+  const int attn_bytes = (int)((attn_smem_bytes(Gq, ns) + 15) / 16 * 16);
+  const int smem_max = 227 * 1024;
+  // Choose the slot size.  In order of priority: every phase can use all its
+  // row groups (TR >= consumer warps per slice), at least 3 slots, the most
+  // bytes in flight in the worst phase, then the smaller slot.
+  int best_Z = 0, best_S = 0;
+  int64_t best_key[4] = {-1, -1, -1, -1};
+  for (auto& kz : ks) {
+    const int rbz = st->g[kz.kind].row_bytes;
+    for (int m = 1; m <= kPMaxTR; ++m) {
+      const int Z = m * rbz;
+      int xbz = attn_bytes, rf = 0;
+      int64_t inflight_min = INT64_MAX;
+      bool okz = true, full_rg = true;
+      int TRs[8];
+      for (auto& k : ks) {
+        PGeom& g = st->g[k.kind];
+        int tr = Z / g.row_bytes;
+        if (tr > kPMaxTR) tr = kPMaxTR;
+        if (k.align == 2) tr &= ~1;
+        if (tr < 1) { okz = false; break; }
+        TRs[k.kind] = tr;
+        int nrg_max = kPConsumers / g.n_slices;
+        if (nrg_max < 1) nrg_max = 1;
+        if (tr < nrg_max) full_rg = false;
+        const int nrg = nrg_max > tr ? tr : nrg_max;
+        const bool staged = qtype != QT_Q6_K || nrg > 1;
+        if (staged) {
+          const int b = (int)((xstage_bytes(qtype, k.K) + 15) / 16 * 16);
+          if (b > xbz) xbz = b;
+        }
+        if (tr * g.n_slices > rf) rf = tr * g.n_slices;
+      }
+      if (!okz) continue;
+      xbz = (xbz + 15) / 16 * 16;
+      int S = 0;
+      while (psmem_bytes(S + 1, Z, xbz, (rf + 3) / 4 * 4, n_layers) <= (size_t)smem_max && S + 1 <= 16) ++S;
+      if (S < 2) continue;
+      for (auto& k : ks) {
+        const int64_t inflight = (int64_t)S * TRs[k.kind] * st->g[k.kind].row_bytes;
+        if (inflight < inflight_min) inflight_min = inflight;
+      }
+      const int64_t key[4] = {full_rg ? 1 : 0, S >= 3 ? 1 : 0, inflight_min, -(int64_t)Z};
+      bool better = false;
+      for (int i = 0; i < 4; ++i) {
+        if (key[i] != best_key[i]) { better = key[i] > best_key[i]; break; }
+      }
+      if (better) {
+        for (int i = 0; i < 4; ++i) best_key[i] = key[i];
+        best_Z = Z;
+        best_S = S;
+      }
+    }
+  }
+  if (best_Z == 0) return -1;
+  int rf = 0, xbz = attn_bytes;
+  for (auto& k : ks) {
+    PGeom& g = st->g[k.kind];
+    int tr = best_Z / g.row_bytes;
+    if (tr > kPMaxTR) tr = kPMaxTR;
+    if (k.align == 2) tr &= ~1;
+    g.TR = tr;
+    int nrg = kPConsumers / g.n_slices;
+    if (nrg < 1) nrg = 1;
+    if (nrg > tr) nrg = tr;
+    g.n_rg = nrg;
+    g.NW = g.n_slices * nrg;
+    g.staged = qtype != QT_Q6_K || nrg > 1;
+    if (g.staged) {
+      const int b = (int)((xstage_bytes(qtype, k.K) + 15) / 16 * 16);
+      if (b > xbz) xbz = b;
+    }
+    if (tr * g.n_slices > rf) rf = tr * g.n_slices;
+  }
+  st->slot_bytes = best_Z;
+  st->n_slots = best_S;
+  st->xstage_bytes = (xbz + 15) / 16 * 16;
+  st->red_floats = (rf + 3) / 4 * 4;  // keeps the tables after it 16-byte aligned
+  *smem = psmem_bytes(best_S, best_Z, st->xstage_bytes, st->red_floats, n_layers);
+  return 0;
+}
+
+cudaError_t launch_persist(int qtype, const PStep& st, size_t smem, int grid, cudaStream_t s) {
+  static unsigned long long done[3] = {0, 0, 0};
+  void (*kern)(const PStep) = qtype == QT_Q8_0 ? persist_kernel<QT_Q8_0>
+                        : qtype == QT_Q4_0 ? persist_kernel<QT_Q4_0>
+                                           : persist_kernel<QT_Q6_K>;
+  const int ki = qtype == QT_Q8_0 ? 0 : qtype == QT_Q4_0 ? 1 : 2;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(done[ki] & (1ull << dev))) {
+    std::lock_guard<std::mutex> g(g_pmu);
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    done[ki] |= 1ull << dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident at once (grid-wide waits)
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, st);
+}
+
+int persist_grid(int qtype, size_t smem) {
+  void (*kern)(const PStep) = qtype == QT_Q8_0 ? persist_kernel<QT_Q8_0>
+                        : qtype == QT_Q4_0 ? persist_kernel<QT_Q4_0>
+                                           : persist_kernel<QT_Q6_K>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess) return 0;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPThreads, smem) != cudaSuccess) return 0;
+  const int g = sm_count();
+  return per_sm >= 1 && g <= 32 * kPPartsPerLane ? g : 0;
+}
+
+}  // namespace ntx

@@ -6,8 +6,11 @@
   GPU's greedy token must be the oracle's argmax wherever the oracle's top two
   logits are more than twice that tolerance apart.
 * CUDA-graph replay and kernel-by-kernel launch give bit-identical logits;
-  tiered (pinned-host layers streamed through two slots) and resident runs
-  give bit-identical logits.
+  tiered (pinned-host layers streamed through two slots) and resident runs of
+  the per-op kernel chain give bit-identical logits.
+* The persistent decode kernel (the default for all-resident models) and the
+  per-op kernel chain each match the oracle; one launch per step.  A long
+  context with query group 8 makes more attention units than CTAs.
 * Cosine skip: calibration cosines within 1e-5 of the oracle's, skip
   decisions equal wherever |cos - tau| > 1e-4, and later steps with the skip set
   applied match the oracle run with the same set.
@@ -140,20 +143,43 @@ def check_logits(got, ref, greedy, step):
         assert greedy == int(np.argmax(ref)), f"step {step}: greedy {greedy} vs oracle {int(np.argmax(ref))}"
 
 
-def test_engine_tiny_teacher_forced_graph_and_nograph():
+@pytest.mark.parametrize("chain", [False, True], ids=["persistent", "per_op_chain"])
+def test_engine_tiny_teacher_forced_graph_and_nograph(chain):
     m = DeviceModel(TINY, ntx.NTX_Q8_0, ntx.NTX_Q8_0, 41, max_ctx=32, n_prior=0, source="host")
     prompt = sg.tokens(41, "prompt", 6, TINY["vocab"])
     toks = list(prompt) + [-1] * 10
+    f = ntx.NTX_NO_PERSIST if chain else 0
     e = Engine(m)
-    lg_g, fed, nxt, _ = e.run(toks)
+    lg_g, fed, nxt, _ = e.run(toks, flags=f)
+    launches = ntx.ntx_engine_launches_per_step(e.h)
     m.reset_kv()
-    lg_n, fed_n, _, _ = e.run(toks, flags=ntx.NTX_NO_GRAPH)
+    lg_n, fed_n, _, _ = e.run(toks, flags=f | ntx.NTX_NO_GRAPH)
     e.close()
+    assert launches == (1 + 5 * TINY["n_layers"] + 2 if chain else 1)
     assert fed == fed_n
     assert np.array_equal(lg_g, lg_n)
     ref, _ = oracle_run(m, fed)
     for s in range(len(fed)):
         check_logits(lg_g[s], ref[s], int(nxt[s]), s)
+
+
+@pytest.mark.parametrize("qtype,d,max_ctx,n_prior", [
+    (ntx.NTX_Q8_0, dict(TINY, n_heads=16, n_kv_heads=2, n_layers=2), 20000, 19990),
+    (ntx.NTX_Q4_0, dict(TINY, n_heads=4, n_kv_heads=4, n_layers=2), 600, 590),
+    (ntx.NTX_Q6_K, dict(TINY, hidden=2048, n_heads=16, n_kv_heads=8, ffn=6144, n_layers=2), 300, 290),
+], ids=["q8_0_g8_ctx20000", "q4_0_g1_ctx600", "q6_k_g2_ctx300"])
+def test_engine_persistent_long_context(qtype, d, max_ctx, n_prior):
+    """Persistent kernel at contexts where a (KV head, split) unit holds many
+    positions and (first case) there are more units than CTAs."""
+    m = DeviceModel(d, qtype, qtype, 49, max_ctx=max_ctx, n_prior=n_prior, source="host")
+    toks = list(sg.tokens(49, "prompt", 2, d["vocab"])) + [-1] * 2
+    e = Engine(m)
+    lg, fed, nxt, _ = e.run(toks, pos0=n_prior)
+    assert ntx.ntx_engine_launches_per_step(e.h) == 1
+    e.close()
+    ref, _ = oracle_run(m, fed, pos0=n_prior, nthreads=os.cpu_count())
+    for s in range(len(fed)):
+        check_logits(lg[s], ref[s], int(nxt[s]), s)
 
 
 @pytest.mark.parametrize("qtype,d", [(ntx.NTX_Q4_0, TINY),
@@ -181,11 +207,17 @@ def test_engine_tiered_equals_resident():
     et.close()
     m.reset_kv()
     er = Engine(m, use_resident_copy=True)
-    lg_r, fed_r, _, _ = er.run(toks, pos0=3)
+    lg_r, fed_r, _, _ = er.run(toks, pos0=3, flags=ntx.NTX_NO_PERSIST)
+    m.reset_kv()
+    lg_p, fed_p, nxt_p, _ = er.run(toks, pos0=3)  # the persistent kernel
     er.close()
     assert fed_t == fed_r
     assert np.array_equal(lg_t, lg_r)
     assert np.array_equal(lg_tn, lg_r)
+    m.reset_kv()
+    ref, _ = oracle_run(m, fed_p, pos0=3)
+    for s in range(len(fed_p)):
+        check_logits(lg_p[s], ref[s], int(nxt_p[s]), s)
 
 
 def test_engine_cosine_skip_calibration():
