@@ -453,8 +453,17 @@ struct Epilogue {
     red_floats = st.red_floats;
   }
 
+  // 1/rms of the phase's input from the per-CTA sum-of-squares partials
+  // (RMSNorm(h) w x = (1/rms) sum_j W_ij w_j h_j: the consumers staged w h).
+  __device__ float rms_scale(const float* parts) const {
+    float ss = 0.f;
+    for (int i = lane; i < (int)gridDim.x; i += 32) ss += __ldcg(parts + (int64_t)i * 4);
+    ss = warp_sum(ss);
+    return 1.0f / sqrtf(ss / (float)st.H + st.eps);
+  }
+
   template <class Epi>
-  __device__ bool run(Epi& epi, const PRows rows, const PGeom g) {
+  __device__ bool run(Epi& epi, const PRows rows, const PGeom g, float scale = 1.f) {
     constexpr int A = Epi::kAlign;
     const int TR = g.TR, nsl = g.n_slices, nst = rows.n;
     const int64_t r0 = rows.r0, r1 = rows.r1;
@@ -476,6 +485,8 @@ struct Epilogue {
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.rempty + slot);
+      a *= scale;
+      b *= scale;
       epi.rotate();
       if (i + 1 < nst) epi.preload(rs + TR, (int)min64(TR, r1 - rs - TR), lane);
       if (mine) epi.apply(rs + row_a, a, b);
@@ -519,67 +530,35 @@ struct Consumer {
   __device__ Consumer(const PStep& st_, PSmem sm_, int warp_, int lane_)
       : st(st_), sm(sm_), warp(warp_), lane(lane_), ctid(warp_ * 32 + lane_), s(0), ph(0), q(0) {}
 
-  // x of a GEMV phase into shared memory (fixed-point limbs or fp32): x = h, or
-  // RMSNorm(h) w with the scale from the per-CTA sum-of-squares partials.  The
-  // partials and the first batch of h (and w) are requested together, so the
-  // staging costs one round trip to L2 for the shapes used here.  Returns the
-  // RMSNorm scale (1 without a norm).
+  // x of a GEMV phase into shared memory (fixed-point limbs or fp32): x = h,
+  // or w h for a phase with an RMSNorm prologue -- the 1/rms scale is applied
+  // to each row's result by the epilogue warp, so staging waits for nothing but
+  // one batch of loads (h, and w).
   template <bool NORM>
-  __device__ float stage(const float* h, const float* w, const float* parts, int64_t K, bool staged,
-                         const XStage& xs) {
+  __device__ void stage(const float* h, const float* w, int64_t K, const XStage& xs) {
     constexpr int kBatch = NORM ? 4 : 8;
     const int nchunk = (int)(K / 128);
-    float pp[kPPartsPerLane];
-    if constexpr (NORM) {
-#pragma unroll
-      for (int k = 0; k < kPPartsPerLane; ++k) {
-        const int i = lane + 32 * k;
-        pp[k] = i < (int)gridDim.x ? __ldcg(parts + (int64_t)i * 4) : 0.f;
-      }
-    }
-    float4 hv[kBatch], wv[NORM ? kBatch : 1];
-    if (staged) {
+    for (int ch0 = warp; ch0 < nchunk; ch0 += kBatch * kPConsumers) {
+      float4 hv[kBatch], wv[NORM ? kBatch : 1];
 #pragma unroll
       for (int b = 0; b < kBatch; ++b) {
-        const int ch = warp + b * kPConsumers;
+        const int ch = ch0 + b * kPConsumers;
         const int64_t col = (int64_t)ch * 128 + 4 * lane;
         hv[b] = ch < nchunk ? __ldcg(reinterpret_cast<const float4*>(h + col)) : make_float4(0.f, 0.f, 0.f, 0.f);
         if constexpr (NORM) wv[b] = ch < nchunk ? ldg4(w + col) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-    }
-    float r = 1.f;
-    if constexpr (NORM) {
-      float ss = 0.f;
-#pragma unroll
-      for (int k = 0; k < kPPartsPerLane; ++k) ss += pp[k];
-      ss = warp_sum(ss);
-      r = 1.0f / sqrtf(ss / (float)st.H + st.eps);
-    }
-    if (!staged) return r;
-    const PX pro{h, NORM ? w : nullptr, r};
-    for (int ch0 = warp;; ch0 += kBatch * kPConsumers) {
 #pragma unroll
       for (int b = 0; b < kBatch; ++b) {
         const int ch = ch0 + b * kPConsumers;
         if (ch >= nchunk) break;  // uniform across the warp
         float4 v = hv[b];
-        if constexpr (NORM) {
-          if (ch0 == warp)  // only the first batch still needs the norm applied
-            v = make_float4(wv[b].x * (v.x * r), wv[b].y * (v.y * r), wv[b].z * (v.z * r), wv[b].w * (v.w * r));
-        }
+        if constexpr (NORM) v = make_float4(wv[b].x * v.x, wv[b].y * v.y, wv[b].z * v.z, wv[b].w * v.w);
         stage_chunk<QT>(v, (int64_t)ch * 128 + 4 * lane, xs, lane);
       }
-      if (ch0 + kBatch * kPConsumers >= nchunk) break;
-#pragma unroll
-      for (int b = 0; b < kBatch; ++b) {
-        const int ch = ch0 + (kBatch + b) * kPConsumers;
-        hv[b] = ch < nchunk ? pro.ld((int64_t)ch * 128 + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
     }
-    return r;
   }
 
-  __device__ bool gemv(int kind, const float* h, const float* w, const float* parts) {
+  __device__ bool gemv(int kind, const float* h, const float* w) {
     const PGeom g = sm.kg[kind].g;
     const PRows rows = sm.kg[kind].rows;
     const int64_t K = phase_K(st, kind);
@@ -592,13 +571,14 @@ struct Consumer {
     const bool active = busy && lane_active<QT>(lane, ucols);
     XRegs<QT> xr;
     const XStage xs = xstage_at(sm.xst, K);
-    const float r = w ? stage<true>(h, w, parts, K, g.staged, xs) : stage<false>(h, w, parts, K, g.staged, xs);
     if (g.staged) {
+      if (w) stage<true>(h, w, K, xs);
+      else stage<false>(h, w, K, xs);
       cons_bar();
       if (active) xr.load(xs, c, lane);
     } else {
       if constexpr (QT == QT_Q6_K) {
-        if (active) xr.load_direct(PX{h, w, r}, c, lane);
+        if (active) xr.load_direct(PX{h, w, 1.f}, c, lane);
       }
     }
     // Stage loop.  Shared-memory locations are 32-bit offsets recomputed from
@@ -894,11 +874,15 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
       int wok = 1;
       if (lane == 0) wok = grid_wait(st.sync + (p - 1), G, gabort, st.status);
       if (!__shfl_sync(0xffffffffu, wok, 0)) { ok = false; break; }
+      // RMSNorm phases: the sum-of-squares partials of the phase input
+      const float* parts = kind == PK_GU ? st.stats_o
+                           : (p == 1 || (kind == PK_HEAD && n == 0)) ? st.stats_embed
+                                                                    : sm.lt[(p - 2) / 5].stats_down;
       switch (kind) {
         case PK_QKV: {
           EpiQKV epi{st.q, L->kc, L->vc, nullptr, st.params[0], (int64_t)st.Hq * st.D, (int64_t)st.Hkv * st.D,
                      st.D, st.max_ctx, st.theta, sm.rope};
-          ok = ep.run(epi, rows, g);
+          ok = ep.run(epi, rows, g, ep.rms_scale(parts));
           break;
         }
         case PK_O: {
@@ -916,7 +900,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
         }
         case PK_GU: {
           EpiSwiGLU epi{st.u};
-          ok = ep.run(epi, rows, g);
+          ok = ep.run(epi, rows, g, ep.rms_scale(parts));
           break;
         }
         case PK_DOWN: {
@@ -935,7 +919,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
         default: {
           EpiArgmax epi{st.logits, st.arg_parts};
           epi.init(nullptr, lane);
-          ok = ep.run(epi, rows, g);
+          ok = ep.run(epi, rows, g, ep.rms_scale(parts));
           if (ok) epi.finish(lane);
           break;
         }
@@ -1004,17 +988,10 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
           break;
         }
         default: {  // GEMV phases
-          const bool norm = kind == PK_QKV || kind == PK_GU || kind == PK_HEAD;
           const float* h = kind == PK_GU ? st.h1 : kind == PK_O ? st.attn_out : kind == PK_DOWN ? st.u : st.hidden;
-          const float* w = nullptr;
-          const float* parts = nullptr;
-          if (norm) {
-            w = kind == PK_QKV ? L->attn_norm : (kind == PK_GU ? L->ffn_norm : st.final_norm);
-            parts = kind == PK_GU ? st.stats_o
-                    : (p == 1 || (kind == PK_HEAD && n == 0)) ? st.stats_embed
-                                                             : sm.lt[(p - 2) / 5].stats_down;
-          }
-          cs.gemv(kind, h, w, parts);  // a failed wait raised the CTA abort flag
+          const float* w = kind == PK_QKV ? L->attn_norm : kind == PK_GU ? L->ffn_norm
+                           : kind == PK_HEAD ? st.final_norm : nullptr;
+          cs.gemv(kind, h, w);  // a failed wait raised the CTA abort flag
           break;
         }
       }
