@@ -161,6 +161,8 @@ def run_ntx(args, dist: Dist):
 
     wk = WORKLOADS[args.workload]
     d = dict(getattr(wl, wk["model"]))
+    if args.layers is not None:
+        d["n_layers"] = args.layers
     L = d["n_layers"]
     qt, hqt = wk["qtype"], wk["head_qtype"]
     sd = wl.seed(wk["workload_id"])
@@ -169,7 +171,7 @@ def run_ntx(args, dist: Dist):
     tier_map = [0] * L
     if wk["tiers"]:
         a, b = (int(t) for t in wk["tiers"].split("-"))
-        for l in range(a, b + 1):
+        for l in range(a, min(b + 1, L)):
             tier_map[l] = 1
     m = DeviceModel(d, qt, hqt, sd, wk["max_ctx"], wk["n_prior"], tier_map=tier_map, source="device")
     cfg = ntx.make_config(d["hidden"], d["n_heads"], d["n_kv_heads"], d["head_dim"], d["ffn"], d["vocab"], L,
@@ -329,11 +331,12 @@ def run_ntx(args, dist: Dist):
     bpt = wl.bytes_per_token(d, qt, hqt, p_first + span // 2)
     ntx.ntx_engine_destroy(eng)
     torch.cuda.synchronize()
+    desc = wk["desc"] if args.layers is None else f"{wk['desc']} -- layer count overridden to {L} (profiling only)"
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "tok/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; random-init weights of the named shapes)",
-        "config": {"workload": wk["desc"], "weights": {8: "Q8_0", 14: "Q6_K", 2: "Q4_0"}[qt], "layers": L,
+        "config": {"workload": desc, "weights": {8: "Q8_0", 14: "Q6_K", 2: "Q4_0"}[qt], "layers": L,
                    "hidden": d["hidden"], "ffn": d["ffn"], "vocab": d["vocab"], "batch": 1,
                    "parallelism": f"replicas x{dist.world}" if dist.world > 1 else "single GPU",
                    "l2": "weights per step >> 126 MB L2 (inputs larger than L2; no flush)",
@@ -441,6 +444,8 @@ def run_reference(args, dist: Dist):
 
     wk = WORKLOADS[args.workload]
     d = dict(getattr(wl, wk["model"]))
+    if args.layers is not None:
+        d["n_layers"] = args.layers
     L = d["n_layers"]
     qt, hqt = wk["qtype"], wk["head_qtype"]
     sd = wl.seed(wk["workload_id"])
@@ -484,6 +489,9 @@ def main():
     ap.add_argument("--no-gemv", action="store_true", help="skip the config 1-2 GEMV sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-chain", action="store_true", help="skip timing the per-op kernel chain for comparison")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="profiling only: run the workload's model with this many layers (the line then describes "
+                         "that smaller model and is not a benchmark of the named workload)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture (reported as is)")
     args = ap.parse_args()

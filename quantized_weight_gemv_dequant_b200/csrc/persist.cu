@@ -261,14 +261,15 @@ __device__ __forceinline__ PSmem psmem_at(uint8_t* base, int S, int Z, int XB, i
 
 // Attention scratch inside the x staging region (consumer warps only).
 struct AttnSmem {
-  uint8_t* k;   // [kPChunk][128] fp16
-  uint8_t* v;   // [kPChunk][128] fp16
-  float* sc;    // [G][kPChunk] scores, then probabilities
-  float* ml;    // [G][2]
-  float* sw;    // [G][ns] merge weights
+  uint8_t* k;   // [kPChunk][128] fp16: one tile of K rows
+  uint8_t* v;   // [kPChunk][128] fp16: one tile of V rows
+  float* sc;    // [G][kPChunk] scores, then exp(score - running max)
+  float* ml;    // [G][2] running (max, sum of exp) of the unit
+  float* fac;   // [G] rescale factor of the running output for this tile
+  float* sw;    // [G][n_split] merge weights
 };
 __host__ __device__ inline size_t attn_smem_bytes(int G, int ns) {
-  return (size_t)2 * kPChunk * kPD * 2 + (size_t)G * kPChunk * 4 + (size_t)G * 2 * 4 + (size_t)G * ns * 4;
+  return (size_t)2 * kPChunk * kPD * 2 + (size_t)G * kPChunk * 4 + (size_t)G * 3 * 4 + (size_t)G * ns * 4;
 }
 __device__ __forceinline__ AttnSmem attn_smem(uint8_t* base, int G) {
   AttnSmem a;
@@ -276,7 +277,8 @@ __device__ __forceinline__ AttnSmem attn_smem(uint8_t* base, int G) {
   a.v = base + kPChunk * kPD * 2;
   a.sc = reinterpret_cast<float*>(a.v + kPChunk * kPD * 2);
   a.ml = a.sc + G * kPChunk;
-  a.sw = a.ml + 2 * G;
+  a.fac = a.ml + 2 * G;
+  a.sw = a.fac + G;
   return a;
 }
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -653,88 +655,141 @@ struct Consumer {
     if (ctid == 0) st.stats_embed[blockIdx.x * 4] = ss;
   }
 
-  // Split-KV attention units (kv head, split) of this CTA, then the merge of
-  // every KV head whose last split finished here.  A unit holds at most
-  // kPChunk positions; its K and V rows (contiguous in the cache) come into
-  // shared memory with 16-byte asynchronous copies issued all at once.
+  // Split-KV attention.  This step's context is cut into ns splits per KV
+  // head (at least kPMinSplit positions each, at most one unit per CTA where
+  // the grid allows); a unit walks its positions in tiles of kPChunk rows of
+  // K and V (contiguous in the cache, brought to shared memory with 16-byte
+  // asynchronous copies) with a running max and sum (online softmax).  With
+  // one split the unit writes the head output; otherwise it writes its
+  // (max, sum, unnormalised output) and the last unit of each KV head to
+  // finish merges the splits (log-sum-exp).
   template <int G>
   __device__ void attention(const LRow& L, int lk) {
     const int n_ctx = st.params[0] + 1;
-    const int ns = st.n_split;
+    int ns = (n_ctx + kPMinSplit - 1) / kPMinSplit;
+    if (ns > st.n_split) ns = st.n_split;
     const int chunk = (n_ctx + ns - 1) / ns;
     const AttnSmem a = attn_smem(sm.xst, G);
     const int units = st.Hkv * ns;
     const int S = kAttnPartStride;
+    constexpr int kOP = (G * (kPD / 2) + kPCThreads - 1) / kPCThreads;  // (head, dim pair)s per thread
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       const int kvh = u / ns, split = u % ns;
       const int p0 = split * chunk;
       const int p1 = min(p0 + chunk, n_ctx);
       const int np = p1 > p0 ? p1 - p0 : 0;
-      // K, V rows p0..p1-1 -> shared memory (np * 256 bytes each)
-      {
-        const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(L.kc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
-        const uint8_t* vsrc = reinterpret_cast<const uint8_t*>(L.vc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
-        const int n16 = np * (kPD * 2 / 16);
-        for (int i = ctid; i < 2 * n16; i += kPCThreads) {
-          const bool isv = i >= n16;
-          const int o = (isv ? i - n16 : i) * 16;
-          cp_async16((isv ? a.v : a.k) + o, (isv ? vsrc : ksrc) + o);
-        }
-        cp_async_commit();
-      }
+      const uint8_t* kbase = reinterpret_cast<const uint8_t*>(L.kc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
+      const uint8_t* vbase = reinterpret_cast<const uint8_t*>(L.vc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
       float qr[G][4];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float4 t = __ldcg(reinterpret_cast<const float4*>(st.q + (int64_t)(kvh * G + h) * kPD + 4 * lane));
         qr[h][0] = t.x; qr[h][1] = t.y; qr[h][2] = t.z; qr[h][3] = t.w;
       }
-      cp_async_wait_all();
-      cons_bar();
-      // scores: a warp per position, lanes split the head dimension
-      for (int i = warp; i < np; i += kPConsumers) {
-        const uint2 kr = *reinterpret_cast<const uint2*>(a.k + (size_t)i * kPD * 2 + 8 * lane);
-        const float k0 = half_bits_to_float(kr.x), k1 = half_bits_to_float(kr.x >> 16);
-        const float k2 = half_bits_to_float(kr.y), k3 = half_bits_to_float(kr.y >> 16);
+      if (ctid < G) {
+        a.ml[2 * ctid] = -INFINITY;
+        a.ml[2 * ctid + 1] = 0.f;
+      }
+      float o[kOP][2];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float d = qr[h][0] * k0;
-          d = fmaf(qr[h][1], k1, d);
-          d = fmaf(qr[h][2], k2, d);
-          d = fmaf(qr[h][3], k3, d);
-          d = warp_sum(d);
-          if (lane == 0) a.sc[h * kPChunk + i] = d * kAttnScale;
+      for (int k = 0; k < kOP; ++k) o[k][0] = o[k][1] = 0.f;
+      cons_bar();  // the running (max, sum) start values are visible
+      for (int t0 = 0; t0 < np; t0 += kPChunk) {
+        const int nt = min(kPChunk, np - t0);
+        {  // K, V rows of the tile -> shared memory (nt * 256 bytes each)
+          const int n16 = nt * (kPD * 2 / 16);
+          const int off = t0 * kPD * 2;
+          for (int i = ctid; i < 2 * n16; i += kPCThreads) {
+            const bool isv = i >= n16;
+            const int ob = (isv ? i - n16 : i) * 16;
+            cp_async16((isv ? a.v : a.k) + ob, (isv ? vbase : kbase) + off + ob);
+          }
+          cp_async_commit();
+          cp_async_wait_all();
         }
+        cons_bar();
+        // scores: a warp per position, lanes split the head dimension
+        for (int i = warp; i < nt; i += kPConsumers) {
+          const uint2 kr = *reinterpret_cast<const uint2*>(a.k + (size_t)i * kPD * 2 + 8 * lane);
+          const float k0 = half_bits_to_float(kr.x), k1 = half_bits_to_float(kr.x >> 16);
+          const float k2 = half_bits_to_float(kr.y), k3 = half_bits_to_float(kr.y >> 16);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float d = qr[h][0] * k0;
+            d = fmaf(qr[h][1], k1, d);
+            d = fmaf(qr[h][2], k2, d);
+            d = fmaf(qr[h][3], k3, d);
+            d = warp_sum(d);
+            if (lane == 0) a.sc[h * kPChunk + i] = d * kAttnScale;
+          }
+        }
+        cons_bar();
+        // running max and sum per head (warp h)
+        for (int h = warp; h < G; h += kPConsumers) {
+          float mt = -INFINITY;
+          for (int i = lane; i < nt; i += 32) mt = fmaxf(mt, a.sc[h * kPChunk + i]);
+          mt = warp_max(mt);
+          const float m_old = a.ml[2 * h], m_new = fmaxf(m_old, mt);
+          float l = 0.f;
+          for (int i = lane; i < nt; i += 32) {
+            const float e = expf(a.sc[h * kPChunk + i] - m_new);
+            a.sc[h * kPChunk + i] = e;
+            l += e;
+          }
+          l = warp_sum(l);
+          if (lane == 0) {
+            const float f = m_old == -INFINITY ? 0.f : expf(m_old - m_new);
+            a.fac[h] = f;
+            a.ml[2 * h] = m_new;
+            a.ml[2 * h + 1] = fmaf(a.ml[2 * h + 1], f, l);
+          }
+        }
+        cons_bar();
+        // P V: thread pair (h, d2) keeps dims 2 d2, 2 d2 + 1 of head h
+#pragma unroll
+        for (int k = 0; k < kOP; ++k) {
+          const int idx = ctid + k * kPCThreads;
+          if (idx < G * (kPD / 2)) {
+            const int h = idx / (kPD / 2), d2 = idx % (kPD / 2);
+            const float* e = a.sc + h * kPChunk;
+            const float f = a.fac[h];
+            float o0 = o[k][0] * f, o1 = o[k][1] * f;
+            for (int i = 0; i < nt; ++i) {
+              const uint32_t wv = *reinterpret_cast<const uint32_t*>(a.v + (size_t)i * kPD * 2 + 4 * d2);
+              o0 = fmaf(e[i], half_bits_to_float(wv), o0);
+              o1 = fmaf(e[i], half_bits_to_float(wv >> 16), o1);
+            }
+            o[k][0] = o0;
+            o[k][1] = o1;
+          }
+        }
+        cons_bar();  // the next tile overwrites K, V and the scores
       }
-      cons_bar();
-      for (int h = warp; h < G; h += kPConsumers) {
-        float m = -INFINITY;
-        for (int i = lane; i < np; i += 32) m = fmaxf(m, a.sc[h * kPChunk + i]);
-        m = warp_max(m);
-        float l = 0.f;
-        for (int i = lane; i < np; i += 32) {
-          const float e = expf(a.sc[h * kPChunk + i] - m);
-          a.sc[h * kPChunk + i] = e;
-          l += e;
+      if (ns == 1) {
+#pragma unroll
+        for (int k = 0; k < kOP; ++k) {
+          const int idx = ctid + k * kPCThreads;
+          if (idx < G * (kPD / 2)) {
+            const int h = idx / (kPD / 2), d2 = idx % (kPD / 2);
+            const float inv = 1.0f / a.ml[2 * h + 1];
+            *reinterpret_cast<float2*>(st.attn_out + (int64_t)(kvh * G + h) * kPD + 2 * d2) =
+                make_float2(o[k][0] * inv, o[k][1] * inv);
+          }
         }
-        l = warp_sum(l);
-        if (lane == 0) { a.ml[2 * h] = m; a.ml[2 * h + 1] = l; }
+        cons_bar();  // scratch reuse by the next unit
+        continue;
       }
-      cons_bar();
-      // P V: thread (h, d2) accumulates dims 2 d2, 2 d2 + 1 of head h
-      for (int idx = ctid; idx < G * (kPD / 2); idx += kPCThreads) {
-        const int h = idx / (kPD / 2), d2 = idx % (kPD / 2);
-        const float* e = a.sc + h * kPChunk;
-        float o0 = 0.f, o1 = 0.f;
-        for (int i = 0; i < np; ++i) {
-          const uint32_t wv = *reinterpret_cast<const uint32_t*>(a.v + (size_t)i * kPD * 2 + 4 * d2);
-          o0 = fmaf(e[i], half_bits_to_float(wv), o0);
-          o1 = fmaf(e[i], half_bits_to_float(wv >> 16), o1);
-        }
-        float* dst = st.attn_part + ((int64_t)(kvh * G + h) * ns + split) * S;
-        *reinterpret_cast<float2*>(dst + 2 + 2 * d2) = make_float2(o0, o1);
-        if (d2 == 0) {
-          dst[0] = np > 0 ? a.ml[2 * h] : -INFINITY;
-          dst[1] = np > 0 ? a.ml[2 * h + 1] : 0.f;
+#pragma unroll
+      for (int k = 0; k < kOP; ++k) {
+        const int idx = ctid + k * kPCThreads;
+        if (idx < G * (kPD / 2)) {
+          const int h = idx / (kPD / 2), d2 = idx % (kPD / 2);
+          float* dst = st.attn_part + ((int64_t)(kvh * G + h) * ns + split) * S;
+          *reinterpret_cast<float2*>(dst + 2 + 2 * d2) = make_float2(o[k][0], o[k][1]);
+          if (d2 == 0) {
+            dst[0] = a.ml[2 * h];
+            dst[1] = a.ml[2 * h + 1];
+          }
         }
       }
       // publish this split (release by one thread after the CTA barrier)
@@ -786,12 +841,12 @@ struct Consumer {
           const float* ph0 = st.attn_part + (int64_t)(kvh * G + h) * ns * S + 2 + d;
           const float* wt = a.sw + h * ns;
           float O = 0.f;
-          for (int t = 0; t < ns; t += 8) {
-            float v[8];
+          for (int t = 0; t < ns; t += 16) {
+            float v[16];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) v[k] = t + k < ns ? __ldcg(ph0 + (int64_t)(t + k) * S) : 0.f;
+            for (int k = 0; k < 16; ++k) v[k] = t + k < ns ? __ldcg(ph0 + (int64_t)(t + k) * S) : 0.f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
+            for (int k = 0; k < 16; ++k)
               if (t + k < ns) O = fmaf(wt[t + k], v[k], O);
           }
           st.attn_out[(int64_t)(kvh * G + h) * kPD + d] = O / a.ml[2 * h + 1];

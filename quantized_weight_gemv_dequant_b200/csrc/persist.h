@@ -11,7 +11,8 @@ constexpr int kPConsumers = 14;      // consumer warps per CTA (plus an epilogue
 constexpr int kPRed = 8;             // depth of the row-partial ring between consumers and the epilogue warp
 constexpr int kPPartsPerLane = 8;    // CTAs at most: 32 * this (sum-of-squares partials read per lane)
 constexpr int kPMaxTR = 32;          // rows per ring slot at most
-constexpr int kPChunk = 64;          // attention positions per (KV head, split) unit at most
+constexpr int kPChunk = 64;          // attention positions per K/V tile
+constexpr int kPMinSplit = 32;       // attention positions per (KV head, split) unit at least, where possible
 constexpr int kPSplitsPerRound = 4;  // split (m, l) loads per lane in flight during the merge
 constexpr int kPD = 128;             // head dimension
 constexpr int kAttnPartStride = kPD + 2;  // floats per (query head, split) partial: m, l, o[128]
@@ -66,12 +67,12 @@ int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int
                  PStep* st, size_t* smem);
 // Grid size (one CTA per SM), or 0 if a CTA of this size cannot be resident.
 int persist_grid(int qtype, size_t smem);
-// Attention splits per KV head for a grid and context limit.
+// Attention splits per KV head at most (at most one unit per CTA); a step
+// uses fewer when its context is short.
 inline int persist_splits(int grid, int Hkv, int max_ctx) {
-  int ns = grid / Hkv;
-  if (ns < 1) ns = 1;
-  const int need = (max_ctx + kPChunk - 1) / kPChunk;
-  return ns < need ? need : ns;
+  (void)max_ctx;
+  const int ns = grid / Hkv;
+  return ns < 1 ? 1 : ns;
 }
 // Words of the sync array for n_layers executed layers.
 inline int persist_sync_words(int n_layers, int Hkv) { return 2 + 5 * n_layers + n_layers * Hkv + 1; }
