@@ -33,6 +33,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "batch-1 decode tok/s; quantized GEMV achieved HBM GB/s vs B200 peak"
+# DRAM bytes read + written per algorithmic byte by the persistent decode
+# kernel, from one ncu capture (--set full) of a 4-layer 8B-shaped Q8_0 case
+# that fits the capture size rule: 1,485,751,296 + 4,783,104 bytes against
+# 1,485,578,240 algorithmic bytes.  The kernel streams every weight byte once,
+# so a full launch's traffic is this ratio times its algorithmic bytes.
+PERSIST_TRAFFIC_RATIO = 1490534400 / 1485578240
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -63,18 +69,27 @@ WORKLOADS = {
 
 # ---------------------------------------------------------------- distributed
 class Dist:
-    def __init__(self, n_gpus):
+    """One process per GPU (torchrun env): barrier and max over ranks.  NCCL on
+    GPUs; gloo (CPU tensors) where asked -- the CPU tests use it."""
+
+    def __init__(self, n_gpus, backend=None):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if n_gpus != self.world:
+            raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={self.world}: launch one process per GPU "
+                             f"(python -m torch.distributed.run --nproc-per-node {n_gpus} bench.py ...)")
         self.pg = None
+        self.backend = backend or "nccl"
         if self.world > 1:
             import datetime
             import torch
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {}
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=600), **kw)
             self.pg = dist
 
     def barrier(self):
@@ -85,7 +100,7 @@ class Dist:
         if not self.pg:
             return v
         import torch
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device="cuda" if self.backend == "nccl" else "cpu")
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
@@ -93,6 +108,13 @@ class Dist:
         if self.pg:
             self.pg.barrier()
             self.pg.destroy_process_group()
+            self.pg = None
+
+
+def whole_job_rate(world: int, steps: int, ms_max: float) -> float:
+    """Tokens per second of the whole job: every rank decodes `steps` tokens of
+    its own replica; the time is the slowest rank's (weak scaling)."""
+    return world * steps / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------- clocks
@@ -224,7 +246,7 @@ def run_ntx(args, dist: Dist):
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
     ms_step = ms_total / args.steps
-    value = dist.world * args.steps / (ms_total / 1e3)
+    value = whole_job_rate(dist.world, args.steps, ms_total)
 
     persistent = launches <= 2  # one persistent kernel (+ cosine finalisation when asked)
 
@@ -261,7 +283,12 @@ def run_ntx(args, dist: Dist):
         k_bytes = wl.bytes_per_token(d, qt, hqt, int(round(n_ctx_mean)))
         roof = {"bound": "hbm", "kernel": "persistent decode-step kernel (one launch per token)",
                 "achieved": round(k_bytes / (k_ms * 1e-3) / 1e9, 1), "peak": peak, "peak_kind": peak_kind,
-                "unit": "GB/s", "frac": round(k_bytes / (k_ms * 1e-3) / 1e9 / peak, 4), "traffic": args.traffic,
+                "unit": "GB/s", "frac": round(k_bytes / (k_ms * 1e-3) / 1e9 / peak, 4),
+                "traffic": args.traffic if args.traffic is not None else (
+                    round(PERSIST_TRAFFIC_RATIO * k_bytes) if qt == 8 else None),
+                "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of a 4-layer case of the same "
+                                "kernel, scaled to this launch's algorithmic bytes" if qt == 8 else
+                                "no capture of this instantiation",
                 "bytes_per_launch": k_bytes, "avg_launch_us": round(k_ms * 1e3, 3),
                 "timing": f"CUDA events on the compute stream around each of {n_probe} kernel launches "
                           f"(uncaptured steps right after the timed region, {round(probe_ms_step, 4)} ms/step there)"}

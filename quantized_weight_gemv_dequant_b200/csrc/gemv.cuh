@@ -208,74 +208,66 @@ __device__ __forceinline__ float row_q4_0(const uint8_t* seg, int lane, const f3
   return r;
 }
 
-// Q6_K: a slice is 8 super-blocks (1680 bytes).  Lane (pp = l>>4, h =
-// (l>>3)&1, j = l&7) owns elements 128h + 32g + 4j + t (g, t < 4) of both
-// super-blocks of pairs P = pp and P = pp + 2.  The even super-block of a pair
-// starts 4-byte aligned (pair stride 420 = 4 x 105), the odd one 2 bytes off;
-// its words are re-aligned with a funnel shift.
-__device__ __forceinline__ uint32_t ld_u32_shift2(const uint8_t* p_aligned) {
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(p_aligned);
-  return __funnelshift_r(w[0], w[1], 16);
+// Q6_K: a slice is 8 super-blocks (1680 bytes).  Lane l owns super-block
+// sb = l >> 2, half h = (l >> 1) & 1 and run r16 = l & 1: the elements
+// 128h + 32g + 16 r16 + i (g < 4, i < 16) -- four runs of 16 that each lie in
+// one 16-element sub-block (scale index 8h + r16 + 2g).  Their low nibbles are
+// 16 consecutive ql bytes at 64h + 32(g & 1) + 16 r16 (low nibble for g < 2,
+// high for g >= 2), their top bits the 2-bit field 2g of the 16 qh bytes at
+// 128 + 32h + 16 r16.  So 12 words of quant bytes and 2 of scales serve 64
+// elements.  Super-blocks sit 210 bytes apart: an odd one starts 2 bytes past
+// a word boundary, and its words are re-aligned with a funnel shift (shift 0
+// for the even ones, so every lane runs the same code).
+
+// Four words at byte offset o of a super-block (o a multiple of 4), given the
+// aligned word pointer below the super-block and the re-alignment shift.
+__device__ __forceinline__ void q6k_run4(const uint32_t* wb, int o, uint32_t sh, uint32_t* w) {
+  const uint32_t* p = wb + (o >> 2);
+  uint32_t a[5];
+#pragma unroll
+  for (int k = 0; k < 5; ++k) a[k] = p[k];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) w[k] = __funnelshift_r(a[k], a[k + 1], sh);
 }
 
 __device__ __forceinline__ float i8_to_f(uint32_t w, int b) { return byte_f(w ^ 0x80808080u, b) - 8388736.0f; }
 
-// sb_aligned: the even super-block's first byte, or for the odd one the
-// 4-byte aligned address 2 bytes before its first byte.  x2: 8 pairs,
-// x2[2g + t/2] = columns 128h + 32g + 4j + t (t even, odd) of the super-block.
-template <bool ODD>
-__device__ __forceinline__ float q6k_sb(const uint8_t* sb_aligned, int h, int j, const f32x2* x2) {
-  uint32_t ql0, ql1, qh, sA, sB, sC;
-  float d;
-  const int jj = j >> 2;
-  if (!ODD) {
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(sb_aligned);
-    ql0 = w[(64 * h + 4 * j) >> 2];
-    ql1 = w[(64 * h + 32 + 4 * j) >> 2];
-    qh = w[(128 + 32 * h + 4 * j) >> 2];
-    sA = w[(192 + 8 * h) >> 2];
-    sB = w[(196 + 8 * h) >> 2];
-    sC = 0;
-    d = half_bits_to_float(w[208 >> 2]);
-  } else {
-    ql0 = ld_u32_shift2(sb_aligned + 64 * h + 4 * j);
-    ql1 = ld_u32_shift2(sb_aligned + 64 * h + 32 + 4 * j);
-    qh = ld_u32_shift2(sb_aligned + 128 + 32 * h + 4 * j);
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(sb_aligned + 192 + 8 * h);
-    sA = w[0]; sB = w[1]; sC = w[2];
-    d = half_bits_to_float(reinterpret_cast<const uint32_t*>(sb_aligned)[208 >> 2] >> 16);
-  }
-  // scales of sub-blocks 8h + jj + 2g, g = 0..3
-  float sc[4];
-  if (!ODD) {
-    sc[0] = i8_to_f(sA, jj); sc[1] = i8_to_f(sA, jj + 2); sc[2] = i8_to_f(sB, jj); sc[3] = i8_to_f(sB, jj + 2);
-  } else {
-    sc[0] = i8_to_f(sA, jj + 2); sc[1] = i8_to_f(sB, jj); sc[2] = i8_to_f(sB, jj + 2); sc[3] = i8_to_f(sC, jj);
-  }
+// x2 layout for Q6_K: x2[8g + j] = (x at 2j, x at 2j+1 of run g).
+__device__ __forceinline__ float row_q6_k(const uint8_t* seg, int lane, const f32x2* x2) {
+  const int sb = lane >> 2, h = (lane >> 1) & 1, r16 = lane & 1;
+  const uint32_t boff = 210u * (uint32_t)sb;
+  const uint32_t* wb = reinterpret_cast<const uint32_t*>(seg + (boff & ~3u));
+  const uint32_t sh = (boff & 3u) * 8u;  // 0 or 16
+  const uint32_t* sp = wb + ((192 + 8 * h) >> 2);
+  const uint32_t s0 = __funnelshift_r(sp[0], sp[1], sh), s1 = __funnelshift_r(sp[1], sp[2], sh);
+  const float d = half_bits_to_float((wb[208 >> 2] >> sh) & 0xFFFFu);
   const f32x2 off = pack2(-8388640.0f, -8388640.0f);  // 2^23 + 32
+  uint32_t ql[4], qh[4];
+  q6k_run4(wb, 128 + 32 * h + 16 * r16, sh, qh);
   float acc = 0.f;
+  // runs g = 0, 2 share one ql run (low / high nibbles), then g = 1, 3 the other
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const uint32_t lo = ((g & 2) ? ((g & 1) ? ql1 : ql0) >> 4 : ((g & 1) ? ql1 : ql0)) & 0x0F0F0F0Fu;
-    const uint32_t q = lo | (((qh >> (2 * g)) & 0x03030303u) << 4);
-    const f32x2 v01 = add2(bytes_pair(q, 0, q, 1), off);
-    const f32x2 v23 = add2(bytes_pair(q, 2, q, 3), off);
-    const f32x2 s = fma2(v23, x2[2 * g + 1], mul2(v01, x2[2 * g]));
-    acc = fmaf(sc[g], hsum2(s), acc);
+  for (int half = 0; half < 2; ++half) {
+    q6k_run4(wb, 64 * h + 32 * half + 16 * r16, sh, ql);
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      const int g = half + 2 * gg;
+      f32x2 s2[2] = {0ull, 0ull};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = (gg ? (ql[k] >> 4) : ql[k]) & 0x0F0F0F0Fu;
+        const uint32_t hi = (g == 3) ? (qh[k] >> 2) : (qh[k] << (4 - 2 * g));
+        const uint32_t q = lo | (hi & 0x30303030u);
+        const f32x2 v01 = add2(bytes_pair(q, 0, q, 1), off);
+        const f32x2 v23 = add2(bytes_pair(q, 2, q, 3), off);
+        s2[k & 1] = fma2(v23, x2[8 * g + 2 * k + 1], fma2(v01, x2[8 * g + 2 * k], s2[k & 1]));
+      }
+      // sub-block scale: byte r16 + 2g of scales[8h .. 8h+7]
+      const float sc = i8_to_f(g < 2 ? s0 : s1, r16 + 2 * (g & 1));
+      acc = fmaf(sc, hsum2(add2(s2[0], s2[1])), acc);
+    }
   }
   return d * acc;
-}
-
-// x2 layout for Q6_K: x2[16 pass + 8 odd + 2g + t/2].
-__device__ __forceinline__ float row_q6_k(const uint8_t* seg, int lane, const f32x2* x2) {
-  const int pp = lane >> 4, h = (lane >> 3) & 1, j = lane & 7;
-  float r = 0.f;
-#pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const uint8_t* base = seg + 420 * (pp + 2 * pass);
-    r += q6k_sb<false>(base, h, j, x2 + 16 * pass) + q6k_sb<true>(base + 208, h, j, x2 + 16 * pass + 8);
-  }
-  return r;
 }
 
 // ---------------------------------------------------------------------------
@@ -385,21 +377,19 @@ __device__ __forceinline__ bool lane_active(int lane, int ucols) {
   else return 2 * lane < ucols / 32;
 }
 
-// The 64 columns of a Q6_K slice a lane keeps, as fp32 pairs.
+// The 64 columns of a Q6_K slice a lane keeps, as fp32 pairs: four runs of 16
+// contiguous columns 256 sb + 128 h + 32 g + 16 r16 (see row_q6_k).
 template <class Pro>
 __device__ __forceinline__ void load_x_slice_q6_k(const Pro& pro, int64_t c0, int lane, f32x2* x2) {
-  const int pp = lane >> 4, h = (lane >> 3) & 1, j = lane & 7;
+  const int sb = lane >> 2, h = (lane >> 1) & 1, r16 = lane & 1;
 #pragma unroll
-  for (int pass = 0; pass < 2; ++pass)
+  for (int g = 0; g < 4; ++g)
 #pragma unroll
-    for (int odd = 0; odd < 2; ++odd)
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float4 v = pro.ld(c0 + 512 * (pp + 2 * pass) + 256 * odd + 128 * h + 32 * g + 4 * j);
-        f32x2* o = x2 + 16 * pass + 8 * odd + 2 * g;
-        o[0] = pack2(v.x, v.y);
-        o[1] = pack2(v.z, v.w);
-      }
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = pro.ld(c0 + 256 * sb + 128 * h + 32 * g + 16 * r16 + 4 * q);
+      x2[8 * g + 2 * q] = pack2(v.x, v.y);
+      x2[8 * g + 2 * q + 1] = pack2(v.z, v.w);
+    }
 }
 
 // ---------------------------------------------------------------------------
