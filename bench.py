@@ -294,6 +294,48 @@ def run_ntx(args, dist: Dist):
                           f"(uncaptured steps right after the timed region, {round(probe_ms_step, 4)} ms/step there)"}
     pos_base += n_probe
 
+    # --------------------------- GEMV phases inside the step (persistent kernel)
+    in_step = None
+    if persistent:
+        n_ph = 2 + 5 * L
+        grid = ntx.ntx_engine_set_phase_probe(eng, None, 0)
+        ts = torch.zeros((1 + n_ph) * grid, dtype=torch.int64, device="cuda")
+        ntx.ntx_engine_set_phase_probe(eng, ts, ts.numel())
+        spans = []
+        n_phase_steps = min(args.steps, 8)
+        for i in range(n_phase_steps):
+            with torch.cuda.stream(cs):
+                ntx.ntx_decode_step(eng, -1, pos_of(pos_base + i), None, next_tok, ntx.NTX_NO_GRAPH, None)
+            cs.synchronize()
+            t = ts.cpu().numpy().reshape(1 + n_ph, grid)
+            done = t[1:].max(axis=1)  # phase p complete when its last CTA published it
+            spans.append(np.diff(np.concatenate([[t[0].min()], done])) / 1e3)  # us per phase
+        ntx.ntx_engine_set_phase_probe(eng, None, 0)
+        pos_base += n_phase_steps
+        spans = np.array(spans)  # [steps][phases]
+        H, F, Hq, Hkv, D = d["hidden"], d["ffn"], d["n_heads"], d["n_kv_heads"], d["head_dim"]
+        kinds = {"q/k/v (RMSNorm, RoPE, KV append)": (0, (Hq + 2 * Hkv) * D, H),
+                 "o (+ residual)": (2, H, Hq * D),
+                 "gate/up (RMSNorm, SwiGLU)": (3, 2 * F, H),
+                 "down (+ residual, cosine statistics)": (4, H, F)}
+        in_step = []
+        for name, (j, M, K) in kinds.items():
+            us = float(spans[:, [1 + 5 * k + j for k in range(L)]].mean())
+            by = wl.mat_bytes(qt, M, K)
+            in_step.append({"phase": name, "M": M, "K": K, "weight_bytes": by, "us": round(us, 3),
+                            "GBs": round(by / (us * 1e-6) / 1e9, 1), "frac": round(by / (us * 1e-6) / 1e9 / peak, 4)})
+        us = float(spans[:, 1 + 5 * L].mean())
+        by = wl.mat_bytes(hqt, d["vocab"], H)
+        in_step.append({"phase": "head (final RMSNorm, argmax)", "M": d["vocab"], "K": H, "weight_bytes": by,
+                        "us": round(us, 3), "GBs": round(by / (us * 1e-6) / 1e9, 1),
+                        "frac": round(by / (us * 1e-6) / 1e9 / peak, 4)})
+        in_step = {"phases": in_step,
+                   "attention_us": round(float(spans[:, [2 + 5 * k for k in range(L)]].mean()), 3),
+                   "embed_us": round(float(spans[:, 0].mean()), 3),
+                   "timing": f"%globaltimer per CTA at each phase's publication, {n_phase_steps} uncaptured steps; "
+                             "a phase's time runs from the previous phase's last publication to its own last one "
+                             "(grid barrier, x staging and the epilogue tail included)"}
+
     # ------------------------------------------- the per-op kernel chain, for comparison
     chain = None
     if not args.no_chain:
@@ -382,6 +424,7 @@ def run_ntx(args, dist: Dist):
         "launches_per_step": launches,
         "clocks": clk,
         "gemv": gemv,
+        "gemv_in_step": in_step,
         "chain": chain,
         "cpu_baseline": cpu,
     }

@@ -269,6 +269,17 @@ NTX_API int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* logits
  * events. */
 NTX_API int ntx_engine_set_probe(ntx_engine* e, void* const* begin_events, void* const* end_events, int n);
 
+/* Profiling the persistent kernel: while set, every ntx_decode_step made
+ * with NTX_NO_GRAPH that runs the persistent kernel writes %globaltimer
+ * nanoseconds into dev_ts (device, 8-byte aligned, n_words 64-bit words):
+ * dev_ts[b] = start of CTA b, dev_ts[(1 + p) * grid + b] = when CTA b published
+ * phase p (p = 0 embed; 1 + 5k + {0..4} = Q/K/V, attention, O, gate/up, down
+ * of the k-th executed layer; 1 + 5n = head).  A step whose phases do not fit
+ * records nothing.  Returns the grid size (CTAs) of the persistent kernel, 0
+ * if this engine does not use it, or a negative error; n_words == 0 clears
+ * the probe. */
+NTX_API int ntx_engine_set_phase_probe(ntx_engine* e, unsigned long long* dev_ts, size_t n_words);
+
 /* Number of libntx kernels one decode step launched (the last step enqueued
  * or captured by this engine), or a negative error. */
 NTX_API int ntx_engine_launches_per_step(ntx_engine* e);

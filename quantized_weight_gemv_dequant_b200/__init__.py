@@ -37,7 +37,7 @@ EXPORTS = (
     "ntx_dequant", "ntx_gemv_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_workspace_bytes", "ntx_attn_decode",
     "ntx_swiglu", "ntx_layer_layout", "ntx_layer_workspace_bytes", "ntx_decode_layer", "ntx_engine_workspace_bytes",
     "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
-    "ntx_engine_launches_per_step", "ntx_attn_decode_static",
+    "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
 )
 
 
@@ -98,6 +98,7 @@ def lib():
             "ntx_engine_set_probe": ([vp, vp, vp, i32], i32),
             "ntx_engine_launches_per_step": ([vp], i32),
             "ntx_attn_decode_static": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp], i32),
+            "ntx_engine_set_phase_probe": ([vp, vp, sz], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -260,6 +261,15 @@ def ntx_engine_set_probe(engine, begin_events, end_events):
     b = (ctypes.c_void_p * max(n, 1))(*begin_events)
     e = (ctypes.c_void_p * max(n, 1))(*end_events)
     _check(lib().ntx_engine_set_probe(engine, b, e, n))
+
+
+def ntx_engine_set_phase_probe(engine, dev_ts, n_words: int) -> int:
+    """dev_ts: device buffer of n_words uint64 (a torch tensor or pointer) or
+    None.  Returns the persistent kernel's grid size (0 if not used)."""
+    rc = lib().ntx_engine_set_phase_probe(engine, _p(dev_ts) if dev_ts is not None else None, n_words)
+    if rc < 0:
+        _check(rc)
+    return rc
 
 
 def ntx_engine_launches_per_step(engine) -> int:

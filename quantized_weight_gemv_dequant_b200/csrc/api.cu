@@ -364,6 +364,8 @@ struct ntx_engine {
   ntx::PLayer *pl_all, *pl_skip;
   int n_skip_run;  // executed layers under the skip set
   unsigned* psync;
+  unsigned long long* phase_ts;  // phase probe (kernel-by-kernel steps only)
+  size_t phase_ts_words;
 };
 
 size_t engine_carve(const ntx_model_config* c, uint8_t* base, ntx_engine* e) {
@@ -457,6 +459,9 @@ cudaError_t persist_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t
   st.next_token = next_token;
   st.head_ctr_index = 2 + 5 * nrun;
   st.abort_index = st.head_ctr_index + nrun * c.n_kv_heads;
+  // phase timestamps only in uncaptured steps, and only if the buffer holds them all
+  const size_t need = (size_t)(1 + 2 + 5 * nrun) * e->pgrid;
+  st.probe_ts = (probe && e->phase_ts && e->phase_ts_words >= need) ? e->phase_ts : nullptr;
   cudaError_t err =
       cudaMemsetAsync(e->psync, 0, sizeof(unsigned) * ntx::persist_sync_words(nrun, c.n_kv_heads), s);
   if (err == cudaSuccess && probe && !e->probe_b.empty()) err = cudaEventRecord(e->probe_b[0], s);
@@ -802,6 +807,15 @@ extern "C" int ntx_engine_set_probe(ntx_engine* e, void* const* begin_events, vo
     e->probe_e.push_back(static_cast<cudaEvent_t>(end_events[k]));
   }
   return NTX_OK;
+}
+
+extern "C" int ntx_engine_set_phase_probe(ntx_engine* e, unsigned long long* dev_ts, size_t n_words) {
+  if (!e) return fail(NTX_ERR_INVALID_ARG, "engine is NULL");
+  if (n_words && !dev_ts) return fail(NTX_ERR_INVALID_ARG, "NULL probe buffer with nonzero size");
+  if (dev_ts && !aligned(dev_ts, 8)) return fail(NTX_ERR_ALIGN, "probe buffer must be 8-byte aligned");
+  e->phase_ts = n_words ? dev_ts : nullptr;
+  e->phase_ts_words = n_words;
+  return e->persist ? e->pgrid : 0;
 }
 
 extern "C" int ntx_engine_launches_per_step(ntx_engine* e) {

@@ -900,16 +900,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
       }
     }
   }
-  // RoPE table of this step's position (the same for every layer)
-  if (warp == kPEpiWarp) {
-    const int pos = st.params[0];
-    for (int i = lane; i < kPD / 2; i += 32) {
-      const double inv_freq = pow((double)st.theta, -2.0 * (double)i / (double)kPD);
-      double sn, cn;
-      sincos((double)pos * inv_freq, &sn, &cn);
-      sm.rope[i] = make_float2((float)cn, (float)sn);
-    }
-  }
+  if (st.probe_ts && threadIdx.x == 0) st.probe_ts[blockIdx.x] = global_ns();
   __syncthreads();
 
   if (warp == kPCopyWarp) {
@@ -917,6 +908,18 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
     cp.run();
   } else if (warp == kPEpiWarp) {
     // ---------------------------------------------------------- epilogue
+    // RoPE table of this step's position (the same for every layer), made
+    // here so that the other warps do not wait for it
+    {
+      const int pos = st.params[0];
+      for (int i = lane; i < kPD / 2; i += 32) {
+        const double inv_freq = pow((double)st.theta, -2.0 * (double)i / (double)kPD);
+        double sn, cn;
+        sincos((double)pos * inv_freq, &sn, &cn);
+        sm.rope[i] = make_float2((float)cn, (float)sn);
+      }
+      __syncwarp();
+    }
     Epilogue ep(st, sm, lane);
     bool ok = true;
     for (int p = 1; p < np && ok; ++p) {
@@ -987,6 +990,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
       if (lane == 0) {
         if (kind == PK_HEAD) old = atom_acq_rel_add(st.sync + p, 1u);
         else red_release_add(st.sync + p, 1u);
+        if (st.probe_ts) st.probe_ts[(size_t)(1 + p) * G + blockIdx.x] = global_ns();
       }
       old = __shfl_sync(0xffffffffu, old, 0);
       if (kind == PK_HEAD && old == G - 1) {
@@ -1053,7 +1057,10 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
       if (kind == PK_EMBED || kind == PK_ATTN) {
         // publish (release by one thread after the CTA barrier)
         cons_bar();
-        if (ctid == 0) red_release_add(st.sync + p, 1u);
+        if (ctid == 0) {
+          red_release_add(st.sync + p, 1u);
+          if (st.probe_ts) st.probe_ts[(size_t)(1 + p) * G + blockIdx.x] = global_ns();
+        }
       }
     }
   }

@@ -12,7 +12,7 @@ constexpr int kPRed = 8;             // depth of the row-partial ring between co
 constexpr int kPPartsPerLane = 8;    // CTAs at most: 32 * this (sum-of-squares partials read per lane)
 constexpr int kPMaxTR = 32;          // rows per ring slot at most
 constexpr int kPChunk = 64;          // attention positions per K/V tile
-constexpr int kPMinSplit = 32;       // attention positions per (KV head, split) unit at least, where possible
+constexpr int kPMinSplit = 128;      // attention positions per (KV head, split) unit at least, where possible
 constexpr int kPSplitsPerRound = 4;  // split (m, l) loads per lane in flight during the merge
 constexpr int kPD = 128;             // head dimension
 constexpr int kAttnPartStride = kPD + 2;  // floats per (query head, split) partial: m, l, o[128]
@@ -59,6 +59,8 @@ struct PStep {
   PGeom g[7];          // indexed by PKind
   int slot_bytes, n_slots, xstage_bytes, red_floats;
   int* status;  // device status word
+  unsigned long long* probe_ts;  // nullable: [1 + phases][grid] %globaltimer ns (row 0: kernel start,
+                                 // row 1 + p: when the CTA published phase p)
 };
 
 // Fills the geometry fields of *st and the dynamic shared memory size; -1 if

@@ -291,3 +291,28 @@ def test_engine_config_4_llama8b_q8_0_144_steps():
     oracle_run(m, fed, tensors=tensors, nthreads=os.cpu_count(),
                check=lambda s, ref: check_logits(lg[s], ref, int(nxt[s]), s))
     print(f"oracle teacher-forced 144 steps: {time.time() - t0:.1f} s")
+
+
+def test_engine_phase_probe_records_every_phase_in_order():
+    import torch
+    m = DeviceModel(TINY, ntx.NTX_Q8_0, ntx.NTX_Q8_0, 51, max_ctx=16, n_prior=0, source="host")
+    e = Engine(m)
+    grid = ntx.ntx_engine_set_phase_probe(e.h, None, 0)
+    assert grid == ntx.ntx_sm_count()
+    n_ph = 2 + 5 * TINY["n_layers"]
+    ts = torch.zeros((1 + n_ph) * grid, dtype=torch.int64, device="cuda")
+    assert ntx.ntx_engine_set_phase_probe(e.h, ts, ts.numel()) == grid
+    e.run([3], flags=ntx.NTX_NO_GRAPH)
+    t = ts.cpu().numpy().reshape(1 + n_ph, grid)
+    assert (t > 0).all()  # every CTA stamped its start and every phase
+    done = t[1:].max(axis=1)
+    assert (done[1:] >= done[:-1]).all()  # phases complete in order
+    assert (t[1:].min(axis=1) >= t[0].min()).all()
+    # graph replays record nothing; a cleared probe records nothing
+    ts.zero_()
+    e.run([-1], pos0=1)
+    assert int(ts.abs().sum()) == 0
+    ntx.ntx_engine_set_phase_probe(e.h, None, 0)
+    e.run([-1], pos0=2, flags=ntx.NTX_NO_GRAPH)
+    assert int(ts.abs().sum()) == 0
+    e.close()
