@@ -35,10 +35,10 @@ sys.path.insert(0, ROOT)
 METRIC = "batch-1 decode tok/s; quantized GEMV achieved HBM GB/s vs B200 peak"
 # DRAM bytes read + written per algorithmic byte by the persistent decode
 # kernel, from one ncu capture (--set full) of a 4-layer 8B-shaped Q8_0 case
-# that fits the capture size rule: 1,485,751,296 + 4,783,104 bytes against
+# that fits the capture size rule: 1,485,997,056 + 6,683,392 bytes against
 # 1,485,578,240 algorithmic bytes.  The kernel streams every weight byte once,
 # so a full launch's traffic is this ratio times its algorithmic bytes.
-PERSIST_TRAFFIC_RATIO = 1490534400 / 1485578240
+PERSIST_TRAFFIC_RATIO = 1492680448 / 1485578240
 FALLBACK_HBM_GBS = 6650.0
 
 
