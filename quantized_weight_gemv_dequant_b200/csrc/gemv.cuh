@@ -125,11 +125,6 @@ struct ProRms {
   }
 };
 
-// x already staged in shared memory (fp32).
-struct ProSmem {
-  const float* x;
-  __device__ __forceinline__ float4 ld(int64_t j) const { return *reinterpret_cast<const float4*>(x + j); }
-};
 
 // ------------------------------------------------------------- decoders
 __device__ __forceinline__ float byte_f(uint32_t w, int b) { return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | b)); }
@@ -206,68 +201,6 @@ __device__ __forceinline__ float row_q4_0(const uint8_t* seg, int lane, const f3
     r = fmaf(d, fmaf(0.0625f, hsum2(hi_acc[0]) + hsum2(hi_acc[1]), hsum2(lo_acc[0]) + hsum2(lo_acc[1])), r);
   }
   return r;
-}
-
-// Q6_K: a slice is 8 super-blocks (1680 bytes).  Lane l owns super-block
-// sb = l >> 2, half h = (l >> 1) & 1 and run r16 = l & 1: the elements
-// 128h + 32g + 16 r16 + i (g < 4, i < 16) -- four runs of 16 that each lie in
-// one 16-element sub-block (scale index 8h + r16 + 2g).  Their low nibbles are
-// 16 consecutive ql bytes at 64h + 32(g & 1) + 16 r16 (low nibble for g < 2,
-// high for g >= 2), their top bits the 2-bit field 2g of the 16 qh bytes at
-// 128 + 32h + 16 r16.  So 12 words of quant bytes and 2 of scales serve 64
-// elements.  Super-blocks sit 210 bytes apart: an odd one starts 2 bytes past
-// a word boundary, and its words are re-aligned with a funnel shift (shift 0
-// for the even ones, so every lane runs the same code).
-
-// Four words at byte offset o of a super-block (o a multiple of 4), given the
-// aligned word pointer below the super-block and the re-alignment shift.
-__device__ __forceinline__ void q6k_run4(const uint32_t* wb, int o, uint32_t sh, uint32_t* w) {
-  const uint32_t* p = wb + (o >> 2);
-  uint32_t a[5];
-#pragma unroll
-  for (int k = 0; k < 5; ++k) a[k] = p[k];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) w[k] = __funnelshift_r(a[k], a[k + 1], sh);
-}
-
-__device__ __forceinline__ float i8_to_f(uint32_t w, int b) { return byte_f(w ^ 0x80808080u, b) - 8388736.0f; }
-
-// x2 layout for Q6_K: x2[8g + j] = (x at 2j, x at 2j+1 of run g).
-__device__ __forceinline__ float row_q6_k(const uint8_t* seg, int lane, const f32x2* x2) {
-  const int sb = lane >> 2, h = (lane >> 1) & 1, r16 = lane & 1;
-  const uint32_t boff = 210u * (uint32_t)sb;
-  const uint32_t* wb = reinterpret_cast<const uint32_t*>(seg + (boff & ~3u));
-  const uint32_t sh = (boff & 3u) * 8u;  // 0 or 16
-  const uint32_t* sp = wb + ((192 + 8 * h) >> 2);
-  const uint32_t s0 = __funnelshift_r(sp[0], sp[1], sh), s1 = __funnelshift_r(sp[1], sp[2], sh);
-  const float d = half_bits_to_float((wb[208 >> 2] >> sh) & 0xFFFFu);
-  const f32x2 off = pack2(-8388640.0f, -8388640.0f);  // 2^23 + 32
-  uint32_t ql[4], qh[4];
-  q6k_run4(wb, 128 + 32 * h + 16 * r16, sh, qh);
-  float acc = 0.f;
-  // runs g = 0, 2 share one ql run (low / high nibbles), then g = 1, 3 the other
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    q6k_run4(wb, 64 * h + 32 * half + 16 * r16, sh, ql);
-#pragma unroll
-    for (int gg = 0; gg < 2; ++gg) {
-      const int g = half + 2 * gg;
-      f32x2 s2[2] = {0ull, 0ull};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t lo = (gg ? (ql[k] >> 4) : ql[k]) & 0x0F0F0F0Fu;
-        const uint32_t hi = (g == 3) ? (qh[k] >> 2) : (qh[k] << (4 - 2 * g));
-        const uint32_t q = lo | (hi & 0x30303030u);
-        const f32x2 v01 = add2(bytes_pair(q, 0, q, 1), off);
-        const f32x2 v23 = add2(bytes_pair(q, 2, q, 3), off);
-        s2[k & 1] = fma2(v23, x2[8 * g + 2 * k + 1], fma2(v01, x2[8 * g + 2 * k], s2[k & 1]));
-      }
-      // sub-block scale: byte r16 + 2g of scales[8h .. 8h+7]
-      const float sc = i8_to_f(g < 2 ? s0 : s1, r16 + 2 * (g & 1));
-      acc = fmaf(sc, hsum2(add2(s2[0], s2[1])), acc);
-    }
-  }
-  return d * acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -369,6 +302,124 @@ __device__ __forceinline__ float rowfix_q4_0(const uint8_t* seg, int lane, const
   return r;
 }
 
+// Q6_K: a slice is 8 super-blocks (1680 bytes).  Lane l owns super-block
+// sb = l >> 2, half h = (l >> 1) & 1 and run r16 = l & 1: the elements
+// 128h + 32g + 16 r16 + i (g < 4, i < 16) -- four runs of 16 that each lie in
+// one 16-element sub-block (scale index 8h + r16 + 2g).  Their low nibbles are
+// 16 consecutive ql bytes at 64h + 32(g & 1) + 16 r16 (low nibble for g < 2,
+// high for g >= 2), their top bits the 2-bit field 2g of the 16 qh bytes at
+// 128 + 32h + 16 r16: 12 words of quant bytes and 2 of scales serve 64
+// elements.  Super-blocks sit 210 bytes apart, so an odd one starts 2 bytes
+// past a word boundary; its words are re-aligned with a funnel shift (shift 0
+// for the even ones, so every lane runs the same code).
+//
+// The dot product is the integer one of Q8_0 / Q4_0: x in 22-bit block fixed
+// point (32-column blocks; run g of a lane is half of block 8 sb + 4h + g of
+// the slice, the other half belongs to lane l ^ 1), byte limbs, dp4a sums of
+// the unsigned 6-bit codes q in int32; the -32 offset is folded into the
+// starting value of each limb's sum (-32 times the run's limb sum), and each
+// run's sum is scaled by its sub-block scale, the block scale of x and d.
+struct XFix6 {
+  uint32_t l0[16], l1[16], l2[16];  // word 4g + w = columns 4w..4w+3 of run g
+  float xs[4];                      // 2^(e - 22) of run g's 32-column block
+  int c[4][3];                      // -32 * sum of run g's limb-j bytes
+};
+
+// Four words at byte offset o of a super-block (o a multiple of 4), given the
+// aligned word pointer below the super-block and the re-alignment shift.
+__device__ __forceinline__ void q6k_run4(const uint32_t* wb, int o, uint32_t sh, uint32_t* w) {
+  const uint32_t* p = wb + (o >> 2);
+  uint32_t a[5];
+#pragma unroll
+  for (int k = 0; k < 5; ++k) a[k] = p[k];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) w[k] = __funnelshift_r(a[k], a[k + 1], sh);
+}
+
+__device__ __forceinline__ float i8_to_f(uint32_t w, int b) { return byte_f(w ^ 0x80808080u, b) - 8388736.0f; }
+
+__device__ __forceinline__ float rowfix_q6_k(const uint8_t* seg, int lane, const XFix6& x) {
+  const int sb = lane >> 2, h = (lane >> 1) & 1, r16 = lane & 1;
+  const uint32_t boff = 210u * (uint32_t)sb;
+  const uint32_t* wb = reinterpret_cast<const uint32_t*>(seg + (boff & ~3u));
+  const uint32_t sh = (boff & 3u) * 8u;  // 0 or 16
+  const uint32_t* sp = wb + ((192 + 8 * h) >> 2);
+  const uint32_t s0 = __funnelshift_r(sp[0], sp[1], sh), s1 = __funnelshift_r(sp[1], sp[2], sh);
+  const float d = half_bits_to_float((wb[208 >> 2] >> sh) & 0xFFFFu);
+  uint32_t ql[4], qh[4];
+  q6k_run4(wb, 128 + 32 * h + 16 * r16, sh, qh);
+  float acc = 0.f;
+  // runs g = 0, 2 share one ql run (low / high nibbles), then g = 1, 3 the other
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    q6k_run4(wb, 64 * h + 32 * half + 16 * r16, sh, ql);
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      const int g = half + 2 * gg;
+      int a0 = x.c[g][0], a1 = x.c[g][1], a2 = x.c[g][2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = (gg ? (ql[k] >> 4) : ql[k]) & 0x0F0F0F0Fu;
+        const uint32_t hi = (g == 3) ? (qh[k] >> 2) : (qh[k] << (4 - 2 * g));
+        const uint32_t q = lo | (hi & 0x30303030u);
+        a0 = dp4a_uu(q, x.l0[4 * g + k], a0);
+        a1 = dp4a_uu(q, x.l1[4 * g + k], a1);
+        a2 = dp4a_us(q, x.l2[4 * g + k], a2);
+      }
+      // sub-block scale: byte r16 + 2g of scales[8h .. 8h+7]
+      const float sc = i8_to_f(g < 2 ? s0 : s1, r16 + 2 * (g & 1));
+      acc = fmaf(sc * x.xs[g], limbs_to_f(a0, a1, a2), acc);
+    }
+  }
+  return d * acc;
+}
+
+// A Q6_K lane's x straight from global memory (no shared staging): the lane
+// converts its four runs itself; a run's 32-column block max is the max over
+// its own 16 columns and the partner lane's (lane ^ 1).
+template <class Pro>
+__device__ __forceinline__ void fix6_direct(const Pro& pro, int64_t c0, int lane, XFix6& x) {
+  const int sb = lane >> 2, h = (lane >> 1) & 1, r16 = lane & 1;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = pro.ld(c0 + 256 * sb + 128 * h + 32 * g + 16 * r16 + 4 * q);
+    float m = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) m = fmaxf(m, fmaxf(fmaxf(fabsf(v[q].x), fabsf(v[q].y)), fmaxf(fabsf(v[q].z), fabsf(v[q].w))));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 126;
+    if (e < -100) e = -100;
+    const float up = __uint_as_float((uint32_t)(127 + 22 - e) << 23);
+    x.xs[g] = __uint_as_float((uint32_t)(127 + e - 22) << 23);
+    int s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float f[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+      uint32_t w0 = 0, w1 = 0, w2 = 0;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int X = __float2int_rn(f[t] * up);
+        const uint32_t b0 = (uint32_t)X & 0xFFu, b1 = ((uint32_t)X >> 8) & 0xFFu;
+        const int hi = X >> 16;
+        w0 |= b0 << (8 * t);
+        w1 |= b1 << (8 * t);
+        w2 |= ((uint32_t)hi & 0xFFu) << (8 * t);
+        s0 += (int)b0;
+        s1 += (int)b1;
+        s2 += hi;
+      }
+      x.l0[4 * g + q] = w0;
+      x.l1[4 * g + q] = w1;
+      x.l2[4 * g + q] = w2;
+    }
+    x.c[g][0] = -32 * s0;
+    x.c[g][1] = -32 * s1;
+    x.c[g][2] = -32 * s2;
+  }
+}
+
 // Columns of x a lane owns within its slice (relative to the slice start):
 // Q8_0/Q4_0: 64 l + i;  Q6_K: 512 P + 256 odd + 128 h + 32 g + 4 j + t.
 template <int QT>
@@ -377,47 +428,31 @@ __device__ __forceinline__ bool lane_active(int lane, int ucols) {
   else return 2 * lane < ucols / 32;
 }
 
-// The 64 columns of a Q6_K slice a lane keeps, as fp32 pairs: four runs of 16
-// contiguous columns 256 sb + 128 h + 32 g + 16 r16 (see row_q6_k).
-template <class Pro>
-__device__ __forceinline__ void load_x_slice_q6_k(const Pro& pro, int64_t c0, int lane, f32x2* x2) {
-  const int sb = lane >> 2, h = (lane >> 1) & 1, r16 = lane & 1;
-#pragma unroll
-  for (int g = 0; g < 4; ++g)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 v = pro.ld(c0 + 256 * sb + 128 * h + 32 * g + 16 * r16 + 4 * q);
-      x2[8 * g + 2 * q] = pack2(v.x, v.y);
-      x2[8 * g + 2 * q + 1] = pack2(v.z, v.w);
-    }
-}
-
 // ---------------------------------------------------------------------------
-// x staging: once per CTA, after the producer of x has finished, the consumer
-// warps read x with coalesced float4 loads (128 columns per warp and load,
-// eight loads in flight per lane) and leave it in shared memory in the form
-// the lanes need; after a named barrier among the consumer warps each lane
-// copies its own part into registers.
-//   Q8_0 / Q4_0 (fixed point, see XFix): the 8 lanes holding a 32-column
-//     block take its max|x| with shuffles; each lane turns its 4 columns into
-//     one 32-bit word per limb, stored at wd[(j*16 + k) * NP + c*32 + l]
-//     (limb j, word k of lane l of slice c; NP = 32 * slices + 2, the pad
-//     making the stores of a warp hit 32 distinct banks); the block scale
-//     2^(e-22) goes to sc[B] and the Q4_0 offsets -8 * sum(limb j) to
-//     cr[3B + j].
-//   Q6_K: x as fp32 in xf[K].
+// x staging: once per CTA, the consumer warps read x (coalesced) and leave it
+// in shared memory in the form the lanes need; after a named barrier among
+// the consumer warps each lane copies its own part into registers.  All
+// formats keep x as 22-bit block fixed point (see XFix): one warp per 128
+// columns, the 8 lanes holding a 32-column block take its max|x| with
+// shuffles, each lane turns its 4 columns into one 32-bit word per limb,
+// stored at wd[(j*16 + k) * NP + c*32 + l] (limb j, word k of lane l of slice
+// c; NP = 32 * slices + 2, the pad making the stores of a warp hit 32
+// distinct banks); the block scale 2^(e-22) goes to sc[B]; cr holds the
+// offset corrections (Q4_0: -8 * sum(limb j) per block; Q6_K: -32 * sum(limb
+// j) per 16-column run).
 struct XStage {
   uint32_t* wd;
   float* sc;
   int* cr;
-  float* xf;
   int np;
 };
 
+// Q6_K keeps one correction triple per 16-column run (K / 16 of them), the
+// other formats one per 32-column block (used by Q4_0).
 __host__ __device__ inline size_t xstage_bytes(int qtype, int64_t K) {
   const int64_t nslices = (K + kSliceCols - 1) / kSliceCols;
-  if (qtype == QT_Q6_K) return (size_t)K * 4;
-  return (size_t)3 * 16 * (32 * nslices + 2) * 4 + (size_t)(K / 32) * 4 + (size_t)(K / 32) * 12;
+  const int64_t ncorr = qtype == QT_Q6_K ? K / 16 : K / 32;
+  return (size_t)3 * 16 * (32 * nslices + 2) * 4 + (size_t)(K / 32) * 4 + (size_t)ncorr * 12;
 }
 
 __device__ __forceinline__ XStage xstage_at(uint8_t* base, int64_t K) {
@@ -427,7 +462,6 @@ __device__ __forceinline__ XStage xstage_at(uint8_t* base, int64_t K) {
   x.wd = reinterpret_cast<uint32_t*>(base);
   x.sc = reinterpret_cast<float*>(base + (size_t)3 * 16 * x.np * 4);
   x.cr = reinterpret_cast<int*>(x.sc + K / 32);
-  x.xf = reinterpret_cast<float*>(base);
   return x;
 }
 
@@ -443,53 +477,75 @@ __device__ __forceinline__ int group8_sum(int v) {
 }
 
 // One 128-column chunk of x (4 columns per lane, starting at col = chunk
-// start + 4 lane) into the staged form.
+// start + 4 lane) into the staged form: 22-bit block fixed point, byte limbs
+// packed four columns to a word, stored where the owning lane will read them.
 template <int QT>
 __device__ __forceinline__ void stage_chunk(const float4 v, int64_t col, const XStage& xs, int lane) {
-  if constexpr (QT == QT_Q6_K) {
-    *reinterpret_cast<float4*>(xs.xf + col) = v;
-  } else {
-    const float m = group8_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-    // e with 2^(e-1) <= m < 2^e from the exponent field (m = 0 or subnormal: the
-    // clamp at -100 makes every X round to 0, as it must); both scales are
-    // normal powers of two built from their exponent fields.
-    int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 126;
-    if (e < -100) e = -100;
-    const float up = __uint_as_float((uint32_t)(127 + 22 - e) << 23);
-    const int X[4] = {__float2int_rn(v.x * up), __float2int_rn(v.y * up), __float2int_rn(v.z * up),
-                      __float2int_rn(v.w * up)};
-    uint32_t w0 = 0, w1 = 0, w2 = 0;
-    int s0 = 0, s1 = 0, s2 = 0;
+  const float m = group8_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  // e with 2^(e-1) <= m < 2^e from the exponent field (m = 0 or subnormal: the
+  // clamp at -100 makes every X round to 0, as it must); both scales are
+  // normal powers of two built from their exponent fields.
+  int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 126;
+  if (e < -100) e = -100;
+  const float up = __uint_as_float((uint32_t)(127 + 22 - e) << 23);
+  const int X[4] = {__float2int_rn(v.x * up), __float2int_rn(v.y * up), __float2int_rn(v.z * up),
+                    __float2int_rn(v.w * up)};
+  uint32_t w0 = 0, w1 = 0, w2 = 0;
+  int s0 = 0, s1 = 0, s2 = 0;
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const uint32_t b0 = (uint32_t)X[t] & 0xFFu, b1 = ((uint32_t)X[t] >> 8) & 0xFFu;
-      const int hi = X[t] >> 16;  // arithmetic: in [-64, 64]
-      w0 |= b0 << (8 * t);
-      w1 |= b1 << (8 * t);
-      w2 |= ((uint32_t)hi & 0xFFu) << (8 * t);
-      s0 += (int)b0;
-      s1 += (int)b1;
-      s2 += hi;
-    }
-    const int c = (int)(col / kSliceCols), u = (int)(col % kSliceCols);
-    const int l = u / 64, k = (u % 64) / 4;
-    const int wi = k * xs.np + c * 32 + l;
-    xs.wd[wi] = w0;
-    xs.wd[16 * xs.np + wi] = w1;
-    xs.wd[32 * xs.np + wi] = w2;
-    const int64_t B = col / 32;
-    if constexpr (QT == QT_Q4_0) {
-      s0 = group8_sum(s0);
-      s1 = group8_sum(s1);
-      s2 = group8_sum(s2);
-      if ((lane & 7) == 0) {
-        xs.cr[3 * B + 0] = -8 * s0;
-        xs.cr[3 * B + 1] = -8 * s1;
-        xs.cr[3 * B + 2] = -8 * s2;
-      }
-    }
-    if ((lane & 7) == 0) xs.sc[B] = __uint_as_float((uint32_t)(127 + e - 22) << 23);
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t b0 = (uint32_t)X[t] & 0xFFu, b1 = ((uint32_t)X[t] >> 8) & 0xFFu;
+    const int hi = X[t] >> 16;  // arithmetic: in [-64, 64]
+    w0 |= b0 << (8 * t);
+    w1 |= b1 << (8 * t);
+    w2 |= ((uint32_t)hi & 0xFFu) << (8 * t);
+    s0 += (int)b0;
+    s1 += (int)b1;
+    s2 += hi;
   }
+  const int c = (int)(col / kSliceCols), u = (int)(col % kSliceCols);
+  // owning lane l and word k (Q8_0/Q4_0: lane l has columns 64 l .. 64 l + 63;
+  // Q6_K: see rowfix_q6_k)
+  int l, k;
+  if constexpr (QT == QT_Q6_K) {
+    const int g = (u % 128) / 32;
+    l = 4 * (u / 256) + 2 * ((u % 256) / 128) + (u % 32) / 16;
+    k = 4 * g + (u % 16) / 4;
+  } else {
+    l = u / 64;
+    k = (u % 64) / 4;
+  }
+  const int wi = k * xs.np + c * 32 + l;
+  xs.wd[wi] = w0;
+  xs.wd[16 * xs.np + wi] = w1;
+  xs.wd[32 * xs.np + wi] = w2;
+  const int64_t B = col / 32;
+  if constexpr (QT == QT_Q4_0) {
+    s0 = group8_sum(s0);
+    s1 = group8_sum(s1);
+    s2 = group8_sum(s2);
+    if ((lane & 7) == 0) {
+      xs.cr[3 * B + 0] = -8 * s0;
+      xs.cr[3 * B + 1] = -8 * s1;
+      xs.cr[3 * B + 2] = -8 * s2;
+    }
+  }
+  if constexpr (QT == QT_Q6_K) {
+    // per 16-column run (4 lanes): -32 times the limb sums
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+    s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
+    if ((lane & 3) == 0) {
+      int* cc = xs.cr + ((int64_t)(c * 32 + l) * 4 + (u % 128) / 32) * 3;
+      cc[0] = -32 * s0;
+      cc[1] = -32 * s1;
+      cc[2] = -32 * s2;
+    }
+  }
+  if ((lane & 7) == 0) xs.sc[B] = __uint_as_float((uint32_t)(127 + e - 22) << 23);
 }
 
 // K is a multiple of 256 on every path that stages x.
@@ -543,15 +599,30 @@ struct XRegs {
 };
 template <>
 struct XRegs<QT_Q6_K> {
-  f32x2 x2[32];
+  XFix6 x;
   __device__ __forceinline__ void load(const XStage& xs, int c, int lane) {
-    load_x_slice_q6_k(ProSmem{xs.xf}, (int64_t)c * kSliceCols, lane, x2);
+    const int idx = c * 32 + lane;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      x.l0[k] = xs.wd[(0 * 16 + k) * xs.np + idx];
+      x.l1[k] = xs.wd[(1 * 16 + k) * xs.np + idx];
+      x.l2[k] = xs.wd[(2 * 16 + k) * xs.np + idx];
+    }
+    const int B0 = c * 64 + 8 * (lane >> 2) + 4 * ((lane >> 1) & 1);  // block of run 0
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      x.xs[g] = xs.sc[B0 + g];
+      const int* cc = xs.cr + ((int64_t)idx * 4 + g) * 3;
+      x.c[g][0] = cc[0];
+      x.c[g][1] = cc[1];
+      x.c[g][2] = cc[2];
+    }
   }
   template <class Pro>
   __device__ __forceinline__ void load_direct(const Pro& pro, int c, int lane) {
-    load_x_slice_q6_k(pro, (int64_t)c * kSliceCols, lane, x2);
+    fix6_direct(pro, (int64_t)c * kSliceCols, lane, x);
   }
-  __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const { return row_q6_k(seg, lane, x2); }
+  __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const { return rowfix_q6_k(seg, lane, x); }
 };
 
 // ------------------------------------------------------------- epilogues
