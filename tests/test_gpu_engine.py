@@ -316,3 +316,44 @@ def test_engine_phase_probe_records_every_phase_in_order():
     e.run([-1], pos0=2, flags=ntx.NTX_NO_GRAPH)
     assert int(ts.abs().sum()) == 0
     e.close()
+
+
+def test_engine_skip_every_layer_and_none():
+    """Degenerate skip sets on the persistent kernel: tau -1 skips every layer
+    (embed feeds the head directly), tau 2 skips none."""
+    d = dict(TINY, n_layers=3)
+    m = DeviceModel(d, ntx.NTX_Q8_0, ntx.NTX_Q8_0, 53, max_ctx=16, n_prior=0, source="host")
+    prompt = list(sg.tokens(53, "prompt", 2, d["vocab"]))
+    for tau, n_skip in ((-1.0, d["n_layers"]), (2.0, 0)):
+        m.reset_kv()
+        e = Engine(m, tau=tau)
+        lg_a, fed_a, nxt_a, _ = e.run(prompt[:1])
+        lg_c, fed_c, nxt_c, _ = e.run(prompt[1:], pos0=1, flags=ntx.NTX_CALIBRATE_SKIP)
+        mask = ntx.ntx_engine_skip_mask(e.h, d["n_layers"])
+        lg_s, fed_s, nxt_s, _ = e.run([-1, -1], pos0=2, flags=ntx.NTX_USE_SKIP)
+        assert ntx.ntx_engine_launches_per_step(e.h) == 1
+        e.close()
+        assert sum(mask) == n_skip
+        m.reset_kv()
+        fed = fed_a + fed_c + fed_s
+        ref, _ = oracle_run(m, fed, skip=[None, None, mask, mask])
+        lg = np.concatenate([lg_a, lg_c, lg_s])
+        greedy = list(nxt_a) + list(nxt_c) + list(nxt_s)
+        for s in range(len(fed)):
+            check_logits(lg[s], ref[s], int(greedy[s]), s)
+
+
+def test_engine_falls_back_to_chain_beyond_persistent_limits():
+    """FFN 30720 needs 15 slices of 2048 columns, one more than the persistent
+    kernel's consumer warps: the engine runs the per-op chain, same results."""
+    d = dict(TINY, ffn=30720, n_layers=1)
+    m = DeviceModel(d, ntx.NTX_Q8_0, ntx.NTX_Q8_0, 55, max_ctx=8, n_prior=0, source="host")
+    toks = list(sg.tokens(55, "prompt", 2, d["vocab"])) + [-1]
+    e = Engine(m)
+    lg, fed, nxt, _ = e.run(toks)
+    assert ntx.ntx_engine_launches_per_step(e.h) > 1
+    assert ntx.ntx_engine_set_phase_probe(e.h, None, 0) == 0  # no persistent kernel
+    e.close()
+    ref, _ = oracle_run(m, fed)
+    for s in range(len(fed)):
+        check_logits(lg[s], ref[s], int(nxt[s]), s)
