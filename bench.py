@@ -431,10 +431,12 @@ def run_ntx(args, dist: Dist):
     return out
 
 
-def time_gemv(ntx, sg, wl, torch, qt, M, K, reps=40):
+def time_gemv(ntx, sg, wl, torch, qt, M, K, reps=40, pdl=False):
     """Device time of one GEMV: `n` back-to-back launches over rotating weight
     copies (more than 3x L2 in total) captured in one CUDA graph, replayed, so
-    the host's per-call cost does not set the pace."""
+    the host's per-call cost does not set the pace.  pdl: launches made with
+    programmatic dependent launch (ntx_set_gemv_pdl), so each GEMV starts
+    streaming its weights while the previous one drains."""
     L2 = 126 * 2 ** 20
     wbytes = wl.mat_bytes(qt, M, K)
     ncopy = max(2, (3 * L2) // wbytes + 1)
@@ -447,14 +449,19 @@ def time_gemv(ntx, sg, wl, torch, qt, M, K, reps=40):
     x = torch.randn(K, device="cuda")
     y = torch.empty(M, device="cuda")
     s = torch.cuda.current_stream()
-    for i in range(4):
-        ntx.ntx_gemv_q(qt, Ws[i % ncopy], M, K, x, y, None, s)
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        cap = torch.cuda.current_stream()
-        for i in range(n):
-            ntx.ntx_gemv_q(qt, Ws[i % ncopy], M, K, x, y, None, cap)
+    ntx.ntx_set_gemv_pdl(1 if pdl else 0)
+    try:
+        for i in range(4):
+            ntx.ntx_gemv_q(qt, Ws[i % ncopy], M, K, x, y, None, s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            cap = torch.cuda.current_stream()
+            for i in range(n):
+                ntx.ntx_gemv_q(qt, Ws[i % ncopy], M, K, x, y, None, cap)
+    finally:
+        ntx.ntx_set_gemv_pdl(0)
     g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -471,13 +478,17 @@ def time_gemv(ntx, sg, wl, torch, qt, M, K, reps=40):
 
 
 def gemv_sweep(ntx, sg, wl, torch, peak):
-    shapes = [(8, 4096, 4096, "config 1")] + [(2, M, K, "config 2") for M, K in wl.Q4_0_SWEEP]
+    shapes = [(8, 4096, 4096, "Q8_0 GEMV 4096x4096, batch 1")] + [(2, M, K, "Q4_0 GEMV sweep over Llama-3-8B projection shapes, batch 1") for M, K in wl.Q4_0_SWEEP]
     out = []
     for qt, M, K, name in shapes:
-        ms, nbytes, ncopy = time_gemv(ntx, sg, wl, torch, qt, M, K)
+        ms, nbytes, ncopy = time_gemv(ntx, sg, wl, torch, qt, M, K, pdl=True)
+        ms_s, _, _ = time_gemv(ntx, sg, wl, torch, qt, M, K, pdl=False)
         gbs = nbytes / (ms * 1e-3) / 1e9
+        gbs_s = nbytes / (ms_s * 1e-3) / 1e9
         out.append({"workload": name, "qtype": {8: "Q8_0", 2: "Q4_0"}[qt], "M": M, "K": K, "us": round(ms * 1e3, 3),
                     "GBs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                    "launch": "programmatic dependent launch (ntx_set_gemv_pdl(1))",
+                    "us_serial": round(ms_s * 1e3, 3), "frac_serial": round(gbs_s / peak, 4),
                     "rotation": f"{ncopy} weight copies (>3x L2), back-to-back launches in one CUDA graph"})
     return out
 
@@ -568,7 +579,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ntx", "reference"], default="ntx")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama8b-q8_0")
-    ap.add_argument("--no-gemv", action="store_true", help="skip the config 1-2 GEMV sweep")
+    ap.add_argument("--no-gemv", action="store_true", help="skip the standalone Q8_0 / Q4_0 GEMV sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-chain", action="store_true", help="skip timing the per-op kernel chain for comparison")
     ap.add_argument("--layers", type=int, default=None,

@@ -85,6 +85,17 @@ NTX_API int ntx_sm_count(void);
  * after the call, process-wide.  Workspace sizes do not depend on it. */
 NTX_API int ntx_set_gemv_ctas_per_sm(int ctas_per_sm);
 
+/* Tuning: programmatic dependent launch for ntx_gemv_q (0 = off, the
+ * default; 1 = on), for calls made after it, process-wide.  When on, a
+ * ntx_gemv_q kernel may start while the kernels enqueued before it on the
+ * same stream are still running: it begins streaming W at once, and reads x,
+ * reads residual and writes y only after those kernels have completed.  So,
+ * while it is on, W must not be written by any kernel enqueued on the stream
+ * since the last host synchronisation of that stream (weights that stay
+ * fixed meet this).  Back-to-back GEMVs then overlap one launch's start with
+ * the previous one's tail.  NTX_ERR_INVALID_ARG for other values. */
+NTX_API int ntx_set_gemv_pdl(int on);
+
 /* ------------------------------------------------------------ per-op calls */
 
 /* Dequantize n weights ([README] 主な機能: GGUF Q4_0/Q8_0/Q6_K; [ShowHN]

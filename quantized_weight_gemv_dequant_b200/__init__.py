@@ -33,7 +33,7 @@ BLOCK_BYTES = {NTX_Q4_0: 18, NTX_Q8_0: 34, NTX_Q6_K: 210}
 
 # Symbols exported by libntx (all declared in include/ntx.h).
 EXPORTS = (
-    "ntx_last_error", "ntx_version", "ntx_device_status", "ntx_sm_count", "ntx_set_gemv_ctas_per_sm",
+    "ntx_last_error", "ntx_version", "ntx_device_status", "ntx_sm_count", "ntx_set_gemv_ctas_per_sm", "ntx_set_gemv_pdl",
     "ntx_dequant", "ntx_gemv_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_workspace_bytes", "ntx_attn_decode",
     "ntx_swiglu", "ntx_layer_layout", "ntx_layer_workspace_bytes", "ntx_decode_layer", "ntx_engine_workspace_bytes",
     "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
@@ -79,6 +79,7 @@ def lib():
             "ntx_device_status": ([P(ctypes.c_int)], i32),
             "ntx_sm_count": ([], i32),
             "ntx_set_gemv_ctas_per_sm": ([i32], i32),
+            "ntx_set_gemv_pdl": ([i32], i32),
             "ntx_dequant": ([i32, vp, vp, i64, vp], i32),
             "ntx_gemv_q": ([i32, vp, i64, i64, vp, vp, vp, vp], i32),
             "ntx_rmsnorm": ([vp, vp, vp, i64, f32, vp], i32),
@@ -155,6 +156,10 @@ def ntx_sm_count() -> int:
 
 def ntx_set_gemv_ctas_per_sm(cps: int) -> None:
     _check(lib().ntx_set_gemv_ctas_per_sm(cps))
+
+
+def ntx_set_gemv_pdl(on: int) -> None:
+    _check(lib().ntx_set_gemv_pdl(on))
 
 
 def ntx_dequant(qtype, blocks, out, n, stream=None):

@@ -152,13 +152,19 @@ int ntx_gemv_q(int qtype, const void* W, int64_t M, int64_t K, const float* x, f
   if (ranges_overlap(x, (size_t)K * 4, y, (size_t)M * 4)) return fail(NTX_ERR_INVALID_ARG, "y overlaps x");
   if (residual && residual != y && ranges_overlap(residual, (size_t)M * 4, y, (size_t)M * 4))
     return fail(NTX_ERR_INVALID_ARG, "residual partially overlaps y");
-  const cudaError_t e = ntx::launch_gemv(qtype, W, M, K, x, y, residual, S(stream), false);
+  const cudaError_t e = ntx::launch_gemv(qtype, W, M, K, x, y, residual, S(stream), ntx::gemv_pdl());
   return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_gemv_q");
 }
 
 int ntx_set_gemv_ctas_per_sm(int cps) {
   if (cps < 1 || cps > 4) return fail(NTX_ERR_INVALID_ARG, "ctas per SM must be 1..4");
   ntx::set_gemv_ctas_per_sm(cps);
+  return NTX_OK;
+}
+
+int ntx_set_gemv_pdl(int on) {
+  if (on != 0 && on != 1) return fail(NTX_ERR_INVALID_ARG, "programmatic launch switch must be 0 or 1");
+  ntx::set_gemv_pdl(on == 1);
   return NTX_OK;
 }
 

@@ -17,6 +17,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 int g_sms[kMaxDevices];
 int g_cps = 1;
+bool g_gemv_pdl = false;
 std::mutex g_mu;
 
 int current_device() {
@@ -138,6 +139,8 @@ int sm_count() {
 
 void set_gemv_ctas_per_sm(int cps) { g_cps = cps < 1 ? 1 : (cps > 4 ? 4 : cps); }
 int gemv_ctas_per_sm() { return g_cps; }
+void set_gemv_pdl(bool on) { g_gemv_pdl = on; }
+bool gemv_pdl() { return g_gemv_pdl; }
 
 int gemv_grid(int64_t M, int align) {
   const int64_t units = (M + align - 1) / align;

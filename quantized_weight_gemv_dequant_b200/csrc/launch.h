@@ -9,6 +9,8 @@ namespace ntx {
 int sm_count();
 void set_gemv_ctas_per_sm(int cps);
 int gemv_ctas_per_sm();
+void set_gemv_pdl(bool on);
+bool gemv_pdl();
 
 // Grid of a GEMV over M logical rows (rows grouped in pairs when align == 2).
 int gemv_grid(int64_t M, int align);

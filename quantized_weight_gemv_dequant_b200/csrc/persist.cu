@@ -520,6 +520,46 @@ struct Epilogue {
 };
 
 // ------------------------------------------------------------ consumers
+// Per-lane partial scores of one K row for the G query heads of a group:
+// lane l holds dimensions 4l .. 4l + 3 (kp points at them, fp16).
+template <int G>
+__device__ __forceinline__ void score_parts(const uint8_t* kp, const float (&qr)[G][4], float (&v)[G]) {
+  const uint2 kr = *reinterpret_cast<const uint2*>(kp);
+  const float k0 = half_bits_to_float(kr.x), k1 = half_bits_to_float(kr.x >> 16);
+  const float k2 = half_bits_to_float(kr.y), k3 = half_bits_to_float(kr.y >> 16);
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float d = qr[h][0] * k0;
+    d = fmaf(qr[h][1], k1, d);
+    d = fmaf(qr[h][2], k2, d);
+    d = fmaf(qr[h][3], k3, d);
+    v[h] = d;
+  }
+}
+
+// Warp sums of G values at once: each halving step exchanges half of the
+// remaining values with the partner lane (lanes with bit o set keep the upper
+// half), then plain butterfly steps finish the sums.  On return lane l holds
+// the full sum of head l / (32 / G).  log2(G) + 5 - log2(G) steps, G - 1 + 5 -
+// log2(G) shuffles in all.
+template <int G>
+__device__ __forceinline__ float heads_reduce(float (&v)[G], int lane) {
+#pragma unroll
+  for (int n = G, o = 16; n > 1; n >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = up ? v[j] : v[j + n / 2];
+      const float keep = up ? v[j + n / 2] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float s = v[0];
+#pragma unroll
+  for (int o = 16 / G; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
 template <int QT>
 struct Consumer {
   const PStep& st;
@@ -655,24 +695,63 @@ struct Consumer {
     if (ctid == 0) st.stats_embed[blockIdx.x * 4] = ss;
   }
 
+  // Splits of this step's context per KV head: at least kPMinSplit positions
+  // each where possible, at most n_split (one unit per CTA).
+  __device__ void attn_splits(int n_ctx, int& ns, int& chunk) const {
+    ns = (n_ctx + kPMinSplit - 1) / kPMinSplit;
+    if (ns > st.n_split) ns = st.n_split;
+    chunk = (n_ctx + ns - 1) / ns;
+  }
+
+  // Brings the K and V rows this CTA's attention units will read (the
+  // positions before this step's) into L2, so the attention phase's tile
+  // loads hit L2.  Issued by one thread at the start of the layer's Q/K/V phase.
+  __device__ void kv_prefetch(const LRow& L) const {
+    const int n_ctx = st.params[0] + 1;
+    int ns, chunk;
+    attn_splits(n_ctx, ns, chunk);
+    for (int u = blockIdx.x; u < st.Hkv * ns; u += gridDim.x) {
+      const int kvh = u / ns, split = u % ns;
+      const int p0 = split * chunk;
+      const int p1 = min(p0 + chunk, n_ctx - 1);
+      for (int c0 = p0; c0 < p1; c0 += 128) {  // 32 KB per request
+        const uint32_t bytes = (uint32_t)(min(p1 - c0, 128) * kPD * 2);
+        const int64_t off = ((int64_t)kvh * st.max_ctx + c0) * kPD;
+        l2_prefetch(L.kc + off, bytes);
+        l2_prefetch(L.vc + off, bytes);
+      }
+    }
+  }
+
   // Split-KV attention.  This step's context is cut into ns splits per KV
-  // head (at least kPMinSplit positions each, at most one unit per CTA where
-  // the grid allows); a unit walks its positions in tiles of kPChunk rows of
+  // head (attn_splits); a unit walks its positions in tiles of kPChunk rows of
   // K and V (contiguous in the cache, brought to shared memory with 16-byte
-  // asynchronous copies) with a running max and sum (online softmax).  With
-  // one split the unit writes the head output; otherwise it writes its
-  // (max, sum, unnormalised output) and the last unit of each KV head to
-  // finish merges the splits (log-sum-exp).
+  // asynchronous copies) with a running max and sum (online softmax).
+  // Scores: a warp per position and group of at most 4 query heads (two
+  // positions in flight), each lane 4 dimensions of each of those heads,
+  // reduced for all of them at once (heads_reduce).
+  // P V: thread (d8, h, pg) keeps dimensions 8 d8 .. 8 d8 + 7 of head h over
+  // the tile positions pg, pg + NPG, ...; the NPG position groups are summed
+  // in a fixed order at the end of the unit.  With one split the unit writes
+  // the head output; otherwise it writes its (max, sum, unnormalised output)
+  // and the last unit of each KV head to finish merges the splits
+  // (log-sum-exp).
   template <int G>
   __device__ void attention(const LRow& L, int lk) {
     const int n_ctx = st.params[0] + 1;
-    int ns = (n_ctx + kPMinSplit - 1) / kPMinSplit;
-    if (ns > st.n_split) ns = st.n_split;
-    const int chunk = (n_ctx + ns - 1) / ns;
+    int ns, chunk;
+    attn_splits(n_ctx, ns, chunk);
     const AttnSmem a = attn_smem(sm.xst, G);
     const int units = st.Hkv * ns;
     const int S = kAttnPartStride;
-    constexpr int kOP = (G * (kPD / 2) + kPCThreads - 1) / kPCThreads;  // (head, dim pair)s per thread
+    constexpr int NPG = kPCThreads / (16 * G);  // P V position groups
+    constexpr int GW = G < 4 ? G : 4;           // query heads per warp in the score step
+    constexpr int NH = G / GW;                  // warps per position (head groups)
+    constexpr int WPG = kPConsumers / NH;       // warps per head group
+    constexpr int LPH = 32 / GW;                // lanes holding one head's score after heads_reduce
+    const int hh0 = (warp % NH) * GW, wpos = warp / NH;
+    const int d8 = ctid % 16, hv = (ctid / 16) % G, pg = ctid / (16 * G);
+    const bool pv_on = pg < NPG;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       const int kvh = u / ns, split = u % ns;
       const int p0 = split * chunk;
@@ -680,19 +759,14 @@ struct Consumer {
       const int np = p1 > p0 ? p1 - p0 : 0;
       const uint8_t* kbase = reinterpret_cast<const uint8_t*>(L.kc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
       const uint8_t* vbase = reinterpret_cast<const uint8_t*>(L.vc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
-      float qr[G][4];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float4 t = __ldcg(reinterpret_cast<const float4*>(st.q + (int64_t)(kvh * G + h) * kPD + 4 * lane));
-        qr[h][0] = t.x; qr[h][1] = t.y; qr[h][2] = t.z; qr[h][3] = t.w;
-      }
+      const float* qg = st.q + (int64_t)kvh * G * kPD + 4 * lane;
       if (ctid < G) {
         a.ml[2 * ctid] = -INFINITY;
         a.ml[2 * ctid + 1] = 0.f;
       }
-      float o[kOP][2];
+      float o[8];
 #pragma unroll
-      for (int k = 0; k < kOP; ++k) o[k][0] = o[k][1] = 0.f;
+      for (int k = 0; k < 8; ++k) o[k] = 0.f;
       cons_bar();  // the running (max, sum) start values are visible
       for (int t0 = 0; t0 < np; t0 += kPChunk) {
         const int nt = min(kPChunk, np - t0);
@@ -705,22 +779,31 @@ struct Consumer {
             cp_async16((isv ? a.v : a.k) + ob, (isv ? vbase : kbase) + off + ob);
           }
           cp_async_commit();
-          cp_async_wait_all();
         }
-        cons_bar();
-        // scores: a warp per position, lanes split the head dimension
-        for (int i = warp; i < nt; i += kPConsumers) {
-          const uint2 kr = *reinterpret_cast<const uint2*>(a.k + (size_t)i * kPD * 2 + 8 * lane);
-          const float k0 = half_bits_to_float(kr.x), k1 = half_bits_to_float(kr.x >> 16);
-          const float k2 = half_bits_to_float(kr.y), k3 = half_bits_to_float(kr.y >> 16);
+        // this lane's 4 dimensions of every query head of the group, loaded
+        // per tile (L2) while the tile lands, so they are not held through P V
+        float qr[GW][4];
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float d = qr[h][0] * k0;
-            d = fmaf(qr[h][1], k1, d);
-            d = fmaf(qr[h][2], k2, d);
-            d = fmaf(qr[h][3], k3, d);
-            d = warp_sum(d);
-            if (lane == 0) a.sc[h * kPChunk + i] = d * kAttnScale;
+        for (int h = 0; h < GW; ++h) {
+          const float4 t = __ldcg(reinterpret_cast<const float4*>(qg + (hh0 + h) * kPD));
+          qr[h][0] = t.x; qr[h][1] = t.y; qr[h][2] = t.z; qr[h][3] = t.w;
+        }
+        cp_async_wait_all();
+        cons_bar();
+        for (int i = wpos; i < nt; i += 2 * WPG) {
+          const int i2 = i + WPG;
+          const bool two = i2 < nt;  // warp-uniform
+          float v1[GW], v2[GW];
+          score_parts<GW>(a.k + (size_t)i * kPD * 2 + 8 * lane, qr, v1);
+          if (two) score_parts<GW>(a.k + (size_t)i2 * kPD * 2 + 8 * lane, qr, v2);
+          else {
+#pragma unroll
+            for (int h = 0; h < GW; ++h) v2[h] = 0.f;
+          }
+          const float s1 = heads_reduce<GW>(v1, lane), s2 = heads_reduce<GW>(v2, lane);
+          if (lane % LPH == 0) {
+            a.sc[(hh0 + lane / LPH) * kPChunk + i] = s1 * kAttnScale;
+            if (two) a.sc[(hh0 + lane / LPH) * kPChunk + i2] = s2 * kAttnScale;
           }
         }
         cons_bar();
@@ -745,52 +828,53 @@ struct Consumer {
           }
         }
         cons_bar();
-        // P V: thread pair (h, d2) keeps dims 2 d2, 2 d2 + 1 of head h
+        if (pv_on) {
+          const float f = a.fac[hv];
 #pragma unroll
-        for (int k = 0; k < kOP; ++k) {
-          const int idx = ctid + k * kPCThreads;
-          if (idx < G * (kPD / 2)) {
-            const int h = idx / (kPD / 2), d2 = idx % (kPD / 2);
-            const float* e = a.sc + h * kPChunk;
-            const float f = a.fac[h];
-            float o0 = o[k][0] * f, o1 = o[k][1] * f;
-            for (int i = 0; i < nt; ++i) {
-              const uint32_t wv = *reinterpret_cast<const uint32_t*>(a.v + (size_t)i * kPD * 2 + 4 * d2);
-              o0 = fmaf(e[i], half_bits_to_float(wv), o0);
-              o1 = fmaf(e[i], half_bits_to_float(wv >> 16), o1);
-            }
-            o[k][0] = o0;
-            o[k][1] = o1;
+          for (int k = 0; k < 8; ++k) o[k] *= f;
+          const float* e = a.sc + hv * kPChunk;
+          for (int i = pg; i < nt; i += NPG) {
+            const uint4 w = *reinterpret_cast<const uint4*>(a.v + (size_t)i * kPD * 2 + 16 * d8);
+            const float ei = e[i];
+            o[0] = fmaf(ei, half_bits_to_float(w.x), o[0]);
+            o[1] = fmaf(ei, half_bits_to_float(w.x >> 16), o[1]);
+            o[2] = fmaf(ei, half_bits_to_float(w.y), o[2]);
+            o[3] = fmaf(ei, half_bits_to_float(w.y >> 16), o[3]);
+            o[4] = fmaf(ei, half_bits_to_float(w.z), o[4]);
+            o[5] = fmaf(ei, half_bits_to_float(w.z >> 16), o[5]);
+            o[6] = fmaf(ei, half_bits_to_float(w.w), o[6]);
+            o[7] = fmaf(ei, half_bits_to_float(w.w >> 16), o[7]);
           }
         }
         cons_bar();  // the next tile overwrites K, V and the scores
       }
-      if (ns == 1) {
-#pragma unroll
-        for (int k = 0; k < kOP; ++k) {
-          const int idx = ctid + k * kPCThreads;
-          if (idx < G * (kPD / 2)) {
-            const int h = idx / (kPD / 2), d2 = idx % (kPD / 2);
-            const float inv = 1.0f / a.ml[2 * h + 1];
-            *reinterpret_cast<float2*>(st.attn_out + (int64_t)(kvh * G + h) * kPD + 2 * d2) =
-                make_float2(o[k][0] * inv, o[k][1] * inv);
-          }
-        }
-        cons_bar();  // scratch reuse by the next unit
-        continue;
+      // the position groups' partial outputs -> the K tile buffer ([NPG][G][128] floats)
+      float* pr = reinterpret_cast<float*>(a.k);
+      if (pv_on) {
+        float4* dst = reinterpret_cast<float4*>(pr + ((size_t)pg * G + hv) * kPD + 8 * d8);
+        dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_float4(o[4], o[5], o[6], o[7]);
       }
-#pragma unroll
-      for (int k = 0; k < kOP; ++k) {
-        const int idx = ctid + k * kPCThreads;
-        if (idx < G * (kPD / 2)) {
-          const int h = idx / (kPD / 2), d2 = idx % (kPD / 2);
+      cons_bar();
+      for (int idx = ctid; idx < G * kPD; idx += kPCThreads) {
+        const int h = idx / kPD, d = idx % kPD;
+        float sum = 0.f;
+#pragma unroll 4
+        for (int g2 = 0; g2 < NPG; ++g2) sum += pr[((size_t)g2 * G + h) * kPD + d];
+        if (ns == 1) {
+          st.attn_out[(int64_t)(kvh * G + h) * kPD + d] = sum / a.ml[2 * h + 1];
+        } else {
           float* dst = st.attn_part + ((int64_t)(kvh * G + h) * ns + split) * S;
-          *reinterpret_cast<float2*>(dst + 2 + 2 * d2) = make_float2(o[k][0], o[k][1]);
-          if (d2 == 0) {
+          dst[2 + d] = sum;
+          if (d == 0) {
             dst[0] = a.ml[2 * h];
             dst[1] = a.ml[2 * h + 1];
           }
         }
+      }
+      if (ns == 1) {
+        cons_bar();  // scratch reuse by the next unit
+        continue;
       }
       // publish this split (release by one thread after the CTA barrier)
       cons_bar();
@@ -1047,6 +1131,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
           break;
         }
         default: {  // GEMV phases
+          if (kind == PK_QKV && ctid == kPCThreads - 32) cs.kv_prefetch(*L);
           const float* h = kind == PK_GU ? st.h1 : kind == PK_O ? st.attn_out : kind == PK_DOWN ? st.u : st.hidden;
           const float* w = kind == PK_QKV ? L->attn_norm : kind == PK_GU ? L->ffn_norm
                            : kind == PK_HEAD ? st.final_norm : nullptr;

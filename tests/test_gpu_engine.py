@@ -256,7 +256,7 @@ def test_engine_cosine_skip_calibration():
 
 
 @pytest.mark.slow
-def test_engine_config_4_llama8b_q8_0_144_steps():
+def test_engine_llama8b_q8_0_144_steps():
     """Config 4: 32-layer 8B-shaped Q8_0 model, 16-token prompt + 128 greedy
     steps (KV grows to 144), checked teacher-forced over all 144 steps.  The
     model is made by the generator's CUDA twin; sampled rows of every tensor are

@@ -35,7 +35,7 @@ def _gpu():
     assert ntx.ntx_device_status() == 0
 
 
-def test_engine_config_5_llama70b_q6_k_resident_and_tiered_with_skip():
+def test_engine_llama70b_q6_k_resident_and_tiered_with_skip():
     d = dict(wl.MODEL_70B)
     L = d["n_layers"]
     sd = wl.seed(5)

@@ -143,7 +143,7 @@ def test_gemv_exact_on_grid(qtype):
     assert np.array_equal(got, ref)
 
 
-def test_gemv_config_1_q8_0_4096():
+def test_gemv_q8_0_4096x4096():
     M = K = 4096
     W = sg.quant_rows(Q8_0, wl.seed(1), "W", M, K)
     x = sg.fill_f32(wl.seed(1), "x", K)
@@ -151,7 +151,7 @@ def test_gemv_config_1_q8_0_4096():
 
 
 @pytest.mark.parametrize("M,K", wl.Q4_0_SWEEP)
-def test_gemv_config_2_q4_0_sweep(M, K):
+def test_gemv_q4_0_llama8b_projection_shapes(M, K):
     W = sg.quant_rows(Q4_0, wl.seed(2), f"W{M}x{K}", M, K)
     x = sg.fill_f32(wl.seed(2), f"x{K}", K)
     gemv_check(Q4_0, W, M, K, x)
@@ -173,6 +173,39 @@ def test_gemv_ctas_per_sm_same_result(cps):
         ntx.ntx_set_gemv_ctas_per_sm(1)
     _sync()
     assert np.array_equal(y1.cpu().numpy(), y2.cpu().numpy())  # each row is one warp's sum either way
+
+
+def test_gemv_pdl_back_to_back_matches_oracle():
+    """Programmatic launch on: a chain of GEMVs on one stream, each reading the
+    previous one's output as x (the dependent reads wait for it), every y
+    checked against the oracle."""
+    M = K = 4096
+    Ws = [sg.quant_rows(q, 11, f"pdl{i}", M, K) for i, q in enumerate([Q8_0, Q4_0, Q6_K, Q8_0])]
+    qts = [Q8_0, Q4_0, Q6_K, Q8_0]
+    x0 = sg.fill_f32(11, "pdlx", K)
+    Wd = [dev(w) for w in Ws]
+    ys = [dev(np.zeros(M, dtype=np.float32)) for _ in Ws]
+    _sync()
+    ntx.ntx_set_gemv_pdl(1)
+    try:
+        xin = dev(x0)
+        for q, w, y in zip(qts, Wd, ys):
+            ntx.ntx_gemv_q(q, w, M, K, xin, y)
+            xin = y
+        _sync()
+    finally:
+        ntx.ntx_set_gemv_pdl(0)
+    x = x0.astype(np.float64)
+    for q, w, y in zip(qts, Ws, ys):
+        got = y.cpu().numpy()
+        ref, b = oracle.gemv(q, w, M, K, x.astype(np.float32).astype(np.float64))
+        assert np.all(np.abs(got.astype(np.float64) - ref) <= 1e-3 * b + 1e-6)
+        x = got.astype(np.float64)
+
+
+def test_gemv_pdl_switch_rejects_other_values():
+    with pytest.raises(ntx.NtxError):
+        ntx.ntx_set_gemv_pdl(2)
 
 
 # ------------------------------------------------------------------ small ops

@@ -106,7 +106,7 @@ def test_layer_long_context_split_combine_path(pos):
     run_layer_case(SMALL, ntx.NTX_Q8_0, 4000 + pos, pos, 4500)
 
 
-def test_layer_config_3_llama8b_q8_0():
+def test_layer_llama8b_q8_0_pos1024():
     """Config 3: the 8B-shaped Q8_0 layer, 1024 prior positions, token at 1024.
     Also checks that the device generator writes this layer bit-identically."""
     import torch
