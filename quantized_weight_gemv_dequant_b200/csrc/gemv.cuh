@@ -125,9 +125,7 @@ struct ProRms {
   }
 };
 
-
 // ------------------------------------------------------------- decoders
-__device__ __forceinline__ float byte_f(uint32_t w, int b) { return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7440u | b)); }
 
 // (2^23 + byte ba of wa, 2^23 + byte bb of wb) as one packed pair.
 __device__ __forceinline__ f32x2 bytes_pair(uint32_t wa, int ba, uint32_t wb, int bb) {
@@ -321,7 +319,7 @@ __device__ __forceinline__ float rowfix_q4_0(const uint8_t* seg, int lane, const
 // run's sum is scaled by its sub-block scale, the block scale of x and d.
 struct XFix6 {
   uint32_t l0[16], l1[16], l2[16];  // word 4g + w = columns 4w..4w+3 of run g
-  float xs[4];                      // 2^(e - 22) of run g's 32-column block
+  float xs;                         // 2^(e - 22) of the lane's 128-column group (all four runs)
   int c[4][3];                      // -32 * sum of run g's limb-j bytes
 };
 
@@ -336,7 +334,6 @@ __device__ __forceinline__ void q6k_run4(const uint32_t* wb, int o, uint32_t sh,
   for (int k = 0; k < 4; ++k) w[k] = __funnelshift_r(a[k], a[k + 1], sh);
 }
 
-__device__ __forceinline__ float i8_to_f(uint32_t w, int b) { return byte_f(w ^ 0x80808080u, b) - 8388736.0f; }
 
 __device__ __forceinline__ float rowfix_q6_k(const uint8_t* seg, int lane, const XFix6& x) {
   const int sb = lane >> 2, h = (lane >> 1) & 1, r16 = lane & 1;
@@ -344,11 +341,16 @@ __device__ __forceinline__ float rowfix_q6_k(const uint8_t* seg, int lane, const
   const uint32_t* wb = reinterpret_cast<const uint32_t*>(seg + (boff & ~3u));
   const uint32_t sh = (boff & 3u) * 8u;  // 0 or 16
   const uint32_t* sp = wb + ((192 + 8 * h) >> 2);
-  const uint32_t s0 = __funnelshift_r(sp[0], sp[1], sh), s1 = __funnelshift_r(sp[1], sp[2], sh);
+  // the lane's sub-scales (bytes r16 + 2g of scales[8h .. 8h+7]) moved to bytes 0 and 2
+  const uint32_t s0 = __funnelshift_r(sp[0], sp[1], sh) >> (8 * r16);
+  const uint32_t s1 = __funnelshift_r(sp[1], sp[2], sh) >> (8 * r16);
   const float d = half_bits_to_float((wb[208 >> 2] >> sh) & 0xFFFFu);
   uint32_t ql[4], qh[4];
   q6k_run4(wb, 128 + 32 * h + 16 * r16, sh, qh);
-  float acc = 0.f;
+  // The four runs share one fixed-point scale, so each run's exact limb sums
+  // are weighted by its int8 sub-scale in int32 (at most 2^26 in magnitude)
+  // and the row's total is converted once.
+  int A0 = 0, A1 = 0, A2 = 0;
   // runs g = 0, 2 share one ql run (low / high nibbles), then g = 1, 3 the other
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
@@ -366,33 +368,42 @@ __device__ __forceinline__ float rowfix_q6_k(const uint8_t* seg, int lane, const
         a1 = dp4a_uu(q, x.l1[4 * g + k], a1);
         a2 = dp4a_us(q, x.l2[4 * g + k], a2);
       }
-      // sub-block scale: byte r16 + 2g of scales[8h .. 8h+7]
-      const float sc = i8_to_f(g < 2 ? s0 : s1, r16 + 2 * (g & 1));
-      acc = fmaf(sc * x.xs[g], limbs_to_f(a0, a1, a2), acc);
+      const int sc = (int)(int8_t)(((g < 2) ? s0 : s1) >> (16 * (g & 1)));
+      A0 += sc * a0;
+      A1 += sc * a1;
+      A2 += sc * a2;
     }
   }
-  return d * acc;
+  return (d * x.xs) * limbs_to_f(A0, A1, A2);
 }
 
 // A Q6_K lane's x straight from global memory (no shared staging): the lane
-// converts its four runs itself; a run's 32-column block max is the max over
-// its own 16 columns and the partner lane's (lane ^ 1).
+// converts its four runs itself.  The scale is shared by the four 32-column
+// blocks the runs lie in (128 columns): the max over the lane's 64 columns and
+// the partner lane's (lane ^ 1), found in a first pass over the values.
 template <class Pro>
 __device__ __forceinline__ void fix6_direct(const Pro& pro, int64_t c0, int lane, XFix6& x) {
   const int sb = lane >> 2, h = (lane >> 1) & 1, r16 = lane & 1;
+  const int64_t base = c0 + 256 * sb + 128 * h + 16 * r16;
+  float m = 0.f;
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     float4 v[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) v[q] = pro.ld(c0 + 256 * sb + 128 * h + 32 * g + 16 * r16 + 4 * q);
-    float m = 0.f;
+    for (int q = 0; q < 4; ++q) v[q] = pro.ld(base + 32 * g + 4 * q);
 #pragma unroll
     for (int q = 0; q < 4; ++q) m = fmaxf(m, fmaxf(fmaxf(fabsf(v[q].x), fabsf(v[q].y)), fmaxf(fabsf(v[q].z), fabsf(v[q].w))));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 126;
-    if (e < -100) e = -100;
-    const float up = __uint_as_float((uint32_t)(127 + 22 - e) << 23);
-    x.xs[g] = __uint_as_float((uint32_t)(127 + e - 22) << 23);
+  }
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 126;
+  if (e < -100) e = -100;
+  const float up = __uint_as_float((uint32_t)(127 + 22 - e) << 23);
+  x.xs = __uint_as_float((uint32_t)(127 + e - 22) << 23);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = pro.ld(base + 32 * g + 4 * q);
     int s0 = 0, s1 = 0, s2 = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -481,7 +492,10 @@ __device__ __forceinline__ int group8_sum(int v) {
 // packed four columns to a word, stored where the owning lane will read them.
 template <int QT>
 __device__ __forceinline__ void stage_chunk(const float4 v, int64_t col, const XStage& xs, int lane) {
-  const float m = group8_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  // Block max: per 32 columns, except Q6_K, whose lanes' four runs lie in four
+  // blocks of one 128-column chunk and share one scale (this warp's chunk).
+  const float am = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+  const float m = QT == QT_Q6_K ? warp_max(am) : group8_max(am);
   // e with 2^(e-1) <= m < 2^e from the exponent field (m = 0 or subnormal: the
   // clamp at -100 makes every X round to 0, as it must); both scales are
   // normal powers of two built from their exponent fields.
@@ -609,9 +623,9 @@ struct XRegs<QT_Q6_K> {
       x.l2[k] = xs.wd[(2 * 16 + k) * xs.np + idx];
     }
     const int B0 = c * 64 + 8 * (lane >> 2) + 4 * ((lane >> 1) & 1);  // block of run 0
+    x.xs = xs.sc[B0];  // the same for the four runs' blocks
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      x.xs[g] = xs.sc[B0 + g];
       const int* cc = xs.cr + ((int64_t)idx * 4 + g) * 3;
       x.c[g][0] = cc[0];
       x.c[g][1] = cc[1];
