@@ -1184,17 +1184,20 @@ int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int
   const int attn_bytes = (int)((attn_smem_bytes(Gq, ns) + 15) / 16 * 16);
   const int smem_max = 227 * 1024;
   // Choose the slot size.  In order of priority: every phase can use all its
-  // row groups (TR >= consumer warps per slice), at least 3 slots, the most
-  // bytes in flight in the worst phase, then the smaller slot.
+  // row groups (TR >= consumer warps per slice), at least 3 slots, for Q6_K
+  // a slot's rows split evenly over every phase's row groups (its dot
+  // products, not DRAM, set the pace, so a row group left without a row is
+  // lost time), the most bytes in flight in the worst phase, then the smaller
+  // slot.
   int best_Z = 0, best_S = 0;
-  int64_t best_key[4] = {-1, -1, -1, -1};
+  int64_t best_key[5] = {-1, -1, -1, -1, -1};
   for (auto& kz : ks) {
     const int rbz = st->g[kz.kind].row_bytes;
     for (int m = 1; m <= kPMaxTR; ++m) {
       const int Z = m * rbz;
       int xbz = attn_bytes, rf = 0;
       int64_t inflight_min = INT64_MAX;
-      bool okz = true, full_rg = true;
+      bool okz = true, full_rg = true, even = true;
       int TRs[8];
       for (auto& k : ks) {
         PGeom& g = st->g[k.kind];
@@ -1207,6 +1210,7 @@ int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int
         if (nrg_max < 1) nrg_max = 1;
         if (tr < nrg_max) full_rg = false;
         const int nrg = nrg_max > tr ? tr : nrg_max;
+        if (tr % nrg) even = false;
         const bool staged = qtype != QT_Q6_K || nrg > 1;
         if (staged) {
           const int b = (int)((xstage_bytes(qtype, k.K) + 15) / 16 * 16);
@@ -1223,13 +1227,14 @@ int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int
         const int64_t inflight = (int64_t)S * TRs[k.kind] * st->g[k.kind].row_bytes;
         if (inflight < inflight_min) inflight_min = inflight;
       }
-      const int64_t key[4] = {full_rg ? 1 : 0, S >= 3 ? 1 : 0, inflight_min, -(int64_t)Z};
+      const int64_t key[5] = {full_rg ? 1 : 0, S >= 3 ? 1 : 0, (qtype == QT_Q6_K && even) ? 1 : 0, inflight_min,
+                              -(int64_t)Z};
       bool better = false;
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 5; ++i) {
         if (key[i] != best_key[i]) { better = key[i] > best_key[i]; break; }
       }
       if (better) {
-        for (int i = 0; i < 4; ++i) best_key[i] = key[i];
+        for (int i = 0; i < 5; ++i) best_key[i] = key[i];
         best_Z = Z;
         best_S = S;
       }
