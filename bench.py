@@ -34,11 +34,13 @@ sys.path.insert(0, ROOT)
 
 METRIC = "batch-1 decode tok/s; quantized GEMV achieved HBM GB/s vs B200 peak"
 # DRAM bytes read + written per algorithmic byte by the persistent decode
-# kernel, from one ncu capture (--set full) of a 4-layer 8B-shaped Q8_0 case
-# that fits the capture size rule: 1,485,997,056 + 6,683,392 bytes against
-# 1,485,578,240 algorithmic bytes.  The kernel streams every weight byte once,
-# so a full launch's traffic is this ratio times its algorithmic bytes.
-PERSIST_TRAFFIC_RATIO = 1492680448 / 1485578240
+# kernel, from one ncu capture (--set full) per instantiation of a cut-down
+# case that fits the capture size rule: Q8_0, 4 layers of the 8B shapes,
+# 1,485,753,088 + 4,944,128 bytes against 1,485,578,240 algorithmic bytes;
+# Q6_K, 2 layers of the 70B shapes, 2,282,915,584 + 3,851,264 bytes against
+# 2,282,651,648.  The kernel streams every weight byte once, so a full
+# launch's traffic is this ratio times its algorithmic bytes.
+PERSIST_TRAFFIC_RATIO = {8: 1490697216 / 1485578240, 14: 2286766848 / 2282651648}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -285,10 +287,11 @@ def run_ntx(args, dist: Dist):
                 "achieved": round(k_bytes / (k_ms * 1e-3) / 1e9, 1), "peak": peak, "peak_kind": peak_kind,
                 "unit": "GB/s", "frac": round(k_bytes / (k_ms * 1e-3) / 1e9 / peak, 4),
                 "traffic": args.traffic if args.traffic is not None else (
-                    round(PERSIST_TRAFFIC_RATIO * k_bytes) if qt == 8 else None),
-                "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of a 4-layer case of the same "
-                                "kernel, scaled to this launch's algorithmic bytes" if qt == 8 else
-                                "no capture of this instantiation",
+                    round(PERSIST_TRAFFIC_RATIO[qt] * k_bytes) if qt in PERSIST_TRAFFIC_RATIO else None),
+                "traffic_note": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of a "
+                                 + ("4-layer" if qt == 8 else "2-layer")
+                                 + " case of the same kernel, scaled to this launch's algorithmic bytes")
+                                if qt in PERSIST_TRAFFIC_RATIO else "no capture of this instantiation",
                 "bytes_per_launch": k_bytes, "avg_launch_us": round(k_ms * 1e3, 3),
                 "timing": f"CUDA events on the compute stream around each of {n_probe} kernel launches "
                           f"(uncaptured steps right after the timed region, {round(probe_ms_step, 4)} ms/step there)"}
