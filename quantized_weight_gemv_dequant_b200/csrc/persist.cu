@@ -643,13 +643,84 @@ struct Consumer {
         }
         return false;
       }
+      if constexpr (QT == QT_Q6_K) {
+        // A Q6_K row slice is a long dependent chain, so a warp keeps two in
+        // flight.  With one row per warp per slot (TR == row groups) the next
+        // slot is opened too and its row runs beside this one.
+        if (TR == nrg && i + 1 < nst) {
+          const int s2 = s + 1 == (int)S ? 0 : s + 1;
+          const uint32_t ph2 = s + 1 == (int)S ? ph ^ 1u : ph;
+          const uint32_t rslot2 = (uint32_t)(q + 1) % kPRed;
+          bool ok2 = pwait_a(sb + o_full + 8 * s2, ph2, cta_abort);
+          if (ok2 && busy)
+            ok2 = pwait_a(sb + o_rempty + 8 * rslot2, (uint32_t)((((q + 1) / kPRed) & 1) ^ 1), cta_abort);
+          if (!ok2) {
+            if (lane == 0) {
+              atomicExch(sm.misc, 1);
+              atomicExch(st.sync + st.abort_index, 1u);
+            }
+            return false;
+          }
+          if (busy) {
+            const int rsa = r0 + i * TR;
+            const int nra = min(TR, r1 - rsa), nrb = min(TR, r1 - rsa - TR);
+            const int ra = (gr + nrg - i % nrg) % nrg, rb = (gr + nrg - (i + 1) % nrg) % nrg;
+            const bool ha = ra < nra, hb = rb < nrb;
+            const uint8_t* sta = p_smem + ring_c + (uint32_t)s * Z + (uint32_t)ra * (uint32_t)rbytes;
+            const uint8_t* stb = p_smem + ring_c + (uint32_t)s2 * Z + (uint32_t)rb * (uint32_t)rbytes;
+            float va = 0.f, vb = 0.f;
+            if (active && ha && hb) {
+              va = xr.dot(sta, lane);
+              vb = xr.dot(stb, lane);
+            } else if (active) {
+              if (ha) va = xr.dot(sta, lane);
+              if (hb) vb = xr.dot(stb, lane);
+            }
+            va = warp_sum(va);
+            vb = warp_sum(vb);
+            if (lane == 0) {
+              if (ha) (reinterpret_cast<float*>(p_smem + o_red) + rslot * RF)[ra * nsl + c] = va;
+              if (hb) (reinterpret_cast<float*>(p_smem + o_red) + rslot2 * RF)[rb * nsl + c] = vb;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_a(sb + o_empty + 8 * s);
+            mbar_arrive_a(sb + o_rfull + 8 * rslot);
+            mbar_arrive_a(sb + o_empty + 8 * s2);
+            mbar_arrive_a(sb + o_rfull + 8 * rslot2);
+          }
+          s = s2;
+          ph = ph2;
+          if (++s == (int)S) { s = 0; ph ^= 1u; }
+          ++i;  // the loop header steps past the second slot
+          ++q;
+          continue;
+        }
+      }
       if (busy) {
         const int rs = r0 + i * TR;
         const int nr = min(TR, r1 - rs);
         const uint8_t* stg = p_smem + ring_c + (uint32_t)s * Z;
         float* rd = reinterpret_cast<float*>(p_smem + o_red) + rslot * RF;
         // the row group that takes the extra rows rotates from stage to stage
-        for (int rr = (gr + nrg - i % nrg) % nrg; rr < nr; rr += nrg) {
+        int rr = (gr + nrg - i % nrg) % nrg;
+        if constexpr (QT == QT_Q6_K) {
+          for (; rr + nrg < nr; rr += 2 * nrg) {  // two rows of this slot side by side
+            float va = 0.f, vb = 0.f;
+            if (active) {
+              va = xr.dot(stg + (uint32_t)rr * (uint32_t)rbytes, lane);
+              vb = xr.dot(stg + (uint32_t)(rr + nrg) * (uint32_t)rbytes, lane);
+            }
+            va = warp_sum(va);
+            vb = warp_sum(vb);
+            if (lane == 0) {
+              rd[rr * nsl + c] = va;
+              rd[(rr + nrg) * nsl + c] = vb;
+            }
+          }
+        }
+        for (; rr < nr; rr += nrg) {
           float v = active ? xr.dot(stg + (uint32_t)rr * (uint32_t)rbytes, lane) : 0.f;
           v = warp_sum(v);
           if (lane == 0) rd[rr * nsl + c] = v;
