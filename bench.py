@@ -36,11 +36,11 @@ METRIC = "batch-1 decode tok/s; quantized GEMV achieved HBM GB/s vs B200 peak"
 # DRAM bytes read + written per algorithmic byte by the persistent decode
 # kernel, from one ncu capture (--set full) per instantiation of a cut-down
 # case that fits the capture size rule: Q8_0, 4 layers of the 8B shapes,
-# 1,485,753,088 + 4,944,128 bytes against 1,485,578,240 algorithmic bytes;
-# Q6_K, 2 layers of the 70B shapes, 2,282,915,584 + 3,851,264 bytes against
+# 1,485,809,408 + 4,275,456 bytes against 1,485,578,240 algorithmic bytes;
+# Q6_K, 2 layers of the 70B shapes, 2,282,932,224 + 4,280,064 bytes against
 # 2,282,651,648.  The kernel streams every weight byte once, so a full
 # launch's traffic is this ratio times its algorithmic bytes.
-PERSIST_TRAFFIC_RATIO = {8: 1490697216 / 1485578240, 14: 2286766848 / 2282651648}
+PERSIST_TRAFFIC_RATIO = {8: 1490084864 / 1485578240, 14: 2287212288 / 2282651648}
 FALLBACK_HBM_GBS = 6650.0
 
 
