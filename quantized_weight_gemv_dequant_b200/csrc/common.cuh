@@ -77,51 +77,6 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Packed fp32x2 arithmetic on 64-bit register pairs (sm_100).
-typedef unsigned long long f32x2;
-
-__device__ __forceinline__ f32x2 pack2(float a, float b) {
-  f32x2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void unpack2(f32x2 v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
-  f32x2 r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
-  f32x2 r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
-  f32x2 r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-// The pair (2^23 + byte ba of wa, 2^23 + byte bb of wb) built by two byte
-// permutes straight into the halves of one 64-bit register.
-template <int BA, int BB>
-__device__ __forceinline__ f32x2 magic_pair(uint32_t wa, uint32_t wb) {
-  f32x2 r;
-  asm("{\n\t.reg .b32 lo, hi;\n\t"
-      "prmt.b32 lo, %1, 0x4B000000, %3;\n\t"
-      "prmt.b32 hi, %2, 0x4B000000, %4;\n\t"
-      "mov.b64 %0, {lo, hi};\n\t}"
-      : "=l"(r)
-      : "r"(wa), "r"(wb), "n"(0x7440 | BA), "n"(0x7440 | BB));
-  return r;
-}
-__device__ __forceinline__ float hsum2(f32x2 v) {
-  float a, b;
-  unpack2(v, a, b);
-  return a + b;
-}
-
 // Waits for the phase with the given parity to complete, for at most
 // kWaitLimitNs.  Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {

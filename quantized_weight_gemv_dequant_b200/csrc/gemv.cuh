@@ -21,10 +21,10 @@
 //    sums the slice partials of each finished stage in a fixed order, runs the
 //    epilogue (store, + residual, RoPE + KV append, SwiGLU pairs, residual +
 //    cosine statistics, argmax) and refills the stage.
-//  * Decode is exact: a byte u becomes the float 2^23 + u with one byte
-//    permute (PRMT) and the offset is removed by one exact subtract; products
-//    and sums use packed fp32x2 FMA (FFMA2).  Block scales multiply the block's
-//    inner sum.
+//  * Dot products are exact integer sums: x is held as 22-bit fixed point in
+//    byte limbs and each block's (Q6_K: each 16-column run's) sum of code x
+//    limb products is formed with dp4a in int32; block scales and the
+//    fixed-point scale are applied once per block (Q6_K: once per row slice).
 #pragma once
 
 #include "common.cuh"
@@ -124,82 +124,6 @@ struct ProRms {
     return make_float4(b.x * (a.x * r), b.y * (a.y * r), b.z * (a.z * r), b.w * (a.w * r));
   }
 };
-
-// ------------------------------------------------------------- decoders
-
-// (2^23 + byte ba of wa, 2^23 + byte bb of wb) as one packed pair.
-__device__ __forceinline__ f32x2 bytes_pair(uint32_t wa, int ba, uint32_t wb, int bb) {
-  f32x2 r;
-  asm("{\n\t.reg .b32 lo, hi;\n\t"
-      "prmt.b32 lo, %1, 0x4B000000, %2;\n\t"
-      "prmt.b32 hi, %3, 0x4B000000, %4;\n\t"
-      "mov.b64 %0, {lo, hi};\n\t}"
-      : "=l"(r)
-      : "r"(wa), "r"(0x7440u | (uint32_t)ba), "r"(wb), "r"(0x7440u | (uint32_t)bb));
-  return r;
-}
-
-// Q8_0: lane l owns blocks 2l, 2l+1 of the slice (68 bytes = 17 words at the
-// 4-byte aligned offset 68 l).  Block 0: scale = low half of word 0, q_i =
-// byte 2+i.  Block 1: scale = high half of word 8, q_i = byte 36+i.
-// x2: the lane's 64 columns of x as 32 packed pairs.
-__device__ __forceinline__ float row_q8_0(const uint8_t* seg, int lane, const f32x2* x2) {
-  const uint32_t* wp = reinterpret_cast<const uint32_t*>(seg + lane * 68);
-  uint32_t w[17], xw[17];
-#pragma unroll
-  for (int i = 0; i < 17; ++i) {
-    w[i] = wp[i];
-    xw[i] = w[i] ^ 0x80808080u;
-  }
-  const f32x2 off = pack2(-8388736.0f, -8388736.0f);  // 2^23 + 128
-  float r = 0.f;
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    const float d = half_bits_to_float(b == 0 ? w[0] : (w[8] >> 16));
-    const int o = (b == 0) ? 2 : 36;
-    f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int i0 = o + 2 * k, i1 = o + 2 * k + 1;
-      const f32x2 v = add2(bytes_pair(xw[i0 >> 2], i0 & 3, xw[i1 >> 2], i1 & 3), off);
-      acc[k & 3] = fma2(v, x2[16 * b + k], acc[k & 3]);
-    }
-    r = fmaf(d, (hsum2(acc[0]) + hsum2(acc[1])) + (hsum2(acc[2]) + hsum2(acc[3])), r);
-  }
-  return r;
-}
-
-// Q4_0: lane l owns blocks 2l, 2l+1 (36 bytes = 9 words at offset 36 l).
-// Block b: scale at byte 18b; nibble byte j at byte 18b + 2 + j (low nibble
-// = element j, high nibble = element j + 16).  Low nibbles decode as
-// 2^23 + n, high nibbles as 2^23 + 16 n (no shift); the high sum is scaled by
-// 1/16, which is exact.
-__device__ __forceinline__ float row_q4_0(const uint8_t* seg, int lane, const f32x2* x2) {
-  const uint32_t* wp = reinterpret_cast<const uint32_t*>(seg + lane * 36);
-  uint32_t w[9];
-#pragma unroll
-  for (int i = 0; i < 9; ++i) w[i] = wp[i];
-  const f32x2 off_lo = pack2(-8388616.0f, -8388616.0f);  // 2^23 + 8
-  const f32x2 off_hi = pack2(-8388736.0f, -8388736.0f);  // 2^23 + 128
-  float r = 0.f;
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    const float d = half_bits_to_float(b == 0 ? w[0] : (w[4] >> 16));
-    const int o = (b == 0) ? 2 : 20;
-    f32x2 lo_acc[2] = {0ull, 0ull}, hi_acc[2] = {0ull, 0ull};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int j0 = o + 2 * k, j1 = o + 2 * k + 1;
-      const uint32_t wa = w[j0 >> 2], wb = w[j1 >> 2];
-      const f32x2 lo = add2(bytes_pair(wa & 0x0F0F0F0Fu, j0 & 3, wb & 0x0F0F0F0Fu, j1 & 3), off_lo);
-      const f32x2 hi = add2(bytes_pair(wa & 0xF0F0F0F0u, j0 & 3, wb & 0xF0F0F0F0u, j1 & 3), off_hi);
-      lo_acc[k & 1] = fma2(lo, x2[16 * b + k], lo_acc[k & 1]);
-      hi_acc[k & 1] = fma2(hi, x2[16 * b + 8 + k], hi_acc[k & 1]);
-    }
-    r = fmaf(d, fmaf(0.0625f, hsum2(hi_acc[0]) + hsum2(hi_acc[1]), hsum2(lo_acc[0]) + hsum2(lo_acc[1])), r);
-  }
-  return r;
-}
 
 // ---------------------------------------------------------------------------
 // Q8_0 / Q4_0: exact integer block dot products.
