@@ -91,6 +91,16 @@ def test_gemv_argument_errors():
     assert "overlaps" in ntx.ntx_last_error()
 
 
+def test_tuning_switch_argument_errors():
+    L = ntx.lib()
+    assert L.ntx_set_gemv_pdl(2) == ntx.NTX_ERR_INVALID_ARG
+    assert L.ntx_set_gemv_pdl(-1) == ntx.NTX_ERR_INVALID_ARG
+    assert L.ntx_set_gemv_pdl(0) == ntx.NTX_OK
+    assert L.ntx_set_gemv_ctas_per_sm(0) == ntx.NTX_ERR_INVALID_ARG
+    assert L.ntx_set_gemv_ctas_per_sm(5) == ntx.NTX_ERR_INVALID_ARG
+    assert L.ntx_set_gemv_ctas_per_sm(1) == ntx.NTX_OK
+
+
 def test_small_op_argument_errors():
     assert _rc(ntx.ntx_dequant, ntx.NTX_Q4_0, FAKE, FAKE + 0x1000, 33) == ntx.NTX_ERR_SHAPE
     assert _rc(ntx.ntx_dequant, 3, FAKE, FAKE + 0x1000, 32) == ntx.NTX_ERR_QTYPE
