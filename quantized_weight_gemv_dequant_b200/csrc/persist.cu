@@ -6,10 +6,14 @@
 // memory bound), so the step can only approach the HBM roofline if the weight
 // stream never pauses.  A chain of per-op kernels pauses at every boundary:
 // each kernel's CTAs must drain before the next kernel's CTAs (one per SM, up
-// to 227 KB of shared memory each) can start copying.  Here the producer warp
-// of each CTA walks one continuous list of weight stages across all phases of
-// the step; the weights never depend on activations, so it keeps the copy ring
-// full while the consumer warps wait at a phase boundary or compute attention.
+// to 227 KB of shared memory each) can start copying.  Here the copy warp of
+// each CTA walks one continuous list of weight stages across all phases of the
+// step; the weights never depend on activations, so it keeps the copy ring full
+// while the other warps wait at a phase boundary or compute attention.
+//
+// Warps of a CTA (16): 14 consumer warps (x staging, dot products, attention),
+// one epilogue warp (row sums, phase epilogues, the phase's grid arrival) and
+// one copy warp (bulk copies of the weight rows into the ring).
 //
 // Phases (index p; one grid-wide counter each):
 //   0            EMBED  h = fp16 row of the token, sum(h^2) partials
@@ -23,18 +27,20 @@
 //                       finish picks the token)
 // where k runs over the executed layers (a skip set removes layers from the
 // list).  A phase's inputs are complete when every CTA has arrived on the
-// previous phase's counter: GEMV phases arrive from the producer warp after
-// its epilogue stores, EMBED and ATTN from the consumer warps.  Every wait is
-// bounded (%globaltimer) and any CTA that gives up raises a grid-wide abort
-// word, so the other CTAs stop waiting too; the producer lets its copies in
-// flight land before the CTA exits.
+// previous phase's counter: GEMV phases arrive from the epilogue warp after
+// its stores, EMBED and ATTN from the consumer warps.  Every wait is bounded
+// (%globaltimer) and any CTA that gives up raises a grid-wide abort word, so
+// the other CTAs stop waiting too; the copy warp lets its copies in flight
+// land before the CTA exits.
 //
-// GEMV work inside a phase is the same as in gemv_tma_kernel: rows are split
-// evenly over the CTAs; consumer warp (c, g) owns K slice c (2048 columns,
-// x in registers) and row group g; partials go through shared memory to the
-// producer warp, which sums them in a fixed order and runs the epilogue.  All
-// phases share one ring of equal-size slots; each phase fits as many whole
-// rows in a slot as it can (an even count where the epilogue pairs rows).
+// GEMV work inside a phase follows gemv_tma_kernel: rows are split evenly over
+// the CTAs; consumer warp (c, g) owns K slice c (2048 columns, x in registers)
+// and row group g; row-slice partials go through a ring of partial slots in
+// shared memory (its own mbarriers) to the epilogue warp, which sums them in a
+// fixed order and runs the epilogue.  All phases share one ring of equal-size
+// weight slots; each phase fits as many whole rows in a slot as it can (an
+// even count where the epilogue pairs rows), and persist_plan picks the slot
+// size.
 // Data written by an earlier phase of this launch is read through L2
 // (ld.global.cg), never through the non-coherent or L1 paths.
 #include <cuda_runtime.h>
