@@ -295,6 +295,18 @@ NTX_API int ntx_engine_set_phase_probe(ntx_engine* e, unsigned long long* dev_ts
  * or captured by this engine), or a negative error. */
 NTX_API int ntx_engine_launches_per_step(ntx_engine* e);
 
+/* The persistent decode kernel's plan for a model whose layers all use block
+ * type qtype, as ntx_engine_create makes it (a host computation: no GPU
+ * needed; the grid is the current device's SM count, 148 without a device).
+ * Outputs (each nullable): *slot_bytes, *n_slots = the weight ring's slot size
+ * and slot count; *smem_bytes = dynamic shared memory per CTA;
+ * rows_per_slot[5] = whole weight rows per slot for the Q/K/V, O, gate/up,
+ * down and head phases.  NTX_ERR_INVALID_ARG for a NULL or non-positive
+ * config, NTX_ERR_QTYPE for other types, NTX_ERR_SHAPE when the persistent
+ * kernel does not take the model (the engine then runs the per-op chain). */
+NTX_API int ntx_persistent_plan(const ntx_model_config* cfg, int qtype, int* slot_bytes, int* n_slots,
+                                size_t* smem_bytes, int* rows_per_slot);
+
 /* Copies the recorded skip set (1 = skipped) into mask_host[L]; returns the
  * number of skipped layers, or a negative error. */
 NTX_API int ntx_engine_skip_mask(ntx_engine* e, uint8_t* mask_host);

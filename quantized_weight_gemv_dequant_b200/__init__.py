@@ -38,6 +38,7 @@ EXPORTS = (
     "ntx_swiglu", "ntx_layer_layout", "ntx_layer_workspace_bytes", "ntx_decode_layer", "ntx_engine_workspace_bytes",
     "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
     "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
+    "ntx_persistent_plan",
 )
 
 
@@ -100,6 +101,7 @@ def lib():
             "ntx_engine_launches_per_step": ([vp], i32),
             "ntx_attn_decode_static": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp], i32),
             "ntx_engine_set_phase_probe": ([vp, vp, sz], i32),
+            "ntx_persistent_plan": ([P(ntx_model_config), i32, P(i32), P(i32), P(sz), P(i32)], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -275,6 +277,18 @@ def ntx_engine_set_phase_probe(engine, dev_ts, n_words: int) -> int:
     if rc < 0:
         _check(rc)
     return rc
+
+
+def ntx_persistent_plan(cfg: ntx_model_config, qtype: int) -> dict:
+    """The persistent decode kernel's plan: slot_bytes, n_slots, smem_bytes and
+    rows per slot for the qkv, o, gu, down and head phases."""
+    zb, ns = ctypes.c_int(), ctypes.c_int()
+    smem = ctypes.c_size_t()
+    rows = (ctypes.c_int * 5)()
+    _check(lib().ntx_persistent_plan(ctypes.byref(cfg), qtype, ctypes.byref(zb), ctypes.byref(ns), ctypes.byref(smem),
+                                     rows))
+    return {"slot_bytes": zb.value, "n_slots": ns.value, "smem_bytes": smem.value,
+            "rows": dict(zip(["qkv", "o", "gu", "down", "head"], list(rows)))}
 
 
 def ntx_engine_launches_per_step(engine) -> int:

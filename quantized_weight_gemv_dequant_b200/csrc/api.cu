@@ -824,6 +824,28 @@ extern "C" int ntx_engine_set_phase_probe(ntx_engine* e, unsigned long long* dev
   return e->persist ? e->pgrid : 0;
 }
 
+extern "C" int ntx_persistent_plan(const ntx_model_config* cfg, int qtype, int* slot_bytes, int* n_slots,
+                                   size_t* smem_bytes, int* rows_per_slot) {
+  if (!cfg || cfg->hidden <= 0 || cfg->n_heads <= 0 || cfg->n_kv_heads <= 0 || cfg->head_dim <= 0 || cfg->ffn <= 0 ||
+      cfg->vocab <= 0 || cfg->n_layers <= 0 || cfg->max_ctx <= 0)
+    return fail(NTX_ERR_INVALID_ARG, "NULL or non-positive model config");
+  if (!qtype_ok(qtype)) return fail(NTX_ERR_QTYPE, "unsupported weight type %d", qtype);
+  ntx::PStep st;
+  memset(&st, 0, sizeof st);
+  size_t smem = 0;
+  if (ntx::persist_plan(qtype, cfg->hidden, cfg->n_heads, cfg->n_kv_heads, cfg->head_dim, cfg->ffn, cfg->vocab,
+                        cfg->max_ctx, ntx::sm_count(), cfg->n_layers, &st, &smem) != 0)
+    return fail(NTX_ERR_SHAPE, "the persistent kernel does not take this model");
+  if (slot_bytes) *slot_bytes = st.slot_bytes;
+  if (n_slots) *n_slots = st.n_slots;
+  if (smem_bytes) *smem_bytes = smem;
+  if (rows_per_slot) {
+    const int kinds[5] = {ntx::PK_QKV, ntx::PK_O, ntx::PK_GU, ntx::PK_DOWN, ntx::PK_HEAD};
+    for (int i = 0; i < 5; ++i) rows_per_slot[i] = st.g[kinds[i]].TR;
+  }
+  return NTX_OK;
+}
+
 extern "C" int ntx_engine_launches_per_step(ntx_engine* e) {
   if (!e) return fail(NTX_ERR_INVALID_ARG, "engine is NULL");
   return e->launches;
