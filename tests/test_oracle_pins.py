@@ -470,3 +470,91 @@ def test_layer_is_causal_in_cache():
     o2, c2 = oracle.layer(cfg, Q8_0, m, m["attn_norm"], m["ffn_norm"], kc2, vc2, h, 4)
     assert np.array_equal(o1, o2) and c1 == c2
     assert abs(c1 - oracle.cosine(h, o1)) < 1e-15
+
+
+def test_layer_ffn_only_path_with_zero_attention_output():
+    """With Wo = 0 attention adds nothing: h_out = h + Wd (silu(Wg n) * Wu n),
+    n = RMSNorm(h) w_ffn.  Rebuild that from the oracle's separately pinned parts."""
+    cfg = _tiny_cfg(D=32, F=64)
+    m = _layer_mats(cfg, Q8_0, 4, zero=("wo",))
+    rs = np.random.RandomState(3)
+    kc, vc = _f16(rs.randn(2, 8, 32)), _f16(rs.randn(2, 8, 32))
+    h = rs.randn(64)
+    out, c = oracle.layer(cfg, Q8_0, m, m["attn_norm"], m["ffn_norm"], kc, vc, h, 2)
+    n2 = oracle.rmsnorm(h, m["ffn_norm"].astype(np.float64), 1e-5)
+    g, _ = oracle.gemv(Q8_0, m["wg"], 64, 64, n2)
+    u, _ = oracle.gemv(Q8_0, m["wu"], 64, 64, n2)
+    d, _ = oracle.gemv(Q8_0, m["wd"], 64, 64, oracle.swiglu(g, u))
+    assert np.allclose(out, h + d, rtol=0, atol=1e-14)
+    assert abs(c - oracle.cosine(h, out)) < 1e-15
+
+
+# ----------------------------------------------------------------- embed / head / model step
+def test_embed_is_the_fp16_row():
+    t = _f16(np.random.RandomState(7).randn(5, 48))
+    for tok in (0, 3, 4):
+        assert np.array_equal(oracle.embed(t, 48, tok), t[tok].view(np.float16).astype(np.float64))
+
+
+def test_head_applies_the_final_norm():
+    """Logits are the head GEMV of RMSNorm(h) w_final: equal to the pinned GEMV of
+    the pinned RMSNorm, and blind to the scale of h up to eps."""
+    cfg = oracle.make_config(64, 4, 2, 16, 96, 40, 1, 1e-5, 500000.0, 8)
+    W = sg.quant_rows(Q8_0, 5, "head", 40, 64)
+    fn = sg.fill_f32(5, "fn", 64, mean=1.0, sigma=0.02)
+    h = np.random.RandomState(4).randn(64)
+    logits = oracle.head(cfg, Q8_0, W, fn, h)
+    ref, _ = oracle.gemv(Q8_0, W, 40, 64, oracle.rmsnorm(h, fn.astype(np.float64), 1e-5))
+    assert np.array_equal(logits, ref)
+    # eps = 1e-5 against mean(h^2) ~ 1 shifts the scale by at most ~5e-6
+    assert np.allclose(oracle.head(cfg, Q8_0, W, fn, 1000.0 * h), logits, rtol=1e-5, atol=0)
+    assert not np.allclose(1000.0 * logits, logits)
+
+
+def _tiny_model(L, seed, zero_layers):
+    cfg = oracle.make_config(64, 4, 2, 16, 96, 40, L, 1e-5, 500000.0, 8)
+    names = ("wq", "wk", "wv", "wo", "wg", "wu", "wd")
+    layers = [_layer_mats(cfg, Q8_0, seed + l, zero=names if zero_layers else ()) for l in range(L)]
+    W = sg.quant_rows(Q8_0, seed, "head", 40, 64)
+    fn = sg.fill_f32(seed, "fn", 64, mean=1.0, sigma=0.02)
+    emb = sg.fill_f16(seed, "emb", 40 * 64, sigma=0.5).reshape(40, 64)
+    return cfg, layers, W, fn, emb
+
+
+def _caches(L, seed):
+    rs = np.random.RandomState(seed)
+    return [_f16(rs.randn(2, 8, 16)) for _ in range(L)], [_f16(rs.randn(2, 8, 16)) for _ in range(L)]
+
+
+def test_model_step_with_every_layer_skipped_is_head_of_embedding():
+    """Skipped layers are neither computed nor appended to their cache."""
+    cfg, layers, W, fn, emb = _tiny_model(3, 11, zero_layers=False)
+    kcs, vcs = _caches(3, 1)
+    k0, v0 = [k.copy() for k in kcs], [v.copy() for v in vcs]
+    logits, cos = oracle.model_step(cfg, Q8_0, layers, Q8_0, W, fn, emb, kcs, vcs, 9, 4, skip=[1, 1, 1])
+    assert np.array_equal(logits, oracle.head(cfg, Q8_0, W, fn, oracle.embed(emb, 64, 9)))
+    assert np.all(np.isnan(cos))
+    assert all(np.array_equal(a, b) for a, b in zip(kcs + vcs, k0 + v0))
+
+
+def test_model_step_skip_changes_only_the_skipped_layer():
+    cfg, layers, W, fn, emb = _tiny_model(3, 12, zero_layers=False)
+    kcs, vcs = _caches(3, 2)
+    k0, v0 = [k.copy() for k in kcs], [v.copy() for v in vcs]
+    _, cos = oracle.model_step(cfg, Q8_0, layers, Q8_0, W, fn, emb, kcs, vcs, 3, 5, skip=[0, 1, 0])
+    assert np.isnan(cos[1]) and not np.isnan(cos[0]) and not np.isnan(cos[2])
+    assert np.array_equal(kcs[1], k0[1]) and np.array_equal(vcs[1], v0[1])
+    assert not np.array_equal(kcs[0][:, 5], k0[0][:, 5]) and not np.array_equal(kcs[2][:, 5], k0[2][:, 5])
+    rows = [p for p in range(8) if p != 5]
+    assert np.array_equal(kcs[0][:, rows], k0[0][:, rows]) and np.array_equal(vcs[2][:, rows], v0[2][:, rows])
+
+
+def test_model_step_of_identity_layers():
+    """All-zero projection weights make every layer the identity (cosine 1), so
+    the logits are the head of the embedding row and the token picks the row."""
+    cfg, layers, W, fn, emb = _tiny_model(2, 13, zero_layers=True)
+    for tok in (0, 17, 39):
+        kcs, vcs = _caches(2, 3)
+        logits, cos = oracle.model_step(cfg, Q8_0, layers, Q8_0, W, fn, emb, kcs, vcs, tok, 6)
+        assert np.array_equal(logits, oracle.head(cfg, Q8_0, W, fn, oracle.embed(emb, 64, tok)))
+        assert np.allclose(cos, 1.0, rtol=0, atol=1e-15)
