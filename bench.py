@@ -401,6 +401,18 @@ def run_ntx(args, dist: Dist):
         cpu = cpu_baseline_from_model(m, wk, d, pos_of(0))
 
     bpt = wl.bytes_per_token(d, qt, hqt, p_first + span // 2)
+    # ------------------------------------------------- host link (tier-B layers)
+    host_link = None
+    if any(tier_map):
+        streamed = sum(tier_map) * m.blob_bytes  # every host layer crosses the link once per step (no skip set)
+        link_peak = h2d_peak_gbs(torch)
+        link_gbs = streamed / (ms_step * 1e-3) / 1e9
+        host_link = {"streamed_bytes_per_step": streamed, "h2d_gbs": round(link_gbs, 1),
+                     "peak_gbs": round(link_peak, 1), "frac": round(link_gbs / link_peak, 4),
+                     "timing": "streamed bytes over the whole step time: a lower bound on the copy stream's rate "
+                               "(the step is bound by its copies; the compute stream waits on them)",
+                     "peak_how": "pinned host -> device cudaMemcpyAsync of 1 GiB on its own stream, best of 10, "
+                                 "CUDA events"}
     ntx.ntx_engine_destroy(eng)
     torch.cuda.synchronize()
     desc = wk["desc"] if args.layers is None else f"{wk['desc']} -- layer count overridden to {L} (profiling only)"
@@ -429,9 +441,29 @@ def run_ntx(args, dist: Dist):
         "gemv": gemv,
         "gemv_in_step": in_step,
         "chain": chain,
+        "host_link": host_link,
         "cpu_baseline": cpu,
     }
     return out
+
+
+def h2d_peak_gbs(torch, nbytes=1 << 30, reps=10):
+    """Host-link peak: one pinned-host -> device copy of nbytes on a stream of
+    its own, the best of reps, timed with CUDA events on that stream."""
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    best = float("inf")
+    with torch.cuda.stream(s):
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            dst.copy_(src, non_blocking=True)
+            e1.record(s)
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+    del src, dst
+    return nbytes / (best * 1e-3) / 1e9
 
 
 def time_gemv(ntx, sg, wl, torch, qt, M, K, reps=40, pdl=False):
