@@ -75,7 +75,11 @@ NTX_API int ntx_version(void); /* major*10000 + minor*100 + patch */
 
 /* Reads and clears the device status word of the current device (0 = no
  * kernel gave up a bounded wait since the last read).  Synchronises the
- * device.  Returns NTX_OK and stores the word in *code. */
+ * device.  Returns NTX_OK and stores the word in *code.  Codes: 1 a weight
+ * copy did not land in time, 2 copies still outstanding when a CTA that gave
+ * up had to exit (the context is then unusable: launch nothing more on it),
+ * 3 a token id outside [0, V) reached the embedding, 4 a grid-wide barrier of
+ * the persistent decode kernel ran out. */
 NTX_API int ntx_device_status(int* code);
 
 /* Number of SMs the kernels size their grids for on the current device. */
@@ -158,11 +162,14 @@ NTX_API int ntx_attn_decode(const float* q, const uint16_t* k_cache, const uint1
  * allocator on that path, latency-critical threads that must not take an
  * allocator's lock.  Limit: n_q_heads x (attention splits) x 130 floats <=
  * 524288, NTX_ERR_NOMEM beyond it (on a 148-SM B200 with 8 KV heads: up to
- * 32256 positions at 32 query heads, 16128 at 64).  The first call on
- * a device looks up the array's address (cudaGetSymbolAddress); make that
- * first call before any stream capture.  Every GPU that loads libntx holds the
- * array until exit, all calls share it and it keeps the last call's contents:
- * calls that overlap on the GPU (e.g. on two streams) race. */
+ * 32256 positions at 32 query heads, 16128 at 64); the size check comes
+ * before any CUDA call.  The first call on a device looks up the array's
+ * address (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture.  Later calls take no lock.  The cached address does not
+ * survive cudaDeviceReset: do not use this call on a device after resetting
+ * it.  Every GPU that loads libntx holds the array until exit, all calls share
+ * it and it keeps the last call's contents: calls that overlap on the GPU
+ * (e.g. on two streams) race. */
 NTX_API int ntx_attn_decode_static(const float* q, const uint16_t* k_cache, const uint16_t* v_cache, float* out,
                                    int n_q_heads, int n_kv_heads, int head_dim, int n_ctx, int max_ctx, void* stream);
 
@@ -239,11 +246,13 @@ NTX_API int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_weight
  * The engine owns only its events, a pinned 16-byte parameter block and the
  * captured CUDA graphs; the caller keeps every buffer alive until
  * ntx_engine_destroy.
- * Execution: when every layer is resident (tier 0) and every layer and the
- * head share one block type, a step runs as ONE persistent kernel (one CTA
- * per SM, grid-wide phase barriers, the weight stream continuing across
- * phases); otherwise, or with NTX_NO_PERSIST, as a chain of per-op kernels
- * (about five per layer) joined by programmatic dependent launch. */
+ * Execution: when every layer and the head share one block type, a step
+ * whose executed layers are all resident (tier 0) -- every step of an engine
+ * without host layers, and the NTX_USE_SKIP steps of one whose recorded skip
+ * set skips every host layer -- runs as ONE persistent kernel (one CTA per
+ * SM, grid-wide phase barriers, the weight stream continuing across phases);
+ * other steps, or any step with NTX_NO_PERSIST, run as a chain of per-op
+ * kernels (about five per layer) joined by programmatic dependent launch. */
 typedef struct ntx_engine ntx_engine;
 
 #define NTX_CALIBRATE_SKIP 1 /* run every layer, record cosines, fix the skip set {l : cos_l >= tau} */

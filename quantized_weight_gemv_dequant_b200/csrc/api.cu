@@ -362,8 +362,11 @@ struct ntx_engine {
   // profiling probe (kernel-by-kernel steps only) and launch count
   std::vector<cudaEvent_t> probe_b, probe_e;
   int launches;
-  // persistent decode kernel (all layers resident, one block type)
-  bool persist;
+  // persistent decode kernel (one block type; runs a step whose executed
+  // layers are all resident)
+  bool persist;       // the plan and launch parameters are valid
+  bool persist_full;  // every layer is resident: steps without the skip set
+  bool persist_skip;  // every layer of the recorded skip set's run list is resident
   ntx::PStep pst;
   size_t psmem;
   int pgrid;
@@ -490,7 +493,11 @@ cudaError_t persist_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t
 // Enqueue the per-token launch sequence (everything after the parameter copy).
 cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t* next_token, float* cos_out,
                            bool calibrate, bool probe, bool no_persist) {
-  if (e->persist && !no_persist) return persist_enqueue(e, use_skip, logits, next_token, cos_out, calibrate, probe);
+  if (e->persist && !no_persist) {
+    const bool sk = use_skip && e->skip_valid;
+    if (sk ? e->persist_skip : e->persist_full)
+      return persist_enqueue(e, use_skip, logits, next_token, cos_out, calibrate, probe);
+  }
   const ntx_model_config& c = e->cfg;
   cudaStream_t s = e->cs;
   const bool pdl = true;
@@ -654,9 +661,11 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   }
   if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->fork_ev, cudaEventDisableTiming);
   if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->join_ev, cudaEventDisableTiming);
-  // persistent kernel: every layer resident and of the head's block type, shapes and alignment it handles
-  e->persist = false;
-  bool one_type = !any_host && (head_qtype == NTX_Q8_0 || head_qtype == NTX_Q4_0 || head_qtype == NTX_Q6_K);
+  // persistent kernel: every layer of the head's block type, shapes and alignment it handles; it runs the
+  // steps whose executed layers are all resident (all steps without a host tier; with one, the steps under a
+  // skip set that skips every host layer)
+  e->persist = e->persist_full = e->persist_skip = false;
+  bool one_type = head_qtype == NTX_Q8_0 || head_qtype == NTX_Q4_0 || head_qtype == NTX_Q6_K;
   for (int l = 0; l < cfg->n_layers && one_type; ++l) one_type = layers[l].qtype == head_qtype;
   if (err == cudaSuccess && one_type) {
     ntx::PStep st;
@@ -686,14 +695,17 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
         st.sync = e->psync;
         st.n_split = ntx::persist_splits(grid, cfg->n_kv_heads, cfg->max_ctx);
         st.status = ntx::device_status_ptr();
-        std::vector<int> all(cfg->n_layers);
-        for (int l = 0; l < cfg->n_layers; ++l) all[l] = l;
-        err = upload_players(e, all, e->pl_all);
+        if (!any_host) {
+          std::vector<int> all(cfg->n_layers);
+          for (int l = 0; l < cfg->n_layers; ++l) all[l] = l;
+          err = upload_players(e, all, e->pl_all);
+        }
         if (err == cudaSuccess) {
           e->pst = st;
           e->psmem = psm;
           e->pgrid = grid;
           e->persist = true;
+          e->persist_full = !any_host;
         }
       }
     }
@@ -772,11 +784,15 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
       e->skip[l] = cs[l] >= c.skip_threshold ? 1 : 0;
       if (!e->skip[l]) list.push_back(l);
     }
+    bool all_resident = true;
+    for (int l : list) all_resident = all_resident && e->tier[l] == 0;
+    e->persist_skip = false;
     if (!list.empty()) {
       err = cudaMemcpy(e->layer_list, list.data(), sizeof(int) * list.size(), cudaMemcpyHostToDevice);
-      if (err == cudaSuccess && e->persist) err = upload_players(e, list, e->pl_skip);
+      if (err == cudaSuccess && e->persist && all_resident) err = upload_players(e, list, e->pl_skip);
       if (err != cudaSuccess) return cuda_fail(err, "layer list");
     }
+    e->persist_skip = e->persist && all_resident;
     e->n_skip_run = (int)list.size();
     e->skip_valid = true;
     // graphs built with an older skip set are stale
@@ -821,7 +837,7 @@ extern "C" int ntx_engine_set_phase_probe(ntx_engine* e, unsigned long long* dev
   if (dev_ts && !aligned(dev_ts, 8)) return fail(NTX_ERR_ALIGN, "probe buffer must be 8-byte aligned");
   e->phase_ts = n_words ? dev_ts : nullptr;
   e->phase_ts_words = n_words;
-  return e->persist ? e->pgrid : 0;
+  return (e->persist_full || e->persist_skip) ? e->pgrid : 0;
 }
 
 extern "C" int ntx_persistent_plan(const ntx_model_config* cfg, int qtype, int* slot_bytes, int* n_slots,

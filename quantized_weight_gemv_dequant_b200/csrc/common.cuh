@@ -16,6 +16,11 @@ namespace ntx {
 enum : int {
   kStatusOk = 0,
   kStatusTmaTimeout = 1,
+  // A copy warp that gave up still lets its issued bulk copies land before
+  // the CTA exits (a second bounded wait).  If that wait runs out too, copies
+  // issued two seconds earlier have not arrived: the memory system has stopped
+  // delivering, the CTA exits with them outstanding, and the context must be
+  // treated as lost (no further launches on it).
   kStatusDrainTimeout = 2,
   kStatusBadToken = 3,
   kStatusGridTimeout = 4,  // a grid-wide barrier of the persistent decode kernel ran out

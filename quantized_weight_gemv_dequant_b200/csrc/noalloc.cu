@@ -14,12 +14,17 @@
 // In host code the array's name is not a device address; the first call on a
 // device (with that device current) looks the address up with
 // cudaGetSymbolAddress and caches it, so that first call should come before
-// any stream capture.  All calls on a device share the one array and it keeps
-// the contents of the last call: calls that overlap on the GPU (for example on
-// two streams) race on it.  Nothing in it needs to start at zero: the split
-// kernel writes every (head, split) partial the combine kernel reads.
+// any stream capture.  Later calls read the cached address with one atomic
+// load and take no lock.  The cache lives as long as the process: after
+// cudaDeviceReset on a device the module is loaded again, possibly at another
+// address, so this call must not be used on that device after a reset.  All
+// calls on a device share the one array and it keeps the contents of the last
+// call: calls that overlap on the GPU (for example on two streams) race on it.
+// Nothing in it needs to start at zero: the split kernel writes every (head,
+// split) partial the combine kernel reads.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "launch.h"
@@ -35,8 +40,8 @@ constexpr size_t kStaticScratchFloats = kStaticScratchBytes / sizeof(float);
 static __device__ __align__(256) float g_attn_static_scratch[kStaticScratchFloats];
 
 constexpr int kMaxDev = 64;
-float* g_scratch_ptr[kMaxDev];
-std::mutex g_scratch_mu;
+std::atomic<float*> g_scratch_ptr[kMaxDev];
+std::mutex g_scratch_mu;  // taken only by the first lookup on a device
 
 // Device address of the static scratch for the current device (looked up once
 // per device), or nullptr with *err set.
@@ -48,14 +53,18 @@ float* static_scratch(cudaError_t* err) {
     *err = cudaErrorInvalidDevice;
     return nullptr;
   }
+  float* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
   std::lock_guard<std::mutex> g(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    *err = cudaGetSymbolAddress(&p, g_attn_static_scratch);
+  p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+  if (!p) {
+    void* a = nullptr;
+    *err = cudaGetSymbolAddress(&a, g_attn_static_scratch);
     if (*err != cudaSuccess) return nullptr;
-    g_scratch_ptr[dev] = static_cast<float*>(p);
+    p = static_cast<float*>(a);
+    g_scratch_ptr[dev].store(p, std::memory_order_release);
   }
-  return g_scratch_ptr[dev];
+  return p;
 }
 
 }  // namespace

@@ -148,3 +148,24 @@ def test_layer_and_engine_argument_errors():
     # a host-tier layer without slots / copy stream
     assert _rc(ntx.ntx_engine_create, cfg, [lw], [1], *common.values(), 1, None) == ntx.NTX_ERR_INVALID_ARG
     assert _rc(ntx.ntx_decode_step, None, 0, 0) == ntx.NTX_ERR_INVALID_ARG
+
+
+def test_static_attention_refuses_oversize_before_any_cuda_call():
+    """The no-workspace attention checks its size against the 2 MiB static
+    array before touching the device.  Run only where no GPU is visible, so the
+    made-up addresses can never reach a kernel; the GPU suite repeats this with
+    real buffers."""
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("covered with real device buffers by the GPU suite")
+    except ImportError:
+        pass
+    # 64 query heads over 8 KV heads at 20000 positions: 79 splits x 64 x 130 floats > 524,288
+    args = [FAKE, FAKE + 0x10000000, FAKE + 0x20000000, FAKE + 0x30000000]
+    assert _rc(ntx.ntx_attn_decode_static, *args, 64, 8, 128, 20000, 20000) == ntx.NTX_ERR_NOMEM
+    assert "2 MiB" in ntx.ntx_last_error()
+    # shape and pointer checks come first
+    assert _rc(ntx.ntx_attn_decode_static, *args, 64, 8, 64, 100, 100) == ntx.NTX_ERR_SHAPE
+    assert _rc(ntx.ntx_attn_decode_static, None, *args[1:], 64, 8, 128, 100, 100) == ntx.NTX_ERR_INVALID_ARG
+    assert _rc(ntx.ntx_attn_decode_static, FAKE + 4, *args[1:], 64, 8, 128, 100, 100) == ntx.NTX_ERR_ALIGN

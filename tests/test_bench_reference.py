@@ -17,7 +17,7 @@ def _run(args, env_extra=None):
 
 
 def test_reference_arm_line():
-    r = _run(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    r = _run(["--impl", "reference", "--steps", "1", "--warmup", "3", "--layers", "1"])
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
