@@ -17,7 +17,8 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 SO = os.path.join(HERE, "libntx_oracle.so")
 
-Q4_0, Q8_0, Q6_K = 2, 8, 14
+F32, F16, Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 0, 1, 2, 8, 12, 13, 14
+MATS = ("wq", "wk", "wv", "wo", "wg", "wu", "wd")
 
 
 def build(force: bool = False) -> None:
@@ -35,8 +36,19 @@ class Config(ctypes.Structure):
 
 
 class LayerWeights(ctypes.Structure):
-    _fields_ = [("qtype", ctypes.c_int32)] + [(n, ctypes.c_void_p) for n in
-                                               ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "attn_norm", "ffn_norm")]
+    _fields_ = [("qt", ctypes.c_int32 * 7)] + [(n, ctypes.c_void_p) for n in
+                                                ("wq", "wk", "wv", "wo", "wg", "wu", "wd", "attn_norm", "ffn_norm")]
+
+
+def mat_types(qtype) -> list:
+    """Block type of each of wq..wd: one type for all, or a sequence of seven
+    (mixed models such as Q4_K_M), or a dict keyed by matrix name."""
+    if isinstance(qtype, dict):
+        return [int(qtype[k]) for k in MATS]
+    if isinstance(qtype, (list, tuple)):
+        assert len(qtype) == 7
+        return [int(t) for t in qtype]
+    return [int(qtype)] * 7
 
 
 _lib = None
@@ -160,13 +172,15 @@ def make_config(hidden, n_heads, n_kv_heads, head_dim, ffn, vocab, n_layers, eps
 
 def layer(cfg: Config, qtype: int, mats: dict, attn_norm, ffn_norm, k_cache, v_cache, h_in, pos,
           nthreads: int | None = None):
-    """One decode layer.  ``mats`` maps wq..wd to uint8 block arrays; the fp16
-    caches (uint16 numpy arrays) are updated in place.  Returns (h_out, cos)."""
-    keep = {k: np.ascontiguousarray(mats[k], dtype=np.uint8) for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd")}
+    """One decode layer.  ``mats`` maps wq..wd to uint8 block arrays (and may
+    carry "qtypes", the seven matrices' block types, which then replace
+    ``qtype``); the fp16 caches (uint16 numpy arrays) are updated in place.
+    Returns (h_out, cos)."""
+    keep = {k: np.ascontiguousarray(mats[k], dtype=np.uint8) for k in MATS}
     an = np.ascontiguousarray(attn_norm, dtype=np.float32)
     fn = np.ascontiguousarray(ffn_norm, dtype=np.float32)
-    L = LayerWeights(qtype, *[keep[k].ctypes.data for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd")],
-                     an.ctypes.data, fn.ctypes.data)
+    L = LayerWeights((ctypes.c_int32 * 7)(*mat_types(mats.get("qtypes", qtype))),
+                     *[keep[k].ctypes.data for k in MATS], an.ctypes.data, fn.ctypes.data)
     assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
     assert k_cache.dtype == np.uint16 and v_cache.dtype == np.uint16
     h = _d(h_in)

@@ -40,6 +40,19 @@
  *  - the layer is the pre-norm Llama block; the model is embed (fp16 row),
  *    layers, final RMSNorm, output head, greedy argmax (ties -> lowest id);
  *  - cosine c = <h_in, h_out> / (|h_in| |h_out|), layer skipped if c >= tau.
+ * The same format table lists Q4_K_M (4.5 bit/weight, blocks of 256, "mixed"),
+ * Q5_K (5.5 bit/weight, blocks of 256) and F16/F32 (16/32 bit/weight, blocks
+ * of 1).  Readings (GGUF's layouts, consistent with those sizes):
+ *  - Q4_K super-block, 144 B: fp16 d, fp16 dmin, 12 bytes of packed 6-bit
+ *    sub-block scales sc[8] and mins m[8], 128 bytes of 4-bit codes;
+ *    element 64c + l (c < 4, l < 32) is the low nibble of qs[32c + l] and
+ *    element 64c + 32 + l its high nibble; w = d sc[n/32] q - dmin m[n/32];
+ *  - Q5_K super-block, 176 B: the same d, dmin and scales, then qh[32] and
+ *    qs[128]; the fifth bit of element 64c + l is bit 2c of qh[l], of element
+ *    64c + 32 + l bit 2c + 1; q in 0..31, same formula;
+ *  - "M" (mixed) means some matrices of the model use another block type; the
+ *    oracle's layer takes one type per matrix;
+ *  - F16: IEEE binary16 per weight; F32: IEEE binary32 per weight.
  */
 #include <math.h>
 #include <pthread.h>
@@ -48,8 +61,12 @@
 #include <string.h>
 
 /* GGUF type ids */
+#define ORC_F32 0
+#define ORC_F16 1
 #define ORC_Q4_0 2
 #define ORC_Q8_0 8
+#define ORC_Q4_K 12
+#define ORC_Q5_K 13
 #define ORC_Q6_K 14
 
 /* ------------------------------------------------------------ binary16 */
@@ -87,10 +104,24 @@ uint16_t orc_to_half(double v) {
 
 /* ------------------------------------------------------------ dequant */
 int orc_block_elems(int qtype) {
-  switch (qtype) { case ORC_Q4_0: case ORC_Q8_0: return 32; case ORC_Q6_K: return 256; default: return 0; }
+  switch (qtype) {
+    case ORC_F32: case ORC_F16: return 1;
+    case ORC_Q4_0: case ORC_Q8_0: return 32;
+    case ORC_Q4_K: case ORC_Q5_K: case ORC_Q6_K: return 256;
+    default: return 0;
+  }
 }
 int orc_block_bytes(int qtype) {
-  switch (qtype) { case ORC_Q4_0: return 18; case ORC_Q8_0: return 34; case ORC_Q6_K: return 210; default: return 0; }
+  switch (qtype) {
+    case ORC_F32: return 4;
+    case ORC_F16: return 2;
+    case ORC_Q4_0: return 18;
+    case ORC_Q8_0: return 34;
+    case ORC_Q4_K: return 144;
+    case ORC_Q5_K: return 176;
+    case ORC_Q6_K: return 210;
+    default: return 0;
+  }
 }
 
 static uint16_t rd16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
@@ -131,10 +162,72 @@ static void dq_q6_k(const uint8_t* blk, double* w) {
   }
 }
 
+/* The 6-bit scale and min of sub-block j (0..7) of a Q4_K / Q5_K super-block
+ * from its 12 packed bytes p: sub-blocks 0-3 keep their scale in the low six
+ * bits of p[j] and their min in the low six bits of p[j + 4]; sub-blocks 4-7
+ * keep the low four bits of the scale in the low nibble of p[j + 4] and of the
+ * min in its high nibble, and the top two bits of each in the top two bits of
+ * p[j - 4] (scale) and p[j] (min). */
+static void k_scale_min(const uint8_t* p, int j, int* sc, int* m) {
+  if (j < 4) {
+    *sc = p[j] & 63;
+    *m = p[j + 4] & 63;
+  } else {
+    *sc = (p[j + 4] & 0x0F) | ((p[j - 4] >> 6) << 4);
+    *m = (p[j + 4] >> 4) | ((p[j] >> 6) << 4);
+  }
+}
+
+/* Q4_K super-block (144 B): d at 0, dmin at 2, scales at 4..15, qs at 16..143.
+ * Element n = 64c + 32h + l takes nibble h of qs[32c + l];
+ * w_n = d sc_j q_n - dmin m_j with j = n / 32. */
+static void dq_q4_k(const uint8_t* blk, double* w) {
+  double d = orc_half(rd16(blk)), dmin = orc_half(rd16(blk + 2));
+  const uint8_t* qs = blk + 16;
+  for (int n = 0; n < 256; ++n) {
+    int c = n / 64, h = (n % 64) / 32, l = n % 32;
+    int q = (qs[32 * c + l] >> (4 * h)) & 0x0F;
+    int sc, m;
+    k_scale_min(blk + 4, n / 32, &sc, &m);
+    w[n] = d * (double)sc * (double)q - dmin * (double)m;
+  }
+}
+
+/* Q5_K super-block (176 B): d at 0, dmin at 2, scales at 4..15, qh at
+ * 16..47, qs at 48..175.  Element n = 64c + 32h + l: low four bits from
+ * nibble h of qs[32c + l], fifth bit = bit (2c + h) of qh[l];
+ * w_n = d sc_j q_n - dmin m_j with j = n / 32. */
+static void dq_q5_k(const uint8_t* blk, double* w) {
+  double d = orc_half(rd16(blk)), dmin = orc_half(rd16(blk + 2));
+  const uint8_t* qh = blk + 16;
+  const uint8_t* qs = blk + 48;
+  for (int n = 0; n < 256; ++n) {
+    int c = n / 64, h = (n % 64) / 32, l = n % 32;
+    int q = ((qs[32 * c + l] >> (4 * h)) & 0x0F) | (((qh[l] >> (2 * c + h)) & 1) << 4);
+    int sc, m;
+    k_scale_min(blk + 4, n / 32, &sc, &m);
+    w[n] = d * (double)sc * (double)q - dmin * (double)m;
+  }
+}
+
+/* F16: one IEEE binary16 per weight; F32: one IEEE binary32 per weight. */
+static void dq_f16(const uint8_t* blk, double* w) { w[0] = orc_half(rd16(blk)); }
+static void dq_f32(const uint8_t* blk, double* w) {
+  float f;
+  memcpy(&f, blk, 4);
+  w[0] = (double)f;
+}
+
 static void dq_block(int qtype, const uint8_t* blk, double* w) {
-  if (qtype == ORC_Q8_0) dq_q8_0(blk, w);
-  else if (qtype == ORC_Q4_0) dq_q4_0(blk, w);
-  else dq_q6_k(blk, w);
+  switch (qtype) {
+    case ORC_Q8_0: dq_q8_0(blk, w); break;
+    case ORC_Q4_0: dq_q4_0(blk, w); break;
+    case ORC_Q4_K: dq_q4_k(blk, w); break;
+    case ORC_Q5_K: dq_q5_k(blk, w); break;
+    case ORC_F16: dq_f16(blk, w); break;
+    case ORC_F32: dq_f32(blk, w); break;
+    default: dq_q6_k(blk, w); break;
+  }
 }
 
 /* n values (n a multiple of the block size) from consecutive blocks. */
@@ -288,7 +381,7 @@ typedef struct {
 } orc_config;
 
 typedef struct {
-  int32_t qtype;
+  int32_t qt[7];                                   /* block type of wq, wk, wv, wo, wg, wu, wd */
   const uint8_t *wq, *wk, *wv, *wo, *wg, *wu, *wd; /* row-major out x in block matrices */
   const float *attn_norm, *ffn_norm;               /* hidden fp32 each */
 } orc_layer_weights;
@@ -314,9 +407,9 @@ int orc_layer(const orc_config* c, const orc_layer_weights* L, uint16_t* k_cache
 
   for (int64_t i = 0; i < H; ++i) wn[i] = (double)L->attn_norm[i];
   orc_rmsnorm(h, wn, H, c->eps, n1);
-  if (orc_gemv(L->qtype, L->wq, Q, H, n1, q, NULL, nthreads)) goto done;
-  if (orc_gemv(L->qtype, L->wk, KV, H, n1, k, NULL, nthreads)) goto done;
-  if (orc_gemv(L->qtype, L->wv, KV, H, n1, v, NULL, nthreads)) goto done;
+  if (orc_gemv(L->qt[0], L->wq, Q, H, n1, q, NULL, nthreads)) goto done;
+  if (orc_gemv(L->qt[1], L->wk, KV, H, n1, k, NULL, nthreads)) goto done;
+  if (orc_gemv(L->qt[2], L->wv, KV, H, n1, v, NULL, nthreads)) goto done;
   orc_rope(q, c->n_heads, (int)D, pos, c->theta);
   orc_rope(k, c->n_kv_heads, (int)D, pos, c->theta);
   for (int kh = 0; kh < c->n_kv_heads; ++kh)
@@ -325,15 +418,15 @@ int orc_layer(const orc_config* c, const orc_layer_weights* L, uint16_t* k_cache
       v_cache[((int64_t)kh * c->max_ctx + pos) * D + d] = orc_to_half(v[kh * D + d]);
     }
   if (orc_attention(q, k_cache, v_cache, c->n_heads, c->n_kv_heads, (int)D, pos + 1, c->max_ctx, a, NULL)) goto done;
-  if (orc_gemv(L->qtype, L->wo, H, Q, a, t, NULL, nthreads)) goto done;
+  if (orc_gemv(L->qt[3], L->wo, H, Q, a, t, NULL, nthreads)) goto done;
   for (int64_t i = 0; i < H; ++i) h1[i] = h[i] + t[i];
 
   for (int64_t i = 0; i < H; ++i) wn[i] = (double)L->ffn_norm[i];
   orc_rmsnorm(h1, wn, H, c->eps, n2);
-  if (orc_gemv(L->qtype, L->wg, F, H, n2, g, NULL, nthreads)) goto done;
-  if (orc_gemv(L->qtype, L->wu, F, H, n2, u, NULL, nthreads)) goto done;
+  if (orc_gemv(L->qt[4], L->wg, F, H, n2, g, NULL, nthreads)) goto done;
+  if (orc_gemv(L->qt[5], L->wu, F, H, n2, u, NULL, nthreads)) goto done;
   orc_swiglu(g, u, F, s);
-  if (orc_gemv(L->qtype, L->wd, H, F, s, t, NULL, nthreads)) goto done;
+  if (orc_gemv(L->qt[6], L->wd, H, F, s, t, NULL, nthreads)) goto done;
   for (int64_t i = 0; i < H; ++i) h2[i] = h1[i] + t[i];
 
   if (cos_out) *cos_out = orc_cosine(h, h2, H);

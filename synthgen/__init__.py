@@ -23,9 +23,9 @@ CUDA_SO = os.path.join(HERE, "libsynthgen_cuda.so")
 
 SEED_BASE = 0x4E54580
 
-Q4_0, Q8_0, Q6_K = 2, 8, 14
-BLOCK_ELEMS = {Q4_0: 32, Q8_0: 32, Q6_K: 256}
-BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q6_K: 210}
+F32, F16, Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 0, 1, 2, 8, 12, 13, 14
+BLOCK_ELEMS = {F32: 1, F16: 1, Q4_0: 32, Q8_0: 32, Q4_K: 256, Q5_K: 256, Q6_K: 256}
+BLOCK_BYTES = {F32: 4, F16: 2, Q4_0: 18, Q8_0: 34, Q4_K: 144, Q5_K: 176, Q6_K: 210}
 
 _NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

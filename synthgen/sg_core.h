@@ -25,8 +25,13 @@
  *    max|w|/127, q = round(w/d); Q4_0: d = (signed max-|w| element)/-8,
  *    q = clamp(round(w/d)+8, 0, 15); Q6_K: 16-element sub-block scales stored
  *    as int8 relative to one fp16 super-scale, q = clamp(round(w/(d*sc))+32,
- *    0, 63)), rounding half away from zero, block byte layouts as GGUF stores
- *    them (per-format layout in the functions below).
+ *    0, 63); Q4_K / Q5_K: per 32-element sub-block a scale (max - min')/n_max
+ *    and a min -min' with min' = min(0, smallest element), both stored as 6-bit
+ *    codes relative to fp16 super-scales d = (largest scale)/63 and dmin =
+ *    (largest min)/63, q = clamp(round((w + dmin m)/(d sc)), 0, n_max) with
+ *    n_max 15 / 31; F16 / F32: the value itself), rounding half away from
+ *    zero, block byte layouts as GGUF stores them (per-format layout in the
+ *    functions below).
  */
 #ifndef SG_CORE_H
 #define SG_CORE_H
@@ -49,6 +54,8 @@
 #define SG_D2F(a) __double2float_rn((a))
 #define SG_FMUL(a, b) __fmul_rn((a), (b))
 #define SG_FDIV(a, b) __fdiv_rn((a), (b))
+#define SG_FADD(a, b) __fadd_rn((a), (b))
+#define SG_FSUB(a, b) __fsub_rn((a), (b))
 #define SG_AS_U64(d) ((uint64_t)__double_as_longlong(d))
 #define SG_AS_DBL(u) (__longlong_as_double((long long)(u)))
 #define SG_AS_U32(f) ((uint32_t)__float_as_uint(f))
@@ -63,6 +70,8 @@
 #define SG_D2F(a) ((float)(a))
 #define SG_FMUL(a, b) ((a) * (b))
 #define SG_FDIV(a, b) ((a) / (b))
+#define SG_FADD(a, b) ((a) + (b))
+#define SG_FSUB(a, b) ((a) - (b))
 SG_HD uint64_t sg_as_u64_(double d) { uint64_t u; memcpy(&u, &d, 8); return u; }
 SG_HD double sg_as_dbl_(uint64_t u) { double d; memcpy(&d, &u, 8); return d; }
 SG_HD uint32_t sg_as_u32_(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
@@ -74,8 +83,12 @@ SG_HD float sg_as_flt_(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
 #endif
 
 /* GGUF type ids of the formats produced here. */
+#define SG_F32 0
+#define SG_F16 1
 #define SG_Q4_0 2
 #define SG_Q8_0 8
+#define SG_Q4_K 12
+#define SG_Q5_K 13
 #define SG_Q6_K 14
 
 /* Counter word 3 tags the use of a draw so streams never overlap. */
@@ -305,17 +318,101 @@ SG_HD void sg_quant_q6_k(const float* w, uint8_t* blk) {
   blk[208] = (uint8_t)(dh & 0xFF); blk[209] = (uint8_t)(dh >> 8);
 }
 
+/* Q4_K (144 bytes) / Q5_K (176 bytes) super-blocks of 256:
+ *   fp16 d | fp16 dmin | scales[12] | (Q5_K: qh[32]) | qs[128];
+ * sub-block j (32 elements) has a 6-bit scale sc_j and min m_j:
+ *   j < 4:  sc_j = scales[j] & 63, m_j = scales[j+4] & 63;
+ *   j >= 4: sc_j = (scales[j+4] & 15) | (scales[j-4] >> 6) << 4,
+ *           m_j  = (scales[j+4] >> 4) | (scales[j] >> 6) << 4;
+ * element n = 64c + 32h + l takes nibble h of qs[32c + l] (and, for Q5_K,
+ * bit 2c + h of qh[l] as its fifth bit);  w = d sc_j q - dmin m_j. */
+SG_HD void sg_quant_kq(const float* w, uint8_t* blk, int five) {
+  const int nmax = five ? 31 : 15;
+  float s[8], mm[8], smax = 0.0f, mmax = 0.0f;
+  for (int j = 0; j < 8; ++j) {
+    float mn = 0.0f, mx = w[32 * j];
+    for (int i = 0; i < 32; ++i) {
+      float v = w[32 * j + i];
+      if (v < mn) mn = v;
+      if (v > mx) mx = v;
+    }
+    s[j] = SG_FDIV(SG_FSUB(mx, mn), (float)nmax);
+    mm[j] = SG_FSUB(0.0f, mn);
+    if (s[j] > smax) smax = s[j];
+    if (mm[j] > mmax) mmax = mm[j];
+  }
+  uint16_t dh = sg_f32_to_f16(SG_FDIV(smax, 63.0f)), mh = sg_f32_to_f16(SG_FDIV(mmax, 63.0f));
+  float df = sg_f16_to_f32(dh), mf = sg_f16_to_f32(mh);
+  int sc[8], mi[8];
+  for (int j = 0; j < 8; ++j) {
+    sc[j] = (df == 0.0f) ? 0 : sg_clampi(sg_round_away(SG_FDIV(s[j], df)), 0, 63);
+    mi[j] = (mf == 0.0f) ? 0 : sg_clampi(sg_round_away(SG_FDIV(mm[j], mf)), 0, 63);
+  }
+  blk[0] = (uint8_t)(dh & 0xFF); blk[1] = (uint8_t)(dh >> 8);
+  blk[2] = (uint8_t)(mh & 0xFF); blk[3] = (uint8_t)(mh >> 8);
+  uint8_t* p = blk + 4;
+  for (int j = 0; j < 4; ++j) {
+    p[j] = (uint8_t)((sc[j] & 63) | ((sc[j + 4] >> 4) << 6));
+    p[j + 4] = (uint8_t)((mi[j] & 63) | ((mi[j + 4] >> 4) << 6));
+    p[j + 8] = (uint8_t)((sc[j + 4] & 15) | ((mi[j + 4] & 15) << 4));
+  }
+  uint8_t* qh = blk + 16;
+  uint8_t* qs = blk + (five ? 48 : 16);
+  for (int i = 0; i < 128; ++i) qs[i] = 0;
+  if (five)
+    for (int i = 0; i < 32; ++i) qh[i] = 0;
+  for (int n = 0; n < 256; ++n) {
+    const int j = n / 32, c = n / 64, h = (n % 64) / 32, l = n % 32;
+    float step = SG_FMUL(df, (float)sc[j]);
+    float off = SG_FMUL(mf, (float)mi[j]);
+    int q = (step == 0.0f) ? 0 : sg_clampi(sg_round_away(SG_FDIV(SG_FADD(w[n], off), step)), 0, nmax);
+    qs[32 * c + l] |= (uint8_t)((q & 15) << (4 * h));
+    if (five) qh[l] |= (uint8_t)(((q >> 4) & 1) << (2 * c + h));
+  }
+}
+
+/* F16: one binary16 per weight (little-endian); F32: the binary32 itself. */
+SG_HD void sg_quant_f16(const float* w, uint8_t* blk) {
+  uint16_t h = sg_f32_to_f16(w[0]);
+  blk[0] = (uint8_t)(h & 0xFF); blk[1] = (uint8_t)(h >> 8);
+}
+SG_HD void sg_quant_f32(const float* w, uint8_t* blk) {
+  uint32_t u = SG_AS_U32(w[0]);
+  for (int i = 0; i < 4; ++i) blk[i] = (uint8_t)(u >> (8 * i));
+}
+
 SG_HD int sg_block_elems(int qtype) {
-  return qtype == SG_Q6_K ? 256 : ((qtype == SG_Q8_0 || qtype == SG_Q4_0) ? 32 : 0);
+  switch (qtype) {
+    case SG_F32: case SG_F16: return 1;
+    case SG_Q4_0: case SG_Q8_0: return 32;
+    case SG_Q4_K: case SG_Q5_K: case SG_Q6_K: return 256;
+    default: return 0;
+  }
 }
 SG_HD int sg_block_bytes(int qtype) {
-  return qtype == SG_Q6_K ? 210 : (qtype == SG_Q8_0 ? 34 : (qtype == SG_Q4_0 ? 18 : 0));
+  switch (qtype) {
+    case SG_F32: return 4;
+    case SG_F16: return 2;
+    case SG_Q4_0: return 18;
+    case SG_Q8_0: return 34;
+    case SG_Q4_K: return 144;
+    case SG_Q5_K: return 176;
+    case SG_Q6_K: return 210;
+    default: return 0;
+  }
 }
 
 SG_HD void sg_quant_block(int qtype, const float* w, uint8_t* blk) {
-  if (qtype == SG_Q8_0) sg_quant_q8_0(w, blk);
-  else if (qtype == SG_Q4_0) sg_quant_q4_0(w, blk);
-  else if (qtype == SG_Q6_K) sg_quant_q6_k(w, blk);
+  switch (qtype) {
+    case SG_Q8_0: sg_quant_q8_0(w, blk); break;
+    case SG_Q4_0: sg_quant_q4_0(w, blk); break;
+    case SG_Q6_K: sg_quant_q6_k(w, blk); break;
+    case SG_Q4_K: sg_quant_kq(w, blk, 0); break;
+    case SG_Q5_K: sg_quant_kq(w, blk, 1); break;
+    case SG_F16: sg_quant_f16(w, blk); break;
+    case SG_F32: sg_quant_f32(w, blk); break;
+    default: break;
+  }
 }
 
 #endif /* SG_CORE_H */

@@ -32,8 +32,9 @@ __global__ void k_tokens(uint32_t seed, uint32_t tid, int64_t n, uint32_t V, int
 template <int QT>
 __global__ void k_quant_rows(uint32_t seed, uint32_t tid, int64_t row0, int64_t nrows, int64_t K, double mean,
                              double sigma, uint8_t* out) {
-  constexpr int BE = QT == SG_Q6_K ? 256 : 32;
-  constexpr int BB = QT == SG_Q6_K ? 210 : (QT == SG_Q8_0 ? 34 : 18);
+  constexpr int BE = (QT == SG_Q6_K || QT == SG_Q4_K || QT == SG_Q5_K) ? 256 : (QT == SG_F16 || QT == SG_F32) ? 1 : 32;
+  constexpr int BB = QT == SG_Q6_K ? 210 : QT == SG_Q4_K ? 144 : QT == SG_Q5_K ? 176 : QT == SG_Q8_0 ? 34
+                   : QT == SG_Q4_0 ? 18 : QT == SG_F16 ? 2 : 4;
   const int64_t nb = K / BE;
   const int64_t total = nrows * nb;
   float w[BE];
@@ -81,12 +82,29 @@ int sgc_quant_rows(int qtype, uint32_t seed, uint32_t tid, int64_t row0, int64_t
   const int64_t total = nrows * (K / be);
   if (total <= 0) return 0;
   cudaStream_t s = (cudaStream_t)stream;
-  if (qtype == SG_Q8_0)
-    k_quant_rows<SG_Q8_0><<<grid_for(total, 128), 128, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
-  else if (qtype == SG_Q4_0)
-    k_quant_rows<SG_Q4_0><<<grid_for(total, 128), 128, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
-  else
-    k_quant_rows<SG_Q6_K><<<grid_for(total, 64), 64, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
+  switch (qtype) {
+    case SG_Q8_0:
+      k_quant_rows<SG_Q8_0><<<grid_for(total, 128), 128, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
+      break;
+    case SG_Q4_0:
+      k_quant_rows<SG_Q4_0><<<grid_for(total, 128), 128, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
+      break;
+    case SG_Q6_K:
+      k_quant_rows<SG_Q6_K><<<grid_for(total, 64), 64, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
+      break;
+    case SG_Q4_K:
+      k_quant_rows<SG_Q4_K><<<grid_for(total, 64), 64, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
+      break;
+    case SG_Q5_K:
+      k_quant_rows<SG_Q5_K><<<grid_for(total, 64), 64, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
+      break;
+    case SG_F16:
+      k_quant_rows<SG_F16><<<grid_for(total, 256), 256, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
+      break;
+    default:
+      k_quant_rows<SG_F32><<<grid_for(total, 256), 256, 0, s>>>(seed, tid, row0, nrows, K, mean, sigma, out);
+      break;
+  }
   return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 
