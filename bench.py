@@ -214,7 +214,8 @@ class Run:
                                    L, d["eps"], d["theta"], max_ctx, 0.98)
         layers = []
         for l in range(L):
-            _, lw = ntx.ntx_layer_layout(self.cfg, qt)
+            _, lw = (ntx.ntx_layer_layout_mixed(self.cfg, qt) if isinstance(qt, (list, tuple))
+                     else ntx.ntx_layer_layout(self.cfg, qt))
             src = m.resident_copy[l] if (resident_layers or tier_map[l] == 0) else m.layers[l]
             lw.base = src.data_ptr()
             layers.append(lw)

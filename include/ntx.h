@@ -62,13 +62,27 @@ extern "C" {
  *         element n (h = n/128, g = (n%128)/32, l = n%32): low 4 bits in
  *         ql[64h + 32(g%2) + l] (low nibble if g < 2, else high), high 2 bits
  *         at bit 2g of qh[32h + l];                               w = d sc[n/16] (q - 32)
+ *   Q4_K: 144 B per 256 weights = fp16 d | fp16 dmin | 12 B scales | qs[128]
+ *         (the super-blocks of the table's Q4_K_M, 4.5 bit/weight);
+ *   Q5_K: 176 B per 256 weights = fp16 d | fp16 dmin | 12 B scales | qh[32] |
+ *         qs[128] (5.5 bit/weight).  Both: eight 32-weight sub-blocks, each a
+ *         6-bit scale sc_j and min m_j (j < 4: low six bits of scale bytes j
+ *         and j+4; j >= 4: low / high nibble of byte j+4 plus the top two bits
+ *         of bytes j-4 / j); element n = 64c + 32h + l: nibble h of
+ *         qs[32c + l], Q5_K fifth bit = bit 2c+h of qh[l];    w = d sc_j q - dmin m_j
+ *   F16, F32: one IEEE binary16 / binary32 per weight.
  * Weight matrices are row-major (out x in) with each row a run of K/block
  * blocks. */
 #define NTX_F32 0
 #define NTX_F16 1
 #define NTX_Q4_0 2
 #define NTX_Q8_0 8
+#define NTX_Q4_K 12
+#define NTX_Q5_K 13
 #define NTX_Q6_K 14
+/* ntx_layer_weights.qtype of a layer whose matrices have their own types
+ * (mat_qtype[]), e.g. a Q4_K_M model ("mixed", [ShowHN] 量子化フォーマット対応表). */
+#define NTX_MIXED (-1)
 
 NTX_API const char* ntx_last_error(void);
 NTX_API int ntx_version(void); /* major*10000 + minor*100 + patch */
@@ -102,11 +116,13 @@ NTX_API int ntx_set_gemv_pdl(int on);
 
 /* ------------------------------------------------------------ per-op calls */
 
-/* Dequantize n weights ([README] 主な機能: GGUF Q4_0/Q8_0/Q6_K; [ShowHN]
- * 量子化フォーマット対応表).  blocks: device, n/block_elems consecutive blocks,
- * 2-byte aligned.  out: device fp32[n].  Exact: every value d*sc*(q-off) is
- * representable in fp32.  NTX_ERR_SHAPE if n is not a multiple of the block
- * length; NTX_ERR_QTYPE for other types. */
+/* Dequantize n weights ([README] 主な機能: GGUF Q4_0/Q8_0/Q4_K_M/Q5_K/Q6_K/F16/F32;
+ * [ShowHN] 量子化フォーマット対応表).  blocks: device, n/block_elems
+ * consecutive blocks, 2-byte aligned (4-byte for F32).  out: device fp32[n].
+ * Q8_0, Q4_0, Q6_K, F16, F32 are exact (every value is representable in
+ * fp32); Q4_K / Q5_K give d sc q - dmin m rounded once to fp32 (the products
+ * are exact).  NTX_ERR_SHAPE if n is not a multiple of the block length;
+ * NTX_ERR_QTYPE for other types. */
 NTX_API int ntx_dequant(int qtype, const void* blocks, float* out, int64_t n, void* stream);
 
 /* Quantized GEMV y = W_deq x (+ residual) with fp32 accumulation ([README]
@@ -115,9 +131,11 @@ NTX_API int ntx_dequant(int qtype, const void* blocks, float* out, int64_t n, vo
  *   W: device, M rows of K/block_elems blocks (row-major), 16-byte aligned.
  *   x: device fp32[K].  y: device fp32[M], must not overlap x.
  *   residual: device fp32[M] or NULL; may be y itself (y = W x + y).
+ * Types: Q8_0, Q4_0, Q4_K, Q5_K, Q6_K, F16, F32.
  * Limits: 1 <= M <= 2^31-1, block_elems | K, K <= 262144.  Shapes with
- * K % 256 == 0 (Q8_0, Q4_0) or K % 2048 == 0 (Q6_K) take the bulk-copy
- * pipeline; other K take a slower generic kernel with the same results.
+ * K % 2048 == 0 (Q6_K) or K % 256 == 0 (the others) and K <= 30720 take the
+ * bulk-copy pipeline; other K take a slower generic kernel with the same
+ * results.
  * Errors: NTX_ERR_QTYPE, NTX_ERR_SHAPE, NTX_ERR_ALIGN (W, x, y or residual
  * not 16-B aligned), NTX_ERR_INVALID_ARG (NULL, y overlapping x, residual
  * partially overlapping y). */
@@ -199,14 +217,21 @@ typedef struct {
  * ffn_norm as fp32[H].  The same layout serves resident and pinned-host
  * copies, so streaming a layer is one contiguous copy. */
 typedef struct {
-  int32_t qtype;
+  int32_t qtype;  /* block type of every matrix, or NTX_MIXED: mat_qtype[] holds them */
   const void* base;
   uint64_t off_wq, off_wk, off_wv, off_wo, off_wg, off_wu, off_wd, off_attn_norm, off_ffn_norm;
+  int32_t mat_qtype[7]; /* wq, wk, wv, wo, wg, wu, wd; read only when qtype == NTX_MIXED */
 } ntx_layer_weights;
 
 /* Fills the canonical offsets of a layer blob for cfg and qtype (base left
  * NULL) and returns the blob size in bytes, 0 on bad arguments. */
 NTX_API uint64_t ntx_layer_layout(const ntx_model_config* cfg, int qtype, ntx_layer_weights* out);
+
+/* The same for a layer whose seven matrices wq, wk, wv, wo, wg, wu, wd have
+ * the block types qtypes[0..6] (host array); sets qtype = NTX_MIXED.  A layer
+ * runs only if wq, wk and wv share one type and wg and wu share one type (each
+ * pair or triple is one fused GEMV).  0 on bad arguments. */
+NTX_API uint64_t ntx_layer_layout_mixed(const ntx_model_config* cfg, const int32_t* qtypes, ntx_layer_weights* out);
 
 /* Workspace one ntx_decode_layer call needs (device bytes). */
 NTX_API size_t ntx_layer_workspace_bytes(const ntx_model_config* cfg);

@@ -25,11 +25,12 @@ NTX_ERR_CUDA = -5
 NTX_ERR_TIMEOUT = -6
 NTX_ERR_NOMEM = -7
 
-NTX_F32, NTX_F16, NTX_Q4_0, NTX_Q8_0, NTX_Q6_K = 0, 1, 2, 8, 14
+NTX_F32, NTX_F16, NTX_Q4_0, NTX_Q8_0, NTX_Q4_K, NTX_Q5_K, NTX_Q6_K = 0, 1, 2, 8, 12, 13, 14
+NTX_MIXED = -1
 NTX_CALIBRATE_SKIP, NTX_USE_SKIP, NTX_NO_GRAPH, NTX_NO_PERSIST = 1, 2, 4, 8
 
-BLOCK_ELEMS = {NTX_Q4_0: 32, NTX_Q8_0: 32, NTX_Q6_K: 256}
-BLOCK_BYTES = {NTX_Q4_0: 18, NTX_Q8_0: 34, NTX_Q6_K: 210}
+BLOCK_ELEMS = {NTX_F32: 1, NTX_F16: 1, NTX_Q4_0: 32, NTX_Q8_0: 32, NTX_Q4_K: 256, NTX_Q5_K: 256, NTX_Q6_K: 256}
+BLOCK_BYTES = {NTX_F32: 4, NTX_F16: 2, NTX_Q4_0: 18, NTX_Q8_0: 34, NTX_Q4_K: 144, NTX_Q5_K: 176, NTX_Q6_K: 210}
 
 # Symbols exported by libntx (all declared in include/ntx.h).
 EXPORTS = (
@@ -38,7 +39,7 @@ EXPORTS = (
     "ntx_swiglu", "ntx_layer_layout", "ntx_layer_workspace_bytes", "ntx_decode_layer", "ntx_engine_workspace_bytes",
     "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
     "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
-    "ntx_persistent_plan",
+    "ntx_persistent_plan", "ntx_layer_layout_mixed",
 )
 
 
@@ -58,7 +59,7 @@ class ntx_model_config(ctypes.Structure):
 class ntx_layer_weights(ctypes.Structure):
     _fields_ = [("qtype", ctypes.c_int32), ("base", ctypes.c_void_p)] + [
         (n, ctypes.c_uint64) for n in ("off_wq", "off_wk", "off_wv", "off_wo", "off_wg", "off_wu", "off_wd",
-                                       "off_attn_norm", "off_ffn_norm")]
+                                       "off_attn_norm", "off_ffn_norm")] + [("mat_qtype", ctypes.c_int32 * 7)]
 
 
 _lib = None
@@ -89,6 +90,8 @@ def lib():
             "ntx_attn_decode": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp], i32),
             "ntx_swiglu": ([vp, vp, vp, i64, vp], i32),
             "ntx_layer_layout": ([P(ntx_model_config), i32, P(ntx_layer_weights)], ctypes.c_uint64),
+            "ntx_layer_layout_mixed": ([P(ntx_model_config), P(ctypes.c_int32), P(ntx_layer_weights)],
+                                       ctypes.c_uint64),
             "ntx_layer_workspace_bytes": ([P(ntx_model_config)], sz),
             "ntx_decode_layer": ([P(ntx_model_config), P(ntx_layer_weights), vp, vp, vp, i32, vp, vp, sz, vp], i32),
             "ntx_engine_workspace_bytes": ([P(ntx_model_config)], sz),
@@ -213,6 +216,17 @@ def ntx_layer_layout(cfg: ntx_model_config, qtype: int):
     n = lib().ntx_layer_layout(ctypes.byref(cfg), qtype, ctypes.byref(w))
     if n == 0:
         raise NtxError(NTX_ERR_INVALID_ARG, "ntx_layer_layout: bad config or type")
+    return int(n), w
+
+
+def ntx_layer_layout_mixed(cfg: ntx_model_config, qtypes):
+    """qtypes: the seven block types of wq, wk, wv, wo, wg, wu, wd.  Returns
+    (blob_bytes, ntx_layer_weights with base NULL and qtype NTX_MIXED)."""
+    w = ntx_layer_weights()
+    t = (ctypes.c_int32 * 7)(*qtypes)
+    n = lib().ntx_layer_layout_mixed(ctypes.byref(cfg), t, ctypes.byref(w))
+    if n == 0:
+        raise NtxError(NTX_ERR_INVALID_ARG, "ntx_layer_layout_mixed: bad config or types")
     return int(n), w
 
 

@@ -36,9 +36,30 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-int block_elems(int qt) { return qt == NTX_Q6_K ? 256 : ((qt == NTX_Q8_0 || qt == NTX_Q4_0) ? 32 : 0); }
-int block_bytes(int qt) { return qt == NTX_Q6_K ? 210 : (qt == NTX_Q8_0 ? 34 : (qt == NTX_Q4_0 ? 18 : 0)); }
-bool qtype_ok(int qt) { return qt == NTX_Q8_0 || qt == NTX_Q4_0 || qt == NTX_Q6_K; }
+int block_elems(int qt) {
+  switch (qt) {
+    case NTX_F32: case NTX_F16: return 1;
+    case NTX_Q4_0: case NTX_Q8_0: return 32;
+    case NTX_Q4_K: case NTX_Q5_K: case NTX_Q6_K: return 256;
+    default: return 0;
+  }
+}
+int block_bytes(int qt) {
+  switch (qt) {
+    case NTX_F32: return 4;
+    case NTX_F16: return 2;
+    case NTX_Q4_0: return 18;
+    case NTX_Q8_0: return 34;
+    case NTX_Q4_K: return 144;
+    case NTX_Q5_K: return 176;
+    case NTX_Q6_K: return 210;
+    default: return 0;
+  }
+}
+bool qtype_ok(int qt) { return block_elems(qt) != 0; }
+
+// Block type of matrix i (0..6 = wq, wk, wv, wo, wg, wu, wd) of a layer.
+int mat_qt(const ntx_layer_weights* w, int i) { return w->qtype == NTX_MIXED ? w->mat_qtype[i] : w->qtype; }
 
 int64_t mat_bytes(int qt, int64_t M, int64_t K) { return M * (K / block_elems(qt)) * block_bytes(qt); }
 
@@ -54,20 +75,38 @@ cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 // K constraint of the fused (bulk-copy) GEMV path.
 bool k_ok_fused(int qt, int64_t K) { return qt == NTX_Q6_K ? K % 2048 == 0 : K % 256 == 0; }
 
-int check_config(const ntx_model_config* c, int qtype) {
+int check_dims(const ntx_model_config* c) {
   if (!c) return fail(NTX_ERR_INVALID_ARG, "config is NULL");
-  if (!qtype_ok(qtype)) return fail(NTX_ERR_QTYPE, "unsupported weight type %d", qtype);
   if (c->hidden <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 || c->ffn <= 0 || c->n_layers < 0 || c->max_ctx <= 0)
     return fail(NTX_ERR_SHAPE, "non-positive dimension in config");
   if (c->head_dim != 128) return fail(NTX_ERR_SHAPE, "head_dim %d unsupported (128 only)", c->head_dim);
   if (c->n_heads % c->n_kv_heads) return fail(NTX_ERR_SHAPE, "n_heads %% n_kv_heads != 0");
   const int G = c->n_heads / c->n_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(NTX_ERR_SHAPE, "query group %d unsupported (1,2,4,8)", G);
-  const int64_t Q = (int64_t)c->n_heads * c->head_dim;
-  if (!k_ok_fused(qtype, c->hidden) || !k_ok_fused(qtype, c->ffn) || !k_ok_fused(qtype, Q))
-    return fail(NTX_ERR_SHAPE, "hidden/ffn/heads*head_dim must be multiples of %d for type %d",
-                qtype == NTX_Q6_K ? 2048 : 256, qtype);
   if (!(c->eps >= 0.f) || !(c->theta > 0.f)) return fail(NTX_ERR_INVALID_ARG, "bad eps/theta");
+  return NTX_OK;
+}
+
+// Dimensions and the block type of every matrix of a layer: each type known,
+// each matrix's input length a whole number of bulk-copy units, and the
+// matrices that share one GEMV (wq/wk/wv, wg/wu) of one type.
+int check_config(const ntx_model_config* c, const ntx_layer_weights* w) {
+  int rc = check_dims(c);
+  if (rc) return rc;
+  if (w->qtype != NTX_MIXED && !qtype_ok(w->qtype)) return fail(NTX_ERR_QTYPE, "unsupported weight type %d", w->qtype);
+  const int64_t Q = (int64_t)c->n_heads * c->head_dim;
+  const int64_t K[7] = {c->hidden, c->hidden, c->hidden, Q, c->hidden, c->hidden, c->ffn};
+  static const char* names[7] = {"wq", "wk", "wv", "wo", "wg", "wu", "wd"};
+  for (int i = 0; i < 7; ++i) {
+    const int qt = mat_qt(w, i);
+    if (!qtype_ok(qt)) return fail(NTX_ERR_QTYPE, "%s: unsupported weight type %d", names[i], qt);
+    if (!k_ok_fused(qt, K[i]))
+      return fail(NTX_ERR_SHAPE, "%s: input length %lld must be a multiple of %d for type %d", names[i],
+                  (long long)K[i], qt == NTX_Q6_K ? 2048 : 256, qt);
+  }
+  if (mat_qt(w, 1) != mat_qt(w, 0) || mat_qt(w, 2) != mat_qt(w, 0))
+    return fail(NTX_ERR_QTYPE, "wq, wk and wv must share one block type (one fused GEMV)");
+  if (mat_qt(w, 5) != mat_qt(w, 4)) return fail(NTX_ERR_QTYPE, "wg and wu must share one block type (one fused GEMV)");
   return NTX_OK;
 }
 
@@ -220,28 +259,37 @@ int ntx_swiglu(const float* gate, const float* up, float* out, int64_t n, void* 
   return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_swiglu");
 }
 
-uint64_t ntx_layer_layout(const ntx_model_config* cfg, int qtype, ntx_layer_weights* out) {
-  if (!cfg || !out || !qtype_ok(qtype) || cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 ||
-      cfg->n_kv_heads <= 0 || cfg->head_dim <= 0)
+uint64_t ntx_layer_layout_mixed(const ntx_model_config* cfg, const int32_t* qtypes, ntx_layer_weights* out) {
+  if (!cfg || !out || !qtypes || cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 || cfg->n_kv_heads <= 0 ||
+      cfg->head_dim <= 0)
     return 0;
   const int64_t H = cfg->hidden, F = cfg->ffn, Q = (int64_t)cfg->n_heads * cfg->head_dim,
                 KV = (int64_t)cfg->n_kv_heads * cfg->head_dim;
-  if (H % block_elems(qtype) || F % block_elems(qtype) || Q % block_elems(qtype)) return 0;
+  const int64_t M[7] = {Q, KV, KV, H, F, F, H}, K[7] = {H, H, H, Q, H, H, F};
+  for (int i = 0; i < 7; ++i)
+    if (!qtype_ok(qtypes[i]) || K[i] % block_elems(qtypes[i])) return 0;
   ntx_layer_weights w;
   memset(&w, 0, sizeof w);
-  w.qtype = qtype;
+  w.qtype = NTX_MIXED;
+  for (int i = 0; i < 7; ++i) w.mat_qtype[i] = qtypes[i];
+  uint64_t* offs[7] = {&w.off_wq, &w.off_wk, &w.off_wv, &w.off_wo, &w.off_wg, &w.off_wu, &w.off_wd};
   uint64_t o = 0;
-  w.off_wq = o; o = align256(o + mat_bytes(qtype, Q, H));
-  w.off_wk = o; o = align256(o + mat_bytes(qtype, KV, H));
-  w.off_wv = o; o = align256(o + mat_bytes(qtype, KV, H));
-  w.off_wo = o; o = align256(o + mat_bytes(qtype, H, Q));
-  w.off_wg = o; o = align256(o + mat_bytes(qtype, F, H));
-  w.off_wu = o; o = align256(o + mat_bytes(qtype, F, H));
-  w.off_wd = o; o = align256(o + mat_bytes(qtype, H, F));
+  for (int i = 0; i < 7; ++i) {
+    *offs[i] = o;
+    o = align256(o + mat_bytes(qtypes[i], M[i], K[i]));
+  }
   w.off_attn_norm = o; o = align256(o + 4 * H);
   w.off_ffn_norm = o; o = align256(o + 4 * H);
   *out = w;
   return o;
+}
+
+uint64_t ntx_layer_layout(const ntx_model_config* cfg, int qtype, ntx_layer_weights* out) {
+  if (!qtype_ok(qtype)) return 0;
+  const int32_t t[7] = {qtype, qtype, qtype, qtype, qtype, qtype, qtype};
+  const uint64_t n = ntx_layer_layout_mixed(cfg, t, out);
+  if (n) out->qtype = qtype;  // one type: the per-matrix list is informational
+  return n;
 }
 
 size_t ntx_layer_workspace_bytes(const ntx_model_config* cfg) {
@@ -255,18 +303,17 @@ namespace {
 
 // Extent of a layer blob given its offsets (for copies and bounds).
 uint64_t layer_extent(const ntx_model_config* c, const ntx_layer_weights* w) {
-  const int qt = w->qtype;
   const int64_t H = c->hidden, F = c->ffn, Q = (int64_t)c->n_heads * c->head_dim,
                 KV = (int64_t)c->n_kv_heads * c->head_dim;
   uint64_t e = 0;
   auto upd = [&](uint64_t off, uint64_t n) { if (off + n > e) e = off + n; };
-  upd(w->off_wq, mat_bytes(qt, Q, H));
-  upd(w->off_wk, mat_bytes(qt, KV, H));
-  upd(w->off_wv, mat_bytes(qt, KV, H));
-  upd(w->off_wo, mat_bytes(qt, H, Q));
-  upd(w->off_wg, mat_bytes(qt, F, H));
-  upd(w->off_wu, mat_bytes(qt, F, H));
-  upd(w->off_wd, mat_bytes(qt, H, F));
+  upd(w->off_wq, mat_bytes(mat_qt(w, 0), Q, H));
+  upd(w->off_wk, mat_bytes(mat_qt(w, 1), KV, H));
+  upd(w->off_wv, mat_bytes(mat_qt(w, 2), KV, H));
+  upd(w->off_wo, mat_bytes(mat_qt(w, 3), H, Q));
+  upd(w->off_wg, mat_bytes(mat_qt(w, 4), F, H));
+  upd(w->off_wu, mat_bytes(mat_qt(w, 5), F, H));
+  upd(w->off_wd, mat_bytes(mat_qt(w, 6), H, F));
   upd(w->off_attn_norm, 4 * H);
   upd(w->off_ffn_norm, 4 * H);
   return e;
@@ -280,10 +327,13 @@ int check_offsets(const ntx_layer_weights* w) {
   return NTX_OK;
 }
 
-ntx::LayerArgs layer_args(const ntx_model_config* c, const uint8_t* base, int qtype, const ntx_layer_weights* w) {
+ntx::LayerArgs layer_args(const ntx_model_config* c, const uint8_t* base, const ntx_layer_weights* w) {
   ntx::LayerArgs a;
   memset(&a, 0, sizeof a);
-  a.qtype = qtype;
+  a.qt_qkv = mat_qt(w, 0);
+  a.qt_o = mat_qt(w, 3);
+  a.qt_gu = mat_qt(w, 4);
+  a.qt_down = mat_qt(w, 6);
   a.H = c->hidden; a.Hq = c->n_heads; a.Hkv = c->n_kv_heads; a.D = c->head_dim; a.F = c->ffn;
   a.max_ctx = c->max_ctx; a.eps = c->eps; a.theta = c->theta;
   a.wq = base + w->off_wq; a.wk = base + w->off_wk; a.wv = base + w->off_wv; a.wo = base + w->off_wo;
@@ -299,7 +349,7 @@ extern "C" int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_wei
                                 uint16_t* v_cache, float* hidden, int pos, float* cos_out, void* workspace,
                                 size_t ws_bytes, void* stream) {
   if (!w) return fail(NTX_ERR_INVALID_ARG, "weights NULL");
-  int rc = check_config(cfg, w->qtype);
+  int rc = check_config(cfg, w);
   if (rc) return rc;
   if (!w->base || !k_cache || !v_cache || !hidden || !workspace) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
   if (pos < 0 || pos >= cfg->max_ctx) return fail(NTX_ERR_SHAPE, "pos %d outside [0, max_ctx)", pos);
@@ -311,7 +361,7 @@ extern "C" int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_wei
   const int n_split = ntx::attn_splits(cfg->n_kv_heads, pos + 1);
   LayerWs ws;
   carve_layer(cfg, ntx::attn_splits(cfg->n_kv_heads, cfg->max_ctx), static_cast<uint8_t*>(workspace), &ws);
-  ntx::LayerArgs a = layer_args(cfg, static_cast<const uint8_t*>(w->base), w->qtype, w);
+  ntx::LayerArgs a = layer_args(cfg, static_cast<const uint8_t*>(w->base), w);
   a.k_cache = k_cache; a.v_cache = v_cache; a.hidden = hidden;
   const int nin = ntx::layer_stats_parts(cfg->hidden);
   a.stats_in = ws.stats_in; a.n_stats_in = nin;
@@ -442,8 +492,7 @@ cudaError_t upload_players(ntx_engine* e, const std::vector<int>& list, ntx::PLa
   std::vector<ntx::PLayer> t(list.size());
   for (size_t i = 0; i < list.size(); ++i) {
     const int l = list[i];
-    const ntx::LayerArgs a = layer_args(&e->cfg, static_cast<const uint8_t*>(e->layers[l].base), e->layers[l].qtype,
-                                        &e->layers[l]);
+    const ntx::LayerArgs a = layer_args(&e->cfg, static_cast<const uint8_t*>(e->layers[l].base), &e->layers[l]);
     ntx::PLayer& p = t[i];
     p.wq = a.wq; p.wk = a.wk; p.wv = a.wv; p.wo = a.wo; p.wg = a.wg; p.wu = a.wu; p.wd = a.wd;
     p.attn_norm = a.attn_norm; p.ffn_norm = a.ffn_norm;
@@ -474,7 +523,7 @@ cudaError_t persist_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t
   cudaError_t err =
       cudaMemsetAsync(e->psync, 0, sizeof(unsigned) * ntx::persist_sync_words(nrun, c.n_kv_heads), s);
   if (err == cudaSuccess && probe && !e->probe_b.empty()) err = cudaEventRecord(e->probe_b[0], s);
-  if (err == cudaSuccess) err = ntx::launch_persist(e->layers.empty() ? e->head_qtype : e->layers[0].qtype, st,
+  if (err == cudaSuccess) err = ntx::launch_persist(e->head_qtype, st,
                                                     e->psmem, e->pgrid, s);
   if (err == cudaSuccess && probe && !e->probe_e.empty()) err = cudaEventRecord(e->probe_e[0], s);
   if (err != cudaSuccess) return err;
@@ -541,7 +590,7 @@ cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t*
       if (err != cudaSuccess) return err;
       base = e->slot[sl];
     }
-    ntx::LayerArgs a = layer_args(&c, base, e->layers[l].qtype, &e->layers[l]);
+    ntx::LayerArgs a = layer_args(&c, base, &e->layers[l]);
     a.k_cache = e->kc[l]; a.v_cache = e->vc[l]; a.hidden = e->hidden;
     a.stats_in = stats_in; a.n_stats_in = n_in;
     a.stats_o = e->stats_o;
@@ -603,7 +652,7 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   *out = nullptr;
   if (!cfg || (cfg->n_layers > 0 && (!layers || !k_caches || !v_caches)))
     return fail(NTX_ERR_INVALID_ARG, "NULL config, layers or caches");
-  int rc = check_config(cfg, cfg->n_layers > 0 ? layers[0].qtype : head_qtype);
+  int rc = check_dims(cfg);
   if (rc) return rc;
   if (!qtype_ok(head_qtype) || !k_ok_fused(head_qtype, cfg->hidden))
     return fail(NTX_ERR_QTYPE, "unsupported head type %d for hidden %d", head_qtype, cfg->hidden);
@@ -615,7 +664,7 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   if (ws_bytes < ntx_engine_workspace_bytes(cfg)) return fail(NTX_ERR_NOMEM, "workspace too small");
   bool any_host = false;
   for (int l = 0; l < cfg->n_layers; ++l) {
-    if ((rc = check_config(cfg, layers[l].qtype))) return rc;
+    if ((rc = check_config(cfg, &layers[l]))) return rc;
     if ((rc = check_offsets(&layers[l]))) return rc;
     if (!layers[l].base || !k_caches[l] || !v_caches[l]) return fail(NTX_ERR_INVALID_ARG, "layer %d: NULL pointer", l);
     const int t = tier_map ? tier_map[l] : 0;
@@ -666,7 +715,8 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   // skip set that skips every host layer)
   e->persist = e->persist_full = e->persist_skip = false;
   bool one_type = head_qtype == NTX_Q8_0 || head_qtype == NTX_Q4_0 || head_qtype == NTX_Q6_K;
-  for (int l = 0; l < cfg->n_layers && one_type; ++l) one_type = layers[l].qtype == head_qtype;
+  for (int l = 0; l < cfg->n_layers && one_type; ++l)
+    for (int i = 0; i < 7; ++i) one_type = one_type && mat_qt(&layers[l], i) == head_qtype;
   if (err == cudaSuccess && one_type) {
     ntx::PStep st;
     memset(&st, 0, sizeof st);
@@ -677,7 +727,7 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
       const int grid = ntx::persist_grid(qt, psm);
       bool ok = grid > 0 && grid == ntx::sm_count() && ntx::gemv_tma_ok(qt, head, cfg->hidden);
       for (int l = 0; l < cfg->n_layers && ok; ++l) {
-        const ntx::LayerArgs a = layer_args(cfg, static_cast<const uint8_t*>(layers[l].base), qt, &layers[l]);
+        const ntx::LayerArgs a = layer_args(cfg, static_cast<const uint8_t*>(layers[l].base), &layers[l]);
         const int64_t KO = (int64_t)cfg->n_heads * cfg->head_dim;
         ok = ntx::gemv_tma_ok(qt, a.wq, cfg->hidden) && ntx::gemv_tma_ok(qt, a.wk, cfg->hidden) &&
              ntx::gemv_tma_ok(qt, a.wv, cfg->hidden) && ntx::gemv_tma_ok(qt, a.wo, KO) &&

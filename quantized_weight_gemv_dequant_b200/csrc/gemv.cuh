@@ -31,7 +31,12 @@
 
 namespace ntx {
 
-constexpr int QT_Q4_0 = 2, QT_Q8_0 = 8, QT_Q6_K = 14;
+constexpr int QT_F32 = 0, QT_F16 = 1, QT_Q4_0 = 2, QT_Q8_0 = 8, QT_Q4_K = 12, QT_Q5_K = 13, QT_Q6_K = 14;
+
+// Formats whose lanes hold x as fp32 in registers (no fixed-point staging).
+__host__ __device__ constexpr bool qt_float(int qt) { return qt == QT_F16 || qt == QT_F32; }
+// Formats with Q4_K-style super-blocks (fp16 d, dmin, packed 6-bit scales and mins).
+__host__ __device__ constexpr bool qt_kmin(int qt) { return qt == QT_Q4_K || qt == QT_Q5_K; }
 
 #ifndef NTX_GEMV_MAX_CONSUMERS
 #define NTX_GEMV_MAX_CONSUMERS 15
@@ -60,6 +65,30 @@ template <>
 struct QTraits<QT_Q6_K> {
   static constexpr int BE = 256, BB = 210, SEG = kSliceCols / 256 * 210;
 };
+template <>
+struct QTraits<QT_Q4_K> {
+  static constexpr int BE = 256, BB = 144, SEG = kSliceCols / 256 * 144;
+};
+template <>
+struct QTraits<QT_Q5_K> {
+  static constexpr int BE = 256, BB = 176, SEG = kSliceCols / 256 * 176;
+};
+template <>
+struct QTraits<QT_F16> {
+  static constexpr int BE = 1, BB = 2, SEG = kSliceCols * 2;
+};
+template <>
+struct QTraits<QT_F32> {
+  static constexpr int BE = 1, BB = 4, SEG = kSliceCols * 4;
+};
+
+__host__ __device__ constexpr int qt_block_elems(int qt) {
+  return qt == QT_Q6_K || qt == QT_Q4_K || qt == QT_Q5_K ? 256 : qt_float(qt) ? 1 : 32;
+}
+__host__ __device__ constexpr int qt_block_bytes(int qt) {
+  return qt == QT_Q6_K ? 210 : qt == QT_Q4_K ? 144 : qt == QT_Q5_K ? 176 : qt == QT_Q8_0 ? 34 : qt == QT_Q4_0 ? 18
+       : qt == QT_F16 ? 2 : 4;
+}
 
 // Launch plan, computed on the host.
 struct GemvPlan {
@@ -142,6 +171,7 @@ struct XFix {
   uint32_t l0[16], l1[16], l2[16];  // block b, word k (columns 4k..4k+3) at [8b + k]
   float xs[2];                      // 2^(e_b - 22)
   int c0[2], c1[2], c2[2];          // -8 * sum of the block's limb bytes (Q4_0)
+  float sx[2];                      // sum of the block's x values (Q4_K / Q5_K: the min term)
 };
 
 __device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
@@ -223,6 +253,130 @@ __device__ __forceinline__ float rowfix_q4_0(const uint8_t* seg, int lane, const
   }
   return r;
 }
+
+// Q4_K / Q5_K rows: a slice is 8 super-blocks; lane l owns super-block
+// sb = l / 4 and its 64-element chunk c = l % 4, i.e. the slice columns
+// 64 l .. 64 l + 63 as for Q8_0: sub-block 2c (low nibbles of the chunk's 32
+// code bytes, x words 0..7) and sub-block 2c + 1 (high nibbles, x words
+// 8..15).  Every super-block starts 16-byte aligned (144 / 176 bytes), so the
+// header (d, dmin, 12 scale bytes) and the codes come in as 16-byte loads.
+// With A_b the exact integer sum of code x limb products of sub-block b and
+// X_b the sum of its fixed-point x, the lane's share of the row is
+//   sum_b 2^(e_b-22) (d sc_b A_b - dmin m_b X_b).
+// The 6-bit scale and min of sub-block j: j < 4 from the low six bits of
+// scale bytes j and j + 4; j >= 4 from the nibbles of byte j + 4 and the top
+// two bits of bytes j - 4 (scale) and j (min) -- chosen without branches
+// since c varies across the warp.
+__device__ __forceinline__ void kq_scale_min(uint32_t s0, uint32_t s1, uint32_t s2, int c, int t, float& sc,
+                                             float& mn) {
+  const uint32_t sh = 8u * (uint32_t)((2 * c + t) & 3);
+  const uint32_t b0 = (s0 >> sh) & 0xFFu, b1 = (s1 >> sh) & 0xFFu, b2 = (s2 >> sh) & 0xFFu;
+  const uint32_t lo_sc = b0 & 63u, lo_m = b1 & 63u;
+  const uint32_t hi_sc = (b2 & 15u) | ((b0 >> 6) << 4), hi_m = (b2 >> 4) | ((b1 >> 6) << 4);
+  sc = (float)(c < 2 ? lo_sc : hi_sc);
+  mn = (float)(c < 2 ? lo_m : hi_m);
+}
+
+template <bool FIVE>
+__device__ __forceinline__ float rowfix_kq(const uint8_t* seg, int lane, const XFix& x) {
+  const int sb = lane >> 2, c = lane & 3;
+  const uint8_t* blk = seg + (FIVE ? 176 : 144) * sb;
+  const uint4 hdr = *reinterpret_cast<const uint4*>(blk);
+  const uint4* qp = reinterpret_cast<const uint4*>(blk + (FIVE ? 48 : 16) + 32 * c);
+  const uint4 qa = qp[0], qb = qp[1];
+  const uint32_t qs[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+  uint32_t qh[8];
+  if constexpr (FIVE) {
+    const uint4* hp = reinterpret_cast<const uint4*>(blk + 16);
+    const uint4 ha = hp[0], hb = hp[1];
+    qh[0] = ha.x; qh[1] = ha.y; qh[2] = ha.z; qh[3] = ha.w;
+    qh[4] = hb.x; qh[5] = hb.y; qh[6] = hb.z; qh[7] = hb.w;
+  }
+  int a0 = 0, a1 = 0, a2 = 0, b0 = 0, b1 = 0, b2 = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t lo = qs[k] & 0x0F0F0F0Fu, hi = (qs[k] >> 4) & 0x0F0F0F0Fu;
+    if constexpr (FIVE) {
+      lo |= ((qh[k] >> (2 * c)) & 0x01010101u) << 4;
+      hi |= ((qh[k] >> (2 * c + 1)) & 0x01010101u) << 4;
+    }
+    a0 = dp4a_uu(lo, x.l0[k], a0);
+    a1 = dp4a_uu(lo, x.l1[k], a1);
+    a2 = dp4a_us(lo, x.l2[k], a2);
+    b0 = dp4a_uu(hi, x.l0[8 + k], b0);
+    b1 = dp4a_uu(hi, x.l1[8 + k], b1);
+    b2 = dp4a_us(hi, x.l2[8 + k], b2);
+  }
+  const float d = half_bits_to_float(hdr.x), dmin = half_bits_to_float(hdr.x >> 16);
+  float sca, mna, scb, mnb;
+  kq_scale_min(hdr.y, hdr.z, hdr.w, c, 0, sca, mna);
+  kq_scale_min(hdr.y, hdr.z, hdr.w, c, 1, scb, mnb);
+  const float ta = (d * sca) * x.xs[0], tb = (d * scb) * x.xs[1];
+  float r = fmaf(ta, limbs_to_f(a0, a1, a2), tb * limbs_to_f(b0, b1, b2));
+  return fmaf(-dmin, fmaf(mna, x.sx[0], mnb * x.sx[1]), r);
+}
+
+// F16 / F32 rows: x stays fp32 in the lane's registers.  F16: lane l owns the
+// slice columns 8 l + 256 i + t (i < 8, t < 8), one 16-byte load per i;
+// F32: columns 4 l + 128 i + t (i < 16, t < 4).  Consecutive lanes read
+// consecutive 16 bytes, so the loads are free of bank conflicts.  ni = the
+// slice's valid 16-byte groups per lane (K a multiple of 256).
+template <int QT>
+struct XFloat {
+  float v[64];
+  int ni;
+  template <class Pro>
+  __device__ __forceinline__ void load_direct(const Pro& pro, int64_t c0, int ucols, int lane) {
+    constexpr int W = QT == QT_F16 ? 8 : 4;   // columns per 16-byte group
+    constexpr int STEP = 32 * W;              // columns between a lane's groups
+    ni = ucols / STEP;
+#pragma unroll
+    for (int i = 0; i < 64 / W; ++i) {
+      if (i < ni) {
+#pragma unroll
+        for (int q = 0; q < W / 4; ++q) {
+          const float4 f = pro.ld(c0 + (int64_t)STEP * i + W * lane + 4 * q);
+          v[W * i + 4 * q + 0] = f.x;
+          v[W * i + 4 * q + 1] = f.y;
+          v[W * i + 4 * q + 2] = f.z;
+          v[W * i + 4 * q + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < W; ++t) v[W * i + t] = 0.f;
+      }
+    }
+  }
+  __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const {
+    float r0 = 0.f, r1 = 0.f;
+    if constexpr (QT == QT_F16) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i < ni) {
+          const uint4 w = *reinterpret_cast<const uint4*>(seg + 512 * i + 16 * lane);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            r0 = fmaf(half_bits_to_float(ww[k]), v[8 * i + 2 * k], r0);
+            r1 = fmaf(half_bits_to_float(ww[k] >> 16), v[8 * i + 2 * k + 1], r1);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i < ni) {
+          const float4 w = *reinterpret_cast<const float4*>(seg + 512 * i + 16 * lane);
+          r0 = fmaf(w.x, v[4 * i + 0], r0);
+          r1 = fmaf(w.y, v[4 * i + 1], r1);
+          r0 = fmaf(w.z, v[4 * i + 2], r0);
+          r1 = fmaf(w.w, v[4 * i + 3], r1);
+        }
+      }
+    }
+    return r0 + r1;
+  }
+};
 
 // Q6_K: a slice is 8 super-blocks (1680 bytes).  Lane l owns super-block
 // sb = l >> 2, half h = (l >> 1) & 1 and run r16 = l & 1: the elements
@@ -360,6 +514,7 @@ __device__ __forceinline__ void fix6_direct(const Pro& pro, int64_t c0, int lane
 template <int QT>
 __device__ __forceinline__ bool lane_active(int lane, int ucols) {
   if constexpr (QT == QT_Q6_K) return ucols == kSliceCols;  // Q6_K slices are always whole
+  else if constexpr (qt_float(QT)) return ucols > 0;        // per-group bounds inside the lane
   else return 2 * lane < ucols / 32;
 }
 
@@ -458,6 +613,13 @@ __device__ __forceinline__ void stage_chunk(const float4 v, int64_t col, const X
   xs.wd[16 * xs.np + wi] = w1;
   xs.wd[32 * xs.np + wi] = w2;
   const int64_t B = col / 32;
+  if constexpr (qt_kmin(QT)) {
+    // the block's sum of fixed-point x (|sum| < 2^27): the min term's weight
+    s0 = group8_sum(s0);
+    s1 = group8_sum(s1);
+    s2 = group8_sum(s2);
+    if ((lane & 7) == 0) xs.cr[3 * B] = s0 + 256 * s1 + 65536 * s2;
+  }
   if constexpr (QT == QT_Q4_0) {
     s0 = group8_sum(s0);
     s1 = group8_sum(s1);
@@ -528,12 +690,33 @@ struct XRegs {
         x.c1[b] = xs.cr[3 * B + 1];
         x.c2[b] = xs.cr[3 * B + 2];
       }
+      if constexpr (qt_kmin(QT)) x.sx[b] = (float)xs.cr[3 * B] * x.xs[b];
     }
   }
   __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const {
     if constexpr (QT == QT_Q8_0) return rowfix_q8_0(seg, lane, x);
+    else if constexpr (QT == QT_Q4_K) return rowfix_kq<false>(seg, lane, x);
+    else if constexpr (QT == QT_Q5_K) return rowfix_kq<true>(seg, lane, x);
     else return rowfix_q4_0(seg, lane, x);
   }
+};
+template <>
+struct XRegs<QT_F16> {
+  XFloat<QT_F16> x;
+  template <class Pro>
+  __device__ __forceinline__ void load_direct(const Pro& pro, int64_t c0, int ucols, int lane) {
+    x.load_direct(pro, c0, ucols, lane);
+  }
+  __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const { return x.dot(seg, lane); }
+};
+template <>
+struct XRegs<QT_F32> {
+  XFloat<QT_F32> x;
+  template <class Pro>
+  __device__ __forceinline__ void load_direct(const Pro& pro, int64_t c0, int ucols, int lane) {
+    x.load_direct(pro, c0, ucols, lane);
+  }
+  __device__ __forceinline__ float dot(const uint8_t* seg, int lane) const { return x.dot(seg, lane); }
 };
 template <>
 struct XRegs<QT_Q6_K> {
@@ -846,11 +1029,15 @@ __global__ void __launch_bounds__((MAXC + 1) * 32, MAXC <= 8 ? 2 : 1)
     const int ucols = (int)min64(kSliceCols, K - c0);
     const bool active = lane_active<QT>(lane, ucols);
     pro.setup(lane);
-    const XStage xs = xstage_at(xstage_base, K);
-    stage_x<QT>(pro, K, xs, warp, p.NW, lane);
-    asm volatile("bar.sync 1, %0;" ::"r"(p.NW * 32) : "memory");  // consumer warps only
     XRegs<QT> xr;
-    if (active) xr.load(xs, c, lane);
+    if constexpr (qt_float(QT)) {
+      if (active) xr.load_direct(pro, c0, ucols, lane);  // fp32 x straight into registers
+    } else {
+      const XStage xs = xstage_at(xstage_base, K);
+      stage_x<QT>(pro, K, xs, warp, p.NW, lane);
+      asm volatile("bar.sync 1, %0;" ::"r"(p.NW * 32) : "memory");  // consumer warps only
+      if (active) xr.load(xs, c, lane);
+    }
     int s = 0;
     uint32_t ph = 0;
     for (int i = 0; i < n_stages; ++i) {
@@ -879,7 +1066,7 @@ __global__ void __launch_bounds__((MAXC + 1) * 32, MAXC <= 8 ? 2 : 1)
 // bytes for the ring; align: 1 or 2 (rows per epilogue unit).
 inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget, int max_consumers) {
   GemvPlan p;
-  const int be = qtype == QT_Q6_K ? 256 : 32, bb = qtype == QT_Q6_K ? 210 : (qtype == QT_Q8_0 ? 34 : 18);
+  const int be = qt_block_elems(qtype), bb = qt_block_bytes(qtype);
   p.row_bytes = (int)(K / be * bb);
   p.n_slices = (int)((K + kSliceCols - 1) / kSliceCols);
   int trmax = kStageTarget / p.row_bytes;
@@ -900,7 +1087,7 @@ inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget,
   p.n_rg = n_rg;
   p.NW = p.n_slices * n_rg;
   p.stage_bytes = p.TR * p.row_bytes;
-  p.xstage_bytes = (int)((xstage_bytes(qtype, K) + 15) / 16 * 16);
+  p.xstage_bytes = qt_float(qtype) ? 0 : (int)((xstage_bytes(qtype, K) + 15) / 16 * 16);
   int S = smem_budget / p.stage_bytes;
   if (S > 8) S = 8;
   if (S < 2) S = 2;
@@ -919,7 +1106,30 @@ inline size_t gemv_smem_bytes(const GemvPlan& p) {
 // the bulk-copy path cannot take.
 template <int QT>
 __device__ __forceinline__ float block_dot_generic(const uint8_t* blk, const float* x) {
-  if constexpr (QT == QT_Q8_0) {
+  if constexpr (qt_kmin(QT)) {
+    const float d = half_bits_to_float(blk[0] | (blk[1] << 8)), dmin = half_bits_to_float(blk[2] | (blk[3] << 8));
+    const uint8_t* p = blk + 4;
+    float s = 0.f;
+    for (int j = 0; j < 8; ++j) {
+      const int sc = j < 4 ? (p[j] & 63) : ((p[j + 4] & 15) | ((p[j - 4] >> 6) << 4));
+      const int mn = j < 4 ? (p[j + 4] & 63) : ((p[j + 4] >> 4) | ((p[j] >> 6) << 4));
+      float t = 0.f, sx = 0.f;
+      for (int i = 0; i < 32; ++i) {
+        const int n = 32 * j + i, c = n >> 6, h = (n >> 5) & 1, l = n & 31;
+        int q = (blk[(QT == QT_Q5_K ? 48 : 16) + 32 * c + l] >> (4 * h)) & 15;
+        if constexpr (QT == QT_Q5_K) q |= ((blk[16 + l] >> (2 * c + h)) & 1) << 4;
+        t = fmaf((float)q, x[n], t);
+        sx += x[n];
+      }
+      s = fmaf(d * (float)sc, t, s);
+      s = fmaf(-dmin * (float)mn, sx, s);
+    }
+    return s;
+  } else if constexpr (QT == QT_F16) {
+    return half_bits_to_float(blk[0] | (blk[1] << 8)) * x[0];
+  } else if constexpr (QT == QT_F32) {
+    return __uint_as_float(blk[0] | (blk[1] << 8) | (blk[2] << 16) | ((uint32_t)blk[3] << 24)) * x[0];
+  } else if constexpr (QT == QT_Q8_0) {
     const float d = half_bits_to_float(blk[0] | (blk[1] << 8));
     float s = 0.f;
     for (int i = 0; i < 32; ++i) s = fmaf((float)(int8_t)blk[2 + i], x[i], s);

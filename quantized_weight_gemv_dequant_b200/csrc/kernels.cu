@@ -1,5 +1,6 @@
 // kernels.cu -- instantiation and launch of every libntx kernel (sm_100a).
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "attn.cuh"
@@ -103,7 +104,7 @@ cudaError_t gemv_tma_v(Map map, Pro pro, Epi epi, int64_t M, int64_t K, int grid
   static unsigned long long done = 0;  // unique per instantiation
   auto kern = gemv_tma_kernel<QT, Map, Pro, Epi, MAXC>;
   // the ring gives up what x staging needs beyond the per-CTA ceiling
-  const int xst = (int)((xstage_bytes(QT, K) + 15) / 16 * 16);
+  const int xst = qt_float(QT) ? 0 : (int)((xstage_bytes(QT, K) + 15) / 16 * 16);
   if (ring > kSmemMax - 8192 - xst) ring = kSmemMax - 8192 - xst;
   const GemvPlan plan = make_gemv_plan(QT, K, Epi::kAlign, ring, MAXC);
   const size_t smem = gemv_smem_bytes(plan);
@@ -122,6 +123,22 @@ cudaError_t gemv_tma(Map map, Pro pro, Epi epi, int64_t M, int64_t K, int grid, 
       return gemv_tma_v<QT, kPairedConsumers>(map, pro, epi, M, K, grid, s, pdl, kRingBudgetPaired);
   }
   return gemv_tma_v<QT, kMaxConsumers>(map, pro, epi, M, K, grid, s, pdl, kRingBudget);
+}
+
+// Calls f(std::integral_constant<int, QT>) for the block type qt (any type the
+// GEMV kernels take); cudaErrorInvalidValue for others.
+template <class F>
+cudaError_t with_qt(int qt, F&& f) {
+  switch (qt) {
+    case QT_Q8_0: return f(std::integral_constant<int, QT_Q8_0>{});
+    case QT_Q4_0: return f(std::integral_constant<int, QT_Q4_0>{});
+    case QT_Q6_K: return f(std::integral_constant<int, QT_Q6_K>{});
+    case QT_Q4_K: return f(std::integral_constant<int, QT_Q4_K>{});
+    case QT_Q5_K: return f(std::integral_constant<int, QT_Q5_K>{});
+    case QT_F16: return f(std::integral_constant<int, QT_F16>{});
+    case QT_F32: return f(std::integral_constant<int, QT_F32>{});
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
@@ -159,19 +176,23 @@ int attn_splits(int n_kv_heads, int n_ctx) {
 
 bool gemv_tma_ok(int qtype, const void* W, int64_t K) {
   if ((reinterpret_cast<uintptr_t>(W) & 15) != 0) return false;
-  if (qtype == QT_Q8_0 || qtype == QT_Q4_0) return K % 256 == 0 && K <= (int64_t)kMaxConsumers * kSliceCols;
-  if (qtype == QT_Q6_K) return K % 2048 == 0 && K <= (int64_t)kMaxConsumers * kSliceCols;
+  if (K > (int64_t)kMaxConsumers * kSliceCols) return false;
+  if (qtype == QT_Q6_K) return K % 2048 == 0;
+  if (qtype == QT_Q8_0 || qtype == QT_Q4_0 || qtype == QT_Q4_K || qtype == QT_Q5_K || qtype == QT_F16 ||
+      qtype == QT_F32)
+    return K % 256 == 0;
   return false;
 }
 
 cudaError_t launch_dequant(int qtype, const void* blocks, float* out, int64_t nblocks, cudaStream_t s) {
   if (nblocks <= 0) return cudaSuccess;
-  const int g = grid_1d(nblocks, 128, sm_count() * 16);
   const uint8_t* b = static_cast<const uint8_t*>(blocks);
-  if (qtype == QT_Q8_0) dequant_kernel<QT_Q8_0><<<g, 128, 0, s>>>(b, out, nblocks);
-  else if (qtype == QT_Q4_0) dequant_kernel<QT_Q4_0><<<g, 128, 0, s>>>(b, out, nblocks);
-  else dequant_kernel<QT_Q6_K><<<g, 128, 0, s>>>(b, out, nblocks);
-  return cudaGetLastError();
+  return with_qt(qtype, [&](auto t) {
+    constexpr int QT = decltype(t)::value;
+    const int g = grid_1d(nblocks, 128, sm_count() * 16);
+    dequant_kernel<QT><<<g, 128, 0, s>>>(b, out, nblocks);
+    return cudaGetLastError();
+  });
 }
 
 template <int QT>
@@ -190,9 +211,9 @@ static cudaError_t gemv_plain_qt(const void* W, int64_t M, int64_t K, const floa
 
 cudaError_t launch_gemv(int qtype, const void* W, int64_t M, int64_t K, const float* x, float* y, const float* resid,
                         cudaStream_t s, bool pdl) {
-  if (qtype == QT_Q8_0) return gemv_plain_qt<QT_Q8_0>(W, M, K, x, y, resid, s, pdl);
-  if (qtype == QT_Q4_0) return gemv_plain_qt<QT_Q4_0>(W, M, K, x, y, resid, s, pdl);
-  return gemv_plain_qt<QT_Q6_K>(W, M, K, x, y, resid, s, pdl);
+  return with_qt(qtype, [&](auto t) {
+    return gemv_plain_qt<decltype(t)::value>(W, M, K, x, y, resid, s, pdl);
+  });
 }
 
 cudaError_t launch_rmsnorm(const float* x, const float* w, float* y, int64_t n, float eps, cudaStream_t s) {
@@ -299,22 +320,26 @@ cudaError_t launch_attn_cluster(const float* q, const uint16_t* kc, const uint16
 int layer_stats_parts(int64_t H) { return gemv_grid(H, 1); }
 
 template <int QT>
-static cudaError_t layer_qt(const LayerArgs& a, cudaStream_t s, bool pdl) {
-  using T = QTraits<QT>;
-  const int64_t rbH = a.H / T::BE * T::BB;  // rows with K = H
-  const int64_t rbQ = a.Hq * a.D / T::BE * T::BB;  // K = Hq*D
-  const int64_t rbF = a.F / T::BE * T::BB;  // K = F
+constexpr int64_t row_bytes_of(int64_t K) {
+  return K / QTraits<QT>::BE * QTraits<QT>::BB;
+}
+
+// One decode layer as a chain of kernels; each GEMV takes its own block type
+// (Q/K/V share one, gate/up share one).
+cudaError_t launch_layer(const LayerArgs& a, cudaStream_t s, bool pdl) {
   const int64_t nq = a.Hq * a.D, nkv = a.Hkv * a.D;
   cudaError_t e;
 
   // 1. RMSNorm prologue + Q/K/V GEMV + RoPE + KV append
-  {
+  e = with_qt(a.qt_qkv, [&](auto t) {
+    constexpr int QT = decltype(t)::value;
     ProRms pro{a.hidden, a.attn_norm, a.stats_in, a.n_stats_in, (int)a.H, a.eps, 0.f};
     EpiQKV epi{a.q, a.k_cache, a.v_cache, a.pos_dev, a.pos, nq, nkv, (int)a.D, a.max_ctx, a.theta};
     const int64_t M = nq + 2 * nkv;
-    e = gemv_tma<QT>(MapQKV{a.wq, a.wk, a.wv, rbH, nq, nkv}, pro, epi, M, a.H, gemv_grid(M, 2), s, pdl);
-    if (e != cudaSuccess) return e;
-  }
+    return gemv_tma<QT>(MapQKV{a.wq, a.wk, a.wv, row_bytes_of<QT>(a.H), nq, nkv}, pro, epi, M, a.H,
+                        gemv_grid(M, 2), s, pdl);
+  });
+  if (e != cudaSuccess) return e;
   // 2. split-KV attention: one cluster per KV head (partials merged through
   //    distributed shared memory), or split + combine kernels for long contexts
   if (a.attn_cluster > 0)
@@ -325,32 +350,31 @@ static cudaError_t layer_qt(const LayerArgs& a, cudaStream_t s, bool pdl) {
                     a.max_ctx, a.n_split, s, pdl);
   if (e != cudaSuccess) return e;
   // 3. O projection + residual: h1 = h + Wo a   (statistics: sum h1^2)
-  {
+  e = with_qt(a.qt_o, [&](auto t) {
+    constexpr int QT = decltype(t)::value;
     EpiResid epi{a.h1, a.hidden, nullptr, a.stats_o, 0.f, 0.f, 0.f};
-    e = gemv_tma<QT>(MapSingle{a.wo, rbQ}, ProPlain{a.attn_out}, epi, a.H, nq, gemv_grid(a.H, 1), s, pdl);
-    if (e != cudaSuccess) return e;
-  }
+    return gemv_tma<QT>(MapSingle{a.wo, row_bytes_of<QT>(nq)}, ProPlain{a.attn_out}, epi, a.H, nq,
+                        gemv_grid(a.H, 1), s, pdl);
+  });
+  if (e != cudaSuccess) return e;
   // 4. RMSNorm prologue + gate/up GEMV + SwiGLU
-  {
+  if (a.probe_begin && (e = cudaEventRecord(a.probe_begin, s)) != cudaSuccess) return e;
+  e = with_qt(a.qt_gu, [&](auto t) {
+    constexpr int QT = decltype(t)::value;
     ProRms pro{a.h1, a.ffn_norm, a.stats_o, gemv_grid(a.H, 1), (int)a.H, a.eps, 0.f};
     EpiSwiGLU epi{a.u};
-    if (a.probe_begin && (e = cudaEventRecord(a.probe_begin, s)) != cudaSuccess) return e;
-    e = gemv_tma<QT>(MapPair{a.wg, a.wu, rbH}, pro, epi, 2 * a.F, a.H, gemv_grid(2 * a.F, 2), s, pdl);
-    if (e != cudaSuccess) return e;
-    if (a.probe_end && (e = cudaEventRecord(a.probe_end, s)) != cudaSuccess) return e;
-  }
+    return gemv_tma<QT>(MapPair{a.wg, a.wu, row_bytes_of<QT>(a.H)}, pro, epi, 2 * a.F, a.H,
+                        gemv_grid(2 * a.F, 2), s, pdl);
+  });
+  if (e != cudaSuccess) return e;
+  if (a.probe_end && (e = cudaEventRecord(a.probe_end, s)) != cudaSuccess) return e;
   // 5. down projection + residual + cosine statistics: h = h1 + Wd u
-  {
+  return with_qt(a.qt_down, [&](auto t) {
+    constexpr int QT = decltype(t)::value;
     EpiResid epi{a.hidden, a.h1, a.hidden, a.stats_down, 0.f, 0.f, 0.f};
-    e = gemv_tma<QT>(MapSingle{a.wd, rbF}, ProPlain{a.u}, epi, a.H, a.F, gemv_grid(a.H, 1), s, pdl);
-  }
-  return e;
-}
-
-cudaError_t launch_layer(const LayerArgs& a, cudaStream_t s, bool pdl) {
-  if (a.qtype == QT_Q8_0) return layer_qt<QT_Q8_0>(a, s, pdl);
-  if (a.qtype == QT_Q4_0) return layer_qt<QT_Q4_0>(a, s, pdl);
-  return layer_qt<QT_Q6_K>(a, s, pdl);
+    return gemv_tma<QT>(MapSingle{a.wd, row_bytes_of<QT>(a.F)}, ProPlain{a.u}, epi, a.H, a.F, gemv_grid(a.H, 1), s,
+                        pdl);
+  });
 }
 
 cudaError_t launch_sumsq(const float* h, int64_t n, float* parts, int nparts, cudaStream_t s, bool pdl) {
@@ -365,23 +389,16 @@ cudaError_t launch_embed(const uint16_t* table, int64_t H, int64_t V, const int*
 
 int head_parts(int64_t V) { return gemv_grid(V, 1); }
 
-template <int QT>
-static cudaError_t head_qt(const void* W, int64_t V, int64_t H, const float* h, const float* final_norm,
-                           const float* stats_in, int n_stats_in, float eps, float* logits, float* arg_parts,
-                           cudaStream_t s, bool pdl) {
-  using T = QTraits<QT>;
-  ProRms pro{h, final_norm, stats_in, n_stats_in, (int)H, eps, 0.f};
-  EpiArgmax epi{logits, arg_parts, 0.f, 0};
-  return gemv_tma<QT>(MapSingle{static_cast<const uint8_t*>(W), H / T::BE * T::BB}, pro, epi, V, H, gemv_grid(V, 1),
-                      s, pdl);
-}
-
 cudaError_t launch_head(int qtype, const void* W, int64_t V, int64_t H, const float* h, const float* final_norm,
                         const float* stats_in, int n_stats_in, float eps, float* logits, float* arg_parts,
                         cudaStream_t s, bool pdl) {
-  if (qtype == QT_Q8_0) return head_qt<QT_Q8_0>(W, V, H, h, final_norm, stats_in, n_stats_in, eps, logits, arg_parts, s, pdl);
-  if (qtype == QT_Q4_0) return head_qt<QT_Q4_0>(W, V, H, h, final_norm, stats_in, n_stats_in, eps, logits, arg_parts, s, pdl);
-  return head_qt<QT_Q6_K>(W, V, H, h, final_norm, stats_in, n_stats_in, eps, logits, arg_parts, s, pdl);
+  return with_qt(qtype, [&](auto t) {
+    constexpr int QT = decltype(t)::value;
+    ProRms pro{h, final_norm, stats_in, n_stats_in, (int)H, eps, 0.f};
+    EpiArgmax epi{logits, arg_parts, 0.f, 0};
+    return gemv_tma<QT>(MapSingle{static_cast<const uint8_t*>(W), row_bytes_of<QT>(H)}, pro, epi, V, H,
+                        gemv_grid(V, 1), s, pdl);
+  });
 }
 
 cudaError_t launch_argmax_finalize(const float* parts, int nparts, int* token_state, int* next_token, cudaStream_t s,

@@ -30,7 +30,7 @@ cudaError_t launch_attn(const float* q, const uint16_t* kc, const uint16_t* vc, 
 
 // The pieces of one fused decode layer.
 struct LayerArgs {
-  int qtype;
+  int qt_qkv, qt_o, qt_gu, qt_down;  // block types of wq/wk/wv, wo, wg/wu, wd
   int64_t H, Hq, Hkv, D, F;
   int max_ctx;
   float eps, theta;

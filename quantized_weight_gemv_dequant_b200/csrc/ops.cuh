@@ -9,14 +9,35 @@
 namespace ntx {
 
 // ------------------------------------------------------------- dequant
-// One thread per block; exact (d * sc * (q - off) fits fp32).
+// One thread per block.  Q8_0, Q4_0, Q6_K: exact (d * sc * (q - off) fits
+// fp32).  Q4_K / Q5_K: d sc q and dmin m are each exact, their difference is
+// rounded once (fp32 round to nearest) -- the exact value when it fits fp32.
+// F16 / F32: the value.
 template <int QT>
 __global__ void dequant_kernel(const uint8_t* __restrict__ blocks, float* __restrict__ out, int64_t nblocks) {
   using T = QTraits<QT>;
   for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblocks; b += (int64_t)gridDim.x * blockDim.x) {
     const uint8_t* p = blocks + b * T::BB;
     float* o = out + b * T::BE;
-    if constexpr (QT == QT_Q8_0) {
+    if constexpr (qt_kmin(QT)) {
+      const float d = half_bits_to_float(p[0] | (p[1] << 8)), dmin = half_bits_to_float(p[2] | (p[3] << 8));
+      const uint8_t* sc = p + 4;
+      for (int j = 0; j < 8; ++j) {
+        const int s = j < 4 ? (sc[j] & 63) : ((sc[j + 4] & 15) | ((sc[j - 4] >> 6) << 4));
+        const int m = j < 4 ? (sc[j + 4] & 63) : ((sc[j + 4] >> 4) | ((sc[j] >> 6) << 4));
+        const float ds = d * (float)s, dm = dmin * (float)m;  // both exact
+        for (int i = 0; i < 32; ++i) {
+          const int n = 32 * j + i, c = n >> 6, h = (n >> 5) & 1, l = n & 31;
+          int q = (p[(QT == QT_Q5_K ? 48 : 16) + 32 * c + l] >> (4 * h)) & 15;
+          if constexpr (QT == QT_Q5_K) q |= ((p[16 + l] >> (2 * c + h)) & 1) << 4;
+          o[n] = __fmaf_rn(ds, (float)q, -dm);  // one rounding of the exact d sc q - dmin m
+        }
+      }
+    } else if constexpr (QT == QT_F16) {
+      o[0] = half_bits_to_float(p[0] | (p[1] << 8));
+    } else if constexpr (QT == QT_F32) {
+      o[0] = __uint_as_float(p[0] | (p[1] << 8) | (p[2] << 16) | ((uint32_t)p[3] << 24));
+    } else if constexpr (QT == QT_Q8_0) {
       const float d = half_bits_to_float(p[0] | (p[1] << 8));
       for (int i = 0; i < 32; ++i) o[i] = d * (float)(int8_t)p[2 + i];
     } else if constexpr (QT == QT_Q4_0) {

@@ -1236,6 +1236,7 @@ std::mutex g_pmu;
 int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int max_ctx, int grid, int n_layers,
                  PStep* st, size_t* smem) {
   (void)V;
+  if (qtype != QT_Q8_0 && qtype != QT_Q4_0 && qtype != QT_Q6_K) return -1;
   if (D != kPD) return -1;
   if (Hkv <= 0 || Hq % Hkv) return -1;
   const int Gq = Hq / Hkv;

@@ -169,3 +169,41 @@ def test_static_attention_refuses_oversize_before_any_cuda_call():
     assert _rc(ntx.ntx_attn_decode_static, *args, 64, 8, 64, 100, 100) == ntx.NTX_ERR_SHAPE
     assert _rc(ntx.ntx_attn_decode_static, None, *args[1:], 64, 8, 128, 100, 100) == ntx.NTX_ERR_INVALID_ARG
     assert _rc(ntx.ntx_attn_decode_static, FAKE + 4, *args[1:], 64, 8, 128, 100, 100) == ntx.NTX_ERR_ALIGN
+
+
+def test_mixed_layer_layout_and_type_rules():
+    d = dict(hidden=2048, n_heads=16, n_kv_heads=4, head_dim=128, ffn=4096, vocab=1000, n_layers=1, eps=1e-5,
+             theta=500000.0)
+    cfg = _cfg(d, max_ctx=16, layers=1)
+    q4km = wl.Q4_K_M
+    n, w = ntx.ntx_layer_layout_mixed(cfg, q4km)
+    n2, offs = wl.layer_layout(d, q4km)
+    assert n == n2 and w.qtype == ntx.NTX_MIXED and list(w.mat_qtype) == list(q4km)
+    for k in wl.MATS + ("attn_norm", "ffn_norm"):
+        assert getattr(w, "off_" + k) == offs[k]
+    # one type: the same offsets as the uniform call
+    n3, w3 = ntx.ntx_layer_layout(cfg, ntx.NTX_Q4_K)
+    n4, w4 = ntx.ntx_layer_layout_mixed(cfg, [ntx.NTX_Q4_K] * 7)
+    assert n3 == n4 and w3.qtype == ntx.NTX_Q4_K and w4.qtype == ntx.NTX_MIXED
+    # wq, wk, wv (and wg, wu) are one fused GEMV each: one type per group
+    ws = ntx.ntx_layer_workspace_bytes(cfg)
+    for bad in ((12, 12, 14, 12, 12, 12, 14), (12, 12, 12, 12, 12, 13, 14)):
+        _, wb = ntx.ntx_layer_layout_mixed(cfg, bad)
+        wb.base = FAKE
+        assert _rc(ntx.ntx_decode_layer, cfg, wb, FAKE, FAKE, FAKE, 0, None, FAKE, ws) == ntx.NTX_ERR_QTYPE
+    # Q6_K needs input lengths that are multiples of 2048
+    small = ntx.make_config(1024, 8, 2, 128, 3072, 1000, 1, 1e-5, 5e5, 16)
+    _, wq6 = ntx.ntx_layer_layout(small, ntx.NTX_Q6_K)
+    wq6.base = FAKE
+    assert _rc(ntx.ntx_decode_layer, small, wq6, FAKE, FAKE, FAKE, 0, None, FAKE,
+               ntx.ntx_layer_workspace_bytes(small)) == ntx.NTX_ERR_SHAPE
+    with pytest.raises(ntx.NtxError):
+        ntx.ntx_layer_layout_mixed(cfg, [99] * 7)
+
+
+def test_new_formats_argument_checks():
+    for qt in (ntx.NTX_Q4_K, ntx.NTX_Q5_K):
+        assert _rc(ntx.ntx_gemv_q, qt, FAKE, 16, 128, FAKE + 0x100000, FAKE + 0x200000) == ntx.NTX_ERR_SHAPE
+        assert _rc(ntx.ntx_dequant, qt, FAKE, FAKE + 0x1000, 255) == ntx.NTX_ERR_SHAPE
+    assert _rc(ntx.ntx_gemv_q, ntx.NTX_MIXED, FAKE, 16, 256, FAKE + 0x100000, FAKE + 0x200000) == ntx.NTX_ERR_QTYPE
+    assert _rc(ntx.ntx_dequant, 3, FAKE, FAKE + 0x1000, 256) == ntx.NTX_ERR_QTYPE

@@ -57,7 +57,8 @@ class Engine:
         tmap = list(m.tier_map) if tier_map is None else list(tier_map)
         layers = []
         for l in range(d["n_layers"]):
-            _, lw = ntx.ntx_layer_layout(self.cfg, m.qtype)
+            _, lw = (ntx.ntx_layer_layout_mixed(self.cfg, m.qtype) if isinstance(m.qtype, (list, tuple))
+                     else ntx.ntx_layer_layout(self.cfg, m.qtype))
             src = m.resident_copy[l] if (use_resident_copy or tmap[l] == 0) else m.layers[l]
             lw.base = src.data_ptr()
             layers.append(lw)
