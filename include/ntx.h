@@ -341,6 +341,39 @@ NTX_API int ntx_engine_launches_per_step(ntx_engine* e);
 NTX_API int ntx_persistent_plan(const ntx_model_config* cfg, int qtype, int* slot_bytes, int* n_slots,
                                 size_t* smem_bytes, int* rows_per_slot);
 
+/* ------------------------------------------------------------ tier sizing
+ * Automatic tier sizing ([README] 3-Tier: tier sizes computed from
+ * cudaMemGetInfo() and /proc/meminfo; [ShowHN] 3層アダプティブキャッシュ詳細:
+ * VRAM resident > pinned RAM > NVMe/mmap).  The NVMe / mmap tier is not
+ * provided here: a model that does not fit the first two is refused. */
+
+/* Device bytes an engine for cfg keeps besides the layer blobs and slots:
+ * fp16 embedding table, final norm, the head (head_qtype), the fp16 KV caches
+ * of all layers, and the engine workspace.  0 on bad arguments.  Host only. */
+NTX_API uint64_t ntx_engine_device_bytes(const ntx_model_config* cfg, int head_qtype);
+
+/* Tier map for cfg->n_layers layers of layer_bytes each (the blob size from
+ * ntx_layer_layout), placed in execution order: the first n resident
+ * (tier_map[l] = 0), the rest in pinned host memory (1), n the largest count
+ * for which n blobs + two device slots of layer_bytes (when n < L) +
+ * ntx_engine_device_bytes(cfg, head_qtype) fit in device_free -
+ * device_reserve.  The host layers must fit in host_available - host_reserve.
+ *   tier_map: host int8[L], written on success.  n_resident: host int or NULL.
+ * Errors: NTX_ERR_INVALID_ARG; NTX_ERR_NOMEM when the non-layer buffers or the
+ * two slots do not fit the device, or the streamed layers do not fit the host
+ * (a third tier would be needed).  Host only; no CUDA call. */
+NTX_API int ntx_auto_tier_map(const ntx_model_config* cfg, uint64_t layer_bytes, int head_qtype,
+                              uint64_t device_free, uint64_t device_reserve, uint64_t host_available,
+                              uint64_t host_reserve, int8_t* tier_map, int* n_resident);
+
+/* Memory the tiers can use: *device_free and *device_total from
+ * cudaMemGetInfo on the current device (skipped when both are NULL), and
+ * *host_available = MemAvailable of meminfo_path (NULL: /proc/meminfo), in
+ * bytes.  NTX_ERR_CUDA if the device query fails, NTX_ERR_INVALID_ARG if the
+ * file cannot be read or has no MemAvailable line. */
+NTX_API int ntx_memory_budget(uint64_t* device_free, uint64_t* device_total, uint64_t* host_available,
+                              const char* meminfo_path);
+
 /* Copies the recorded skip set (1 = skipped) into mask_host[L]; returns the
  * number of skipped layers, or a negative error. */
 NTX_API int ntx_engine_skip_mask(ntx_engine* e, uint8_t* mask_host);

@@ -39,7 +39,8 @@ EXPORTS = (
     "ntx_swiglu", "ntx_layer_layout", "ntx_layer_workspace_bytes", "ntx_decode_layer", "ntx_engine_workspace_bytes",
     "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
     "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
-    "ntx_persistent_plan", "ntx_layer_layout_mixed",
+    "ntx_persistent_plan", "ntx_layer_layout_mixed", "ntx_engine_device_bytes", "ntx_auto_tier_map",
+    "ntx_memory_budget",
 )
 
 
@@ -105,6 +106,11 @@ def lib():
             "ntx_attn_decode_static": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp], i32),
             "ntx_engine_set_phase_probe": ([vp, vp, sz], i32),
             "ntx_persistent_plan": ([P(ntx_model_config), i32, P(i32), P(i32), P(sz), P(i32)], i32),
+            "ntx_engine_device_bytes": ([P(ntx_model_config), i32], ctypes.c_uint64),
+            "ntx_auto_tier_map": ([P(ntx_model_config), ctypes.c_uint64, i32, ctypes.c_uint64, ctypes.c_uint64,
+                                   ctypes.c_uint64, ctypes.c_uint64, P(ctypes.c_int8), P(i32)], i32),
+            "ntx_memory_budget": ([P(ctypes.c_uint64), P(ctypes.c_uint64), P(ctypes.c_uint64), ctypes.c_char_p],
+                                  i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -310,3 +316,28 @@ def ntx_engine_launches_per_step(engine) -> int:
     if rc < 0:
         _check(rc)
     return rc
+
+
+# ---------------------------------------------------------------- tier sizing
+def ntx_engine_device_bytes(cfg: ntx_model_config, head_qtype: int) -> int:
+    return int(lib().ntx_engine_device_bytes(ctypes.byref(cfg), head_qtype))
+
+
+def ntx_auto_tier_map(cfg: ntx_model_config, layer_bytes: int, head_qtype: int, device_free: int,
+                      device_reserve: int, host_available: int, host_reserve: int):
+    """Returns (tier_map list of 0/1, number of resident layers)."""
+    n = cfg.n_layers
+    tm = (ctypes.c_int8 * max(n, 1))()
+    nres = ctypes.c_int(0)
+    _check(lib().ntx_auto_tier_map(ctypes.byref(cfg), layer_bytes, head_qtype, device_free, device_reserve,
+                                   host_available, host_reserve, tm, ctypes.byref(nres)))
+    return [int(t) for t in tm[:n]], nres.value
+
+
+def ntx_memory_budget(device=True, meminfo_path=None):
+    """Returns (device_free, device_total, host_available) in bytes; the device
+    figures are None when device is False."""
+    f, t, h = ctypes.c_uint64(0), ctypes.c_uint64(0), ctypes.c_uint64(0)
+    _check(lib().ntx_memory_budget(ctypes.byref(f) if device else None, ctypes.byref(t) if device else None,
+                                   ctypes.byref(h), meminfo_path.encode() if meminfo_path else None))
+    return (f.value if device else None), (t.value if device else None), h.value

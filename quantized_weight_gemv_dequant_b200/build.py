@@ -9,7 +9,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libntx.so")
-SOURCES = ["kernels.cu", "api.cu", "noalloc.cu", "persist.cu"]
+SOURCES = ["kernels.cu", "api.cu", "noalloc.cu", "persist.cu", "tiers.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -523,7 +523,7 @@ cudaError_t persist_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t
   cudaError_t err =
       cudaMemsetAsync(e->psync, 0, sizeof(unsigned) * ntx::persist_sync_words(nrun, c.n_kv_heads), s);
   if (err == cudaSuccess && probe && !e->probe_b.empty()) err = cudaEventRecord(e->probe_b[0], s);
-  if (err == cudaSuccess) err = ntx::launch_persist(e->head_qtype, st,
+  if (err == cudaSuccess) err = ntx::launch_persist(st,
                                                     e->psmem, e->pgrid, s);
   if (err == cudaSuccess && probe && !e->probe_e.empty()) err = cudaEventRecord(e->probe_e[0], s);
   if (err != cudaSuccess) return err;
@@ -710,30 +710,41 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   }
   if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->fork_ev, cudaEventDisableTiming);
   if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->join_ev, cudaEventDisableTiming);
-  // persistent kernel: every layer of the head's block type, shapes and alignment it handles; it runs the
-  // steps whose executed layers are all resident (all steps without a host tier; with one, the steps under a
-  // skip set that skips every host layer)
+  // persistent kernel: each GEMV phase kind (Q/K/V, O, gate/up, down, head) of one block type over all
+  // layers, a type pair it is built for, shapes and alignment it handles; it runs the steps whose executed
+  // layers are all resident (all steps without a host tier; with one, the steps under a skip set that skips
+  // every host layer)
   e->persist = e->persist_full = e->persist_skip = false;
-  bool one_type = head_qtype == NTX_Q8_0 || head_qtype == NTX_Q4_0 || head_qtype == NTX_Q6_K;
-  for (int l = 0; l < cfg->n_layers && one_type; ++l)
-    for (int i = 0; i < 7; ++i) one_type = one_type && mat_qt(&layers[l], i) == head_qtype;
-  if (err == cudaSuccess && one_type) {
+  int kt[7] = {0, 0, 0, 0, 0, 0, 0};
+  kt[ntx::PK_HEAD] = head_qtype;
+  bool uniform = true;
+  if (cfg->n_layers > 0) {
+    kt[ntx::PK_QKV] = mat_qt(&layers[0], 0);
+    kt[ntx::PK_O] = mat_qt(&layers[0], 3);
+    kt[ntx::PK_GU] = mat_qt(&layers[0], 4);
+    kt[ntx::PK_DOWN] = mat_qt(&layers[0], 6);
+  } else {
+    kt[ntx::PK_QKV] = kt[ntx::PK_O] = kt[ntx::PK_GU] = kt[ntx::PK_DOWN] = head_qtype;
+  }
+  for (int l = 1; l < cfg->n_layers && uniform; ++l)
+    uniform = mat_qt(&layers[l], 0) == kt[ntx::PK_QKV] && mat_qt(&layers[l], 3) == kt[ntx::PK_O] &&
+              mat_qt(&layers[l], 4) == kt[ntx::PK_GU] && mat_qt(&layers[l], 6) == kt[ntx::PK_DOWN];
+  if (err == cudaSuccess && uniform) {
     ntx::PStep st;
     memset(&st, 0, sizeof st);
     size_t psm = 0;
-    const int qt = head_qtype;
-    if (ntx::persist_plan(qt, cfg->hidden, cfg->n_heads, cfg->n_kv_heads, cfg->head_dim, cfg->ffn, cfg->vocab,
+    if (ntx::persist_plan(kt, cfg->hidden, cfg->n_heads, cfg->n_kv_heads, cfg->head_dim, cfg->ffn, cfg->vocab,
                           cfg->max_ctx, ntx::sm_count(), cfg->n_layers, &st, &psm) == 0) {
-      const int grid = ntx::persist_grid(qt, psm);
-      bool ok = grid > 0 && grid == ntx::sm_count() && ntx::gemv_tma_ok(qt, head, cfg->hidden);
+      const int grid = ntx::persist_grid(st, psm);
+      bool ok = grid > 0 && grid == ntx::sm_count() && ntx::gemv_tma_ok(head_qtype, head, cfg->hidden);
       for (int l = 0; l < cfg->n_layers && ok; ++l) {
         const ntx::LayerArgs a = layer_args(cfg, static_cast<const uint8_t*>(layers[l].base), &layers[l]);
         const int64_t KO = (int64_t)cfg->n_heads * cfg->head_dim;
-        ok = ntx::gemv_tma_ok(qt, a.wq, cfg->hidden) && ntx::gemv_tma_ok(qt, a.wk, cfg->hidden) &&
-             ntx::gemv_tma_ok(qt, a.wv, cfg->hidden) && ntx::gemv_tma_ok(qt, a.wo, KO) &&
-             ntx::gemv_tma_ok(qt, a.wg, cfg->hidden) && ntx::gemv_tma_ok(qt, a.wu, cfg->hidden) &&
-             ntx::gemv_tma_ok(qt, a.wd, cfg->ffn) && aligned(a.attn_norm, 16) && aligned(a.ffn_norm, 16) &&
-             aligned(e->kc[l], 16) && aligned(e->vc[l], 16);
+        ok = ntx::gemv_tma_ok(a.qt_qkv, a.wq, cfg->hidden) && ntx::gemv_tma_ok(a.qt_qkv, a.wk, cfg->hidden) &&
+             ntx::gemv_tma_ok(a.qt_qkv, a.wv, cfg->hidden) && ntx::gemv_tma_ok(a.qt_o, a.wo, KO) &&
+             ntx::gemv_tma_ok(a.qt_gu, a.wg, cfg->hidden) && ntx::gemv_tma_ok(a.qt_gu, a.wu, cfg->hidden) &&
+             ntx::gemv_tma_ok(a.qt_down, a.wd, cfg->ffn) && aligned(a.attn_norm, 16) &&
+             aligned(a.ffn_norm, 16) && aligned(e->kc[l], 16) && aligned(e->vc[l], 16);
       }
       if (ok) {
         st.H = cfg->hidden; st.Hq = cfg->n_heads; st.Hkv = cfg->n_kv_heads; st.D = cfg->head_dim; st.F = cfg->ffn;
@@ -899,7 +910,8 @@ extern "C" int ntx_persistent_plan(const ntx_model_config* cfg, int qtype, int* 
   ntx::PStep st;
   memset(&st, 0, sizeof st);
   size_t smem = 0;
-  if (ntx::persist_plan(qtype, cfg->hidden, cfg->n_heads, cfg->n_kv_heads, cfg->head_dim, cfg->ffn, cfg->vocab,
+  const int kt[7] = {qtype, qtype, qtype, qtype, qtype, qtype, qtype};
+  if (ntx::persist_plan(kt, cfg->hidden, cfg->n_heads, cfg->n_kv_heads, cfg->head_dim, cfg->ffn, cfg->vocab,
                         cfg->max_ctx, ntx::sm_count(), cfg->n_layers, &st, &smem) != 0)
     return fail(NTX_ERR_SHAPE, "the persistent kernel does not take this model");
   if (slot_bytes) *slot_bytes = st.slot_bytes;

@@ -566,7 +566,6 @@ __device__ __forceinline__ float heads_reduce(float (&v)[G], int lane) {
   return s;
 }
 
-template <int QT>
 struct Consumer {
   const PStep& st;
   PSmem sm;  // used outside the GEMV stage loop only
@@ -582,7 +581,7 @@ struct Consumer {
   // or w h for a phase with an RMSNorm prologue -- the 1/rms scale is applied
   // to each row's result by the epilogue warp, so staging waits for nothing but
   // one batch of loads (h, and w).
-  template <bool NORM>
+  template <int QT, bool NORM>
   __device__ void stage(const float* h, const float* w, int64_t K, const XStage& xs) {
     constexpr int kBatch = NORM ? 4 : 8;
     const int nchunk = (int)(K / 128);
@@ -606,7 +605,18 @@ struct Consumer {
     }
   }
 
+  // A GEMV phase in the block type of its kind: QA, or QB where the step's
+  // plan gives that kind the second type (QB == QA: one type for all).
+  template <int QA, int QB>
   __device__ bool gemv(int kind, const float* h, const float* w) {
+    if constexpr (QA != QB) {
+      if (st.qt[kind] == QB) return gemv_t<QB>(kind, h, w);
+    }
+    return gemv_t<QA>(kind, h, w);
+  }
+
+  template <int QT>
+  __device__ bool gemv_t(int kind, const float* h, const float* w) {
     const PGeom g = sm.kg[kind].g;
     const PRows rows = sm.kg[kind].rows;
     const int64_t K = phase_K(st, kind);
@@ -620,8 +630,8 @@ struct Consumer {
     XRegs<QT> xr;
     const XStage xs = xstage_at(sm.xst, K);
     if (g.staged) {
-      if (w) stage<true>(h, w, K, xs);
-      else stage<false>(h, w, K, xs);
+      if (w) stage<QT, true>(h, w, K, xs);
+      else stage<QT, false>(h, w, K, xs);
       cons_bar();
       if (active) xr.load(xs, c, lane);
     } else {
@@ -1018,7 +1028,10 @@ struct Consumer {
   }
 };
 
-template <int QT>
+// QA: the block type of the step's GEMV phases; QB: a second type some phase
+// kinds may use instead (st.qt[kind]), e.g. the Q6_K down projections and head
+// of a Q4_K_M model.  QA == QB: one type.
+template <int QA, int QB>
 __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_constant__ PStep st) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const PSmem sm = psmem_at(p_smem, st.n_slots, st.slot_bytes, st.xstage_bytes, st.red_floats, st.n_layers);
@@ -1181,7 +1194,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
     }
   } else {
     // ---------------------------------------------------------- consumers
-    Consumer<QT> cs(st, sm, warp, lane);
+    Consumer cs(st, sm, warp, lane);
     const int ctid = cs.ctid;
     for (int p = 0; p < np; ++p) {
       const int kind = phase_kind(p, n);
@@ -1201,10 +1214,10 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
           break;
         case PK_ATTN: {
           const int Gq = st.Hq / st.Hkv, lk = (p - 1) / 5;
-          if (Gq == 8) cs.template attention<8>(*L, lk);
-          else if (Gq == 4) cs.template attention<4>(*L, lk);
-          else if (Gq == 2) cs.template attention<2>(*L, lk);
-          else cs.template attention<1>(*L, lk);
+          if (Gq == 8) cs.attention<8>(*L, lk);
+          else if (Gq == 4) cs.attention<4>(*L, lk);
+          else if (Gq == 2) cs.attention<2>(*L, lk);
+          else cs.attention<1>(*L, lk);
           break;
         }
         default: {  // GEMV phases
@@ -1212,7 +1225,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
           const float* h = kind == PK_GU ? st.h1 : kind == PK_O ? st.attn_out : kind == PK_DOWN ? st.u : st.hidden;
           const float* w = kind == PK_QKV ? L->attn_norm : kind == PK_GU ? L->ffn_norm
                            : kind == PK_HEAD ? st.final_norm : nullptr;
-          cs.gemv(kind, h, w);  // a failed wait raised the CTA abort flag
+          cs.template gemv<QA, QB>(kind, h, w);  // a failed wait raised the CTA abort flag
           break;
         }
       }
@@ -1232,29 +1245,50 @@ std::mutex g_pmu;
 
 }  // namespace
 
+// The (QA, QB) instantiation that runs a step whose phase kinds have the
+// block types kt[] (QKV, O, GU, DOWN, HEAD), or (0, 0) when none does.
+void persist_pair(const int* kt, int* qa, int* qb) {
+  *qa = *qb = 0;
+  const int a = kt[PK_QKV];
+  int b = a;
+  for (int k : {PK_O, PK_GU, PK_DOWN, PK_HEAD})
+    if (kt[k] != a) {
+      if (b != a && kt[k] != b) return;
+      b = kt[k];
+    }
+  const bool one = a == b && (a == QT_Q8_0 || a == QT_Q4_0 || a == QT_Q6_K || a == QT_Q4_K || a == QT_Q5_K);
+  const bool kq6 = (a == QT_Q4_K || a == QT_Q5_K) && b == QT_Q6_K;
+  if (one || kq6) {
+    *qa = a;
+    *qb = b;
+  }
+}
+
 // Host-side plan: slot size, stages, per-phase geometry.
-int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int max_ctx, int grid, int n_layers,
-                 PStep* st, size_t* smem) {
+int persist_plan(const int* kt, int H, int Hq, int Hkv, int D, int F, int64_t V, int max_ctx, int grid,
+                 int n_layers, PStep* st, size_t* smem) {
   (void)V;
-  if (qtype != QT_Q8_0 && qtype != QT_Q4_0 && qtype != QT_Q6_K) return -1;
+  int qa = 0, qb = 0;
+  persist_pair(kt, &qa, &qb);
+  if (qa == 0) return -1;
   if (D != kPD) return -1;
   if (Hkv <= 0 || Hq % Hkv) return -1;
   const int Gq = Hq / Hkv;
   if (Gq != 1 && Gq != 2 && Gq != 4 && Gq != 8) return -1;
-  const int be = qtype == QT_Q6_K ? 256 : 32, bb = qtype == QT_Q6_K ? 210 : (qtype == QT_Q8_0 ? 34 : 18);
   const int64_t KO = (int64_t)Hq * D;
   struct KInfo {
     int kind;
     int64_t K;
     int align;
   } ks[5] = {{PK_QKV, H, 2}, {PK_O, KO, 1}, {PK_GU, H, 2}, {PK_DOWN, F, 1}, {PK_HEAD, H, 1}};
+  for (int k = 0; k < 7; ++k) st->qt[k] = kt[k];
   for (auto& k : ks) {
-    const bool fixed = qtype != QT_Q6_K;
-    if (fixed ? (k.K % 256) : (k.K % 2048)) return -1;
+    const int qt = kt[k.kind];
+    if (qt == QT_Q6_K ? (k.K % 2048) : (k.K % 256)) return -1;
     if (k.K > (int64_t)kPConsumers * kSliceCols) return -1;
     PGeom& g = st->g[k.kind];
     g.align = k.align;
-    g.row_bytes = (int)(k.K / be * bb);
+    g.row_bytes = (int)(k.K / qt_block_elems(qt) * qt_block_bytes(qt));
     g.n_slices = (int)((k.K + kSliceCols - 1) / kSliceCols);
   }
   // attention scratch lives in the x staging region
@@ -1288,10 +1322,10 @@ int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int
         if (nrg_max < 1) nrg_max = 1;
         if (tr < nrg_max) full_rg = false;
         const int nrg = nrg_max > tr ? tr : nrg_max;
-        if (tr % nrg) even = false;
-        const bool staged = qtype != QT_Q6_K || nrg > 1;
+        if (kt[k.kind] == QT_Q6_K && tr % nrg) even = false;
+        const bool staged = kt[k.kind] != QT_Q6_K || nrg > 1;
         if (staged) {
-          const int b = (int)((xstage_bytes(qtype, k.K) + 15) / 16 * 16);
+          const int b = (int)((xstage_bytes(kt[k.kind], k.K) + 15) / 16 * 16);
           if (b > xbz) xbz = b;
         }
         if (tr * g.n_slices > rf) rf = tr * g.n_slices;
@@ -1305,7 +1339,7 @@ int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int
         const int64_t inflight = (int64_t)S * TRs[k.kind] * st->g[k.kind].row_bytes;
         if (inflight < inflight_min) inflight_min = inflight;
       }
-      const int64_t key[5] = {full_rg ? 1 : 0, S >= 3 ? 1 : 0, (qtype == QT_Q6_K && even) ? 1 : 0, inflight_min,
+      const int64_t key[5] = {full_rg ? 1 : 0, S >= 3 ? 1 : 0, (qb == QT_Q6_K && even) ? 1 : 0, inflight_min,
                               -(int64_t)Z};
       bool better = false;
       for (int i = 0; i < 5; ++i) {
@@ -1331,9 +1365,9 @@ int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int
     if (nrg > tr) nrg = tr;
     g.n_rg = nrg;
     g.NW = g.n_slices * nrg;
-    g.staged = qtype != QT_Q6_K || nrg > 1;
+    g.staged = kt[k.kind] != QT_Q6_K || nrg > 1;
     if (g.staged) {
-      const int b = (int)((xstage_bytes(qtype, k.K) + 15) / 16 * 16);
+      const int b = (int)((xstage_bytes(kt[k.kind], k.K) + 15) / 16 * 16);
       if (b > xbz) xbz = b;
     }
     if (tr * g.n_slices > rf) rf = tr * g.n_slices;
@@ -1346,12 +1380,36 @@ int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int
   return 0;
 }
 
-cudaError_t launch_persist(int qtype, const PStep& st, size_t smem, int grid, cudaStream_t s) {
-  static unsigned long long done[3] = {0, 0, 0};
-  void (*kern)(const PStep) = qtype == QT_Q8_0 ? persist_kernel<QT_Q8_0>
-                        : qtype == QT_Q4_0 ? persist_kernel<QT_Q4_0>
-                                           : persist_kernel<QT_Q6_K>;
-  const int ki = qtype == QT_Q8_0 ? 0 : qtype == QT_Q4_0 ? 1 : 2;
+namespace {
+// The instantiation for a type pair (see persist_pair) and its index.
+using PKern = void (*)(const PStep);
+PKern persist_kern(int qa, int qb, int* index) {
+  struct {
+    int a, b;
+    PKern k;
+  } const table[] = {{QT_Q8_0, QT_Q8_0, persist_kernel<QT_Q8_0, QT_Q8_0>},
+                     {QT_Q4_0, QT_Q4_0, persist_kernel<QT_Q4_0, QT_Q4_0>},
+                     {QT_Q6_K, QT_Q6_K, persist_kernel<QT_Q6_K, QT_Q6_K>},
+                     {QT_Q4_K, QT_Q4_K, persist_kernel<QT_Q4_K, QT_Q4_K>},
+                     {QT_Q5_K, QT_Q5_K, persist_kernel<QT_Q5_K, QT_Q5_K>},
+                     {QT_Q4_K, QT_Q6_K, persist_kernel<QT_Q4_K, QT_Q6_K>},
+                     {QT_Q5_K, QT_Q6_K, persist_kernel<QT_Q5_K, QT_Q6_K>}};
+  for (int i = 0; i < (int)(sizeof table / sizeof table[0]); ++i)
+    if (table[i].a == qa && table[i].b == qb) {
+      *index = i;
+      return table[i].k;
+    }
+  *index = -1;
+  return nullptr;
+}
+}  // namespace
+
+cudaError_t launch_persist(const PStep& st, size_t smem, int grid, cudaStream_t s) {
+  static unsigned long long done[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int qa = 0, qb = 0, ki = -1;
+  persist_pair(st.qt, &qa, &qb);
+  PKern kern = persist_kern(qa, qb, &ki);
+  if (!kern) return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(done[ki] & (1ull << dev))) {
@@ -1373,10 +1431,11 @@ cudaError_t launch_persist(int qtype, const PStep& st, size_t smem, int grid, cu
   return cudaLaunchKernelEx(&cfg, kern, st);
 }
 
-int persist_grid(int qtype, size_t smem) {
-  void (*kern)(const PStep) = qtype == QT_Q8_0 ? persist_kernel<QT_Q8_0>
-                        : qtype == QT_Q4_0 ? persist_kernel<QT_Q4_0>
-                                           : persist_kernel<QT_Q6_K>;
+int persist_grid(const PStep& st, size_t smem) {
+  int qa = 0, qb = 0, ki = -1;
+  persist_pair(st.qt, &qa, &qb);
+  PKern kern = persist_kern(qa, qb, &ki);
+  if (!kern) return 0;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess) return 0;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPThreads, smem) != cudaSuccess) return 0;

@@ -57,18 +57,22 @@ struct PStep {
   int abort_index;     // grid-wide abort word in sync
   int n_split;         // attention splits per KV head
   PGeom g[7];          // indexed by PKind
+  int qt[7];           // block type of each GEMV phase kind (indexed by PKind)
   int slot_bytes, n_slots, xstage_bytes, red_floats;
   int* status;  // device status word
   unsigned long long* probe_ts;  // nullable: [1 + phases][grid] %globaltimer ns (row 0: kernel start,
                                  // row 1 + p: when the CTA published phase p)
 };
 
-// Fills the geometry fields of *st and the dynamic shared memory size; -1 if
-// the shapes are outside what the persistent kernel handles.
-int persist_plan(int qtype, int H, int Hq, int Hkv, int D, int F, int64_t V, int max_ctx, int grid, int n_layers,
-                 PStep* st, size_t* smem);
+// Fills the geometry fields and phase types of *st and the dynamic shared
+// memory size for phase kinds of block types kt[] (indexed by PKind); -1 if
+// the shapes or types are outside what the persistent kernel handles.
+int persist_plan(const int* kt, int H, int Hq, int Hkv, int D, int F, int64_t V, int max_ctx, int grid,
+                 int n_layers, PStep* st, size_t* smem);
+// The instantiation (type pair) that runs phase kinds of types kt[]; 0, 0 if none.
+void persist_pair(const int* kt, int* qa, int* qb);
 // Grid size (one CTA per SM), or 0 if a CTA of this size cannot be resident.
-int persist_grid(int qtype, size_t smem);
+int persist_grid(const PStep& st, size_t smem);
 // Attention splits per KV head at most (at most one unit per CTA); a step
 // uses fewer when its context is short.
 inline int persist_splits(int grid, int Hkv, int max_ctx) {
@@ -78,6 +82,6 @@ inline int persist_splits(int grid, int Hkv, int max_ctx) {
 }
 // Words of the sync array for n_layers executed layers.
 inline int persist_sync_words(int n_layers, int Hkv) { return 2 + 5 * n_layers + n_layers * Hkv + 1; }
-cudaError_t launch_persist(int qtype, const PStep& st, size_t smem, int grid, cudaStream_t s);
+cudaError_t launch_persist(const PStep& st, size_t smem, int grid, cudaStream_t s);
 
 }  // namespace ntx

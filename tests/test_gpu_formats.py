@@ -216,18 +216,26 @@ def test_decode_layer_mixed_types(types):
     assert abs(float(cos.item()) - cref) <= 1e-5
 
 
-def test_engine_q4_k_m_model_teacher_forced():
-    """A 4-layer Q4_K_M model (Q4_K matrices, Q6_K down projections and head)
-    through the engine: every step's logits within 2e-2 * RMS of the oracle's,
-    teacher-forced on the GPU's tokens, greedy token where the gap allows."""
+@pytest.mark.parametrize("types,head", [(wl.Q4_K_M, wl.Q4_K_M_HEAD), ((Q5_K,) * 6 + (Q6_K,), Q6_K),
+                                        ((Q4_K,) * 7, Q4_K)], ids=["q4_k_m", "q5_k_q6_k", "q4_k"])
+def test_engine_k_quant_models_persistent_and_chain(types, head):
+    """4-layer K-quant models (Q4_K_M: Q4_K matrices, Q6_K down projections and
+    head) through the engine, as the persistent kernel (one launch per step,
+    per-phase block types) and as the per-op chain: every step's logits within
+    2e-2 * RMS of the oracle's, teacher-forced on the GPU's tokens, greedy
+    token where the gap allows."""
     from synthgen.devmodel import DeviceModel
     from test_gpu_engine import Engine, check_logits, oracle_run
     d = dict(MIX_D, n_layers=4)
-    m = DeviceModel(d, wl.Q4_K_M, wl.Q4_K_M_HEAD, 91, max_ctx=24, n_prior=0, source="host")
-    e = Engine(m)
+    m = DeviceModel(d, types, head, 91, max_ctx=24, n_prior=0, source="host")
     prompt = [int(t) for t in sg.tokens(91, "prompt", 3, d["vocab"])]
-    lg, fed, nx, _ = e.run(prompt + [-1] * 3)
-    e.close()
-    refs = oracle_run(m, fed)
-    for s in range(len(fed)):
-        check_logits(lg[s], refs[s][0], int(nx[s]), s)
+    for flags in (0, ntx.NTX_NO_PERSIST):
+        m.reset_kv()
+        e = Engine(m)
+        lg, fed, nx, _ = e.run(prompt + [-1] * 3, flags=flags)
+        launches = ntx.ntx_engine_launches_per_step(e.h)
+        e.close()
+        assert (launches == 1) == (flags == 0), launches
+        refs, _ = oracle_run(m, fed)
+        for s in range(len(fed)):
+            check_logits(lg[s], refs[s], int(nx[s]), s)
