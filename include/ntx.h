@@ -378,7 +378,31 @@ NTX_API int ntx_memory_budget(uint64_t* device_free, uint64_t* device_total, uin
  * number of skipped layers, or a negative error. */
 NTX_API int ntx_engine_skip_mask(ntx_engine* e, uint8_t* mask_host);
 
-NTX_API void ntx_engine_destroy(ntx_engine* e);
+/* Waits (bounded, see ntx_set_host_wait_limit) for the engine's streams and
+ * frees the engine.  NTX_ERR_TIMEOUT if its work has not completed in time:
+ * the engine is then kept (nothing is freed under running work) and the call
+ * may be repeated. */
+NTX_API int ntx_engine_destroy(ntx_engine* e);
+
+/* Failure detection.  Every host wait of the engine (ntx_engine_create,
+ * the parameter ring of ntx_decode_step, the calibration read-back,
+ * ntx_engine_destroy) polls its stream with a deadline of `ms` milliseconds
+ * (default 60000, process-wide) and returns NTX_ERR_TIMEOUT past it, leaving
+ * the GPU work running.  NTX_ERR_INVALID_ARG for 0.  Environment hook for
+ * tests: NTX_FAULT=<name>[,<name>...] makes the named point fail as if its
+ * operation had failed, before the call enqueues anything: pinned_alloc
+ * (ntx_engine_create: NTX_ERR_NOMEM), h2d_submit (ntx_decode_step of a step
+ * that streams host layers: NTX_ERR_CUDA), host_wait (every bounded host
+ * wait: NTX_ERR_TIMEOUT). */
+NTX_API int ntx_set_host_wait_limit(uint64_t ms);
+
+/* Failure-path testing of the persistent kernel: for steps enqueued after the
+ * call without a graph (NTX_NO_GRAPH; captured graphs keep their settings),
+ * CTA stall_cta (-1: none) withholds its publication of the embed phase, and
+ * every wait of the kernel gives up after wait_ns nanoseconds (0: the default
+ * 2 s).  With a stalled CTA the others' grid-wide waits run out: the kernel
+ * returns with device status 4 (ntx_device_status) and no CTA left waiting. */
+NTX_API int ntx_engine_set_fault(ntx_engine* e, int stall_cta, uint64_t wait_ns);
 
 #ifdef __cplusplus
 }

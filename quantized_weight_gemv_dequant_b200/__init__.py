@@ -40,7 +40,7 @@ EXPORTS = (
     "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
     "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
     "ntx_persistent_plan", "ntx_layer_layout_mixed", "ntx_engine_device_bytes", "ntx_auto_tier_map",
-    "ntx_memory_budget",
+    "ntx_memory_budget", "ntx_set_host_wait_limit", "ntx_engine_set_fault",
 )
 
 
@@ -100,7 +100,9 @@ def lib():
                                    vp, vp, sz, vp, vp, P(vp)], i32),
             "ntx_decode_step": ([vp, ctypes.c_int32, i32, vp, vp, i32, vp], i32),
             "ntx_engine_skip_mask": ([vp, vp], i32),
-            "ntx_engine_destroy": ([vp], None),
+            "ntx_engine_destroy": ([vp], i32),
+            "ntx_set_host_wait_limit": ([ctypes.c_uint64], i32),
+            "ntx_engine_set_fault": ([vp, i32, ctypes.c_uint64], i32),
             "ntx_engine_set_probe": ([vp, vp, vp, i32], i32),
             "ntx_engine_launches_per_step": ([vp], i32),
             "ntx_attn_decode_static": ([vp, vp, vp, vp, i32, i32, i32, i32, i32, vp], i32),
@@ -279,7 +281,15 @@ def ntx_engine_skip_mask(engine, n_layers):
 
 
 def ntx_engine_destroy(engine):
-    lib().ntx_engine_destroy(engine)
+    _check(lib().ntx_engine_destroy(engine))
+
+
+def ntx_set_host_wait_limit(ms: int) -> None:
+    _check(lib().ntx_set_host_wait_limit(ms))
+
+
+def ntx_engine_set_fault(engine, stall_cta: int, wait_ns: int = 0) -> None:
+    _check(lib().ntx_engine_set_fault(engine, stall_cta, wait_ns))
 
 
 def ntx_engine_set_probe(engine, begin_events, end_events):

@@ -4,11 +4,15 @@
 // layer skip, CUDA-graph replay of the per-token launch sequence).
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <chrono>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <string>
+#include <thread>
 #include <tuple>
 #include <vector>
 
@@ -71,6 +75,58 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+// ------------------------------------------------------------ host waits
+// Every host wait of the engine polls with a deadline instead of blocking:
+// a stream or event that has not completed within the limit gives
+// NTX_ERR_TIMEOUT (the GPU work is left running; the caller decides).
+std::atomic<uint64_t> g_host_wait_ms{60000};
+
+// Host-side fault injection for tests: NTX_FAULT is a comma-separated list
+// of names; a call that reaches the named point fails as if the underlying
+// operation had failed, before it enqueues any work.
+//   pinned_alloc  ntx_engine_create's pinned parameter block
+//   h2d_submit    ntx_decode_step of a step that streams host layers
+//   host_wait     every bounded host wait (reports NTX_ERR_TIMEOUT at once)
+bool fault(const char* name) {
+  const char* env = getenv("NTX_FAULT");
+  if (!env || !*env) return false;
+  const size_t n = strlen(name);
+  for (const char* p = env; *p;) {
+    const char* q = strchr(p, ',');
+    const size_t len = q ? (size_t)(q - p) : strlen(p);
+    if (len == n && strncmp(p, name, n) == 0) return true;
+    if (!q) break;
+    p = q + 1;
+  }
+  return false;
+}
+
+// Waits for `ev` (already recorded) with the host deadline: cudaSuccess,
+// cudaErrorTimeout, or the event's error.
+cudaError_t wait_event(cudaEvent_t ev) {
+  if (fault("host_wait")) return cudaErrorTimeout;
+  const auto t0 = std::chrono::steady_clock::now();
+  const auto limit = std::chrono::milliseconds(g_host_wait_ms.load());
+  for (unsigned spin = 0;; ++spin) {
+    const cudaError_t e = cudaEventQuery(ev);
+    if (e != cudaErrorNotReady) return e;
+    if (std::chrono::steady_clock::now() - t0 > limit) return cudaErrorTimeout;
+    if (spin > 64) std::this_thread::sleep_for(std::chrono::microseconds(20));
+  }
+}
+
+// Records `ev` on stream s and waits for it with the host deadline.
+cudaError_t wait_stream(cudaStream_t s, cudaEvent_t ev) {
+  const cudaError_t e = cudaEventRecord(ev, s);
+  return e == cudaSuccess ? wait_event(ev) : e;
+}
+
+int wait_fail(cudaError_t e, const char* what) {
+  if (e == cudaErrorTimeout) return fail(NTX_ERR_TIMEOUT, "%s: the GPU work did not complete within %llu ms", what,
+                                         (unsigned long long)g_host_wait_ms.load());
+  return cuda_fail(e, what);
+}
 
 // K constraint of the fused (bulk-copy) GEMV path.
 bool k_ok_fused(int qt, int64_t K) { return qt == NTX_Q6_K ? K % 2048 == 0 : K % 256 == 0; }
@@ -403,7 +459,7 @@ struct ntx_engine {
   int* pinned;
   cudaEvent_t ring_ev[64];
   int ring_pos;
-  cudaEvent_t copy_done[2], slot_free[2], fork_ev, join_ev;
+  cudaEvent_t copy_done[2], slot_free[2], fork_ev, join_ev, sync_ev;
   // skip set
   std::vector<uint8_t> skip;
   bool skip_valid;
@@ -483,6 +539,7 @@ void engine_free(ntx_engine* e) {
   }
   if (e->fork_ev) cudaEventDestroy(e->fork_ev);
   if (e->join_ev) cudaEventDestroy(e->join_ev);
+  if (e->sync_ev) cudaEventDestroy(e->sync_ev);
   if (e->pinned) cudaFreeHost(e->pinned);
   delete e;
 }
@@ -702,6 +759,10 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   engine_carve(cfg, static_cast<uint8_t*>(workspace), e);
   e->skip.assign(cfg->n_layers, 0);
   e->skip_valid = false;
+  if (fault("pinned_alloc")) {
+    engine_free(e);
+    return fail(NTX_ERR_NOMEM, "ntx_engine_create: pinned parameter block allocation failed (injected)");
+  }
   cudaError_t err = cudaHostAlloc(reinterpret_cast<void**>(&e->pinned), 64 * 4 * sizeof(int), cudaHostAllocDefault);
   for (int i = 0; i < 64 && err == cudaSuccess; ++i) err = cudaEventCreateWithFlags(&e->ring_ev[i], cudaEventDisableTiming);
   for (int i = 0; i < 2 && err == cudaSuccess; ++i) {
@@ -710,6 +771,7 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   }
   if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->fork_ev, cudaEventDisableTiming);
   if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->join_ev, cudaEventDisableTiming);
+  if (err == cudaSuccess) err = cudaEventCreateWithFlags(&e->sync_ev, cudaEventDisableTiming);
   // persistent kernel: each GEMV phase kind (Q/K/V, O, gate/up, down, head) of one block type over all
   // layers, a type pair it is built for, shapes and alignment it handles; it runs the steps whose executed
   // layers are all resident (all steps without a host tier; with one, the steps under a skip set that skips
@@ -756,6 +818,8 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
         st.sync = e->psync;
         st.n_split = ntx::persist_splits(grid, cfg->n_kv_heads, cfg->max_ctx);
         st.status = ntx::device_status_ptr();
+        st.wait_ns = ntx::kDefaultWaitNs;
+        st.stall_cta = -1;
         if (!any_host) {
           std::vector<int> all(cfg->n_layers);
           for (int l = 0; l < cfg->n_layers; ++l) all[l] = l;
@@ -773,7 +837,10 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   }
   // token state starts at 0
   if (err == cudaSuccess) err = cudaMemsetAsync(e->token_state, 0, 4 * sizeof(int), e->cs);
-  if (err == cudaSuccess) err = cudaStreamSynchronize(e->cs);
+  if (err == cudaSuccess) {
+    err = wait_stream(e->cs, e->sync_ev);
+    if (err == cudaErrorTimeout) return wait_fail(err, "ntx_engine_create");  // work in flight: leak, do not free
+  }
   if (err != cudaSuccess) {
     engine_free(e);
     return cuda_fail(err, "ntx_engine_create");
@@ -800,8 +867,15 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
   // step parameters: pinned ring slot -> device
   const int slot = e->ring_pos;
   e->ring_pos = (e->ring_pos + 1) % 64;
-  cudaError_t err = cudaEventSynchronize(e->ring_ev[slot]);
-  if (err != cudaSuccess) return cuda_fail(err, "param ring");
+  // a step that streams host layers: the copies are submitted below (injected failure: nothing enqueued)
+  if (fault("h2d_submit")) {
+    bool streams = false;
+    for (int l = 0; l < c.n_layers && !streams; ++l)
+      streams = e->tier[l] == 1 && !(use_skip && e->skip[l]);
+    if (streams) return fail(NTX_ERR_CUDA, "ntx_decode_step: host-to-device copy submission failed (injected)");
+  }
+  cudaError_t err = wait_event(e->ring_ev[slot]);
+  if (err != cudaSuccess) return wait_fail(err, "param ring");
   e->pinned[slot * 4 + 0] = pos;
   e->pinned[slot * 4 + 1] = token;
   err = cudaMemcpyAsync(e->params, e->pinned + slot * 4, 2 * sizeof(int), cudaMemcpyHostToDevice, e->cs);
@@ -838,8 +912,8 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
   if (calibrate) {
     std::vector<float> cs(c.n_layers);
     err = cudaMemcpyAsync(cs.data(), e->cos_int, sizeof(float) * c.n_layers, cudaMemcpyDeviceToHost, e->cs);
-    if (err == cudaSuccess) err = cudaStreamSynchronize(e->cs);
-    if (err != cudaSuccess) return cuda_fail(err, "calibration read-back");
+    if (err == cudaSuccess) err = wait_stream(e->cs, e->sync_ev);
+    if (err != cudaSuccess) return wait_fail(err, "calibration read-back");
     std::vector<int> list;
     for (int l = 0; l < c.n_layers; ++l) {
       e->skip[l] = cs[l] >= c.skip_threshold ? 1 : 0;
@@ -929,9 +1003,25 @@ extern "C" int ntx_engine_launches_per_step(ntx_engine* e) {
   return e->launches;
 }
 
-extern "C" void ntx_engine_destroy(ntx_engine* e) {
-  if (!e) return;
-  cudaStreamSynchronize(e->cs);
-  if (e->xs) cudaStreamSynchronize(e->xs);
+extern "C" int ntx_engine_destroy(ntx_engine* e) {
+  if (!e) return NTX_OK;
+  cudaError_t err = wait_stream(e->cs, e->sync_ev);
+  if (err == cudaSuccess && e->xs) err = wait_stream(e->xs, e->sync_ev);
+  if (err == cudaErrorTimeout) return wait_fail(err, "ntx_engine_destroy");  // work in flight: the engine is kept
   engine_free(e);
+  return err == cudaSuccess ? NTX_OK : cuda_fail(err, "ntx_engine_destroy");
+}
+
+extern "C" int ntx_set_host_wait_limit(uint64_t ms) {
+  if (ms == 0) return fail(NTX_ERR_INVALID_ARG, "host wait limit must be > 0 ms");
+  g_host_wait_ms.store(ms);
+  return NTX_OK;
+}
+
+extern "C" int ntx_engine_set_fault(ntx_engine* e, int stall_cta, uint64_t wait_ns) {
+  if (!e) return fail(NTX_ERR_INVALID_ARG, "engine is NULL");
+  if (stall_cta < -1) return fail(NTX_ERR_INVALID_ARG, "stall_cta must be >= -1");
+  e->pst.stall_cta = stall_cta;
+  e->pst.wait_ns = wait_ns ? wait_ns : ntx::kDefaultWaitNs;
+  return NTX_OK;
 }

@@ -81,14 +81,14 @@ __device__ __forceinline__ unsigned atom_acq_rel_add(unsigned* p, unsigned v) {
 
 // One thread: wait until *ctr >= target.  False if the grid-wide abort word is
 // raised or the wait runs out (which raises it).
-__device__ bool grid_wait(const unsigned* ctr, unsigned target, unsigned* gabort, int* status) {
+__device__ bool grid_wait(const unsigned* ctr, unsigned target, unsigned* gabort, int* status, uint64_t limit) {
   if (ld_acquire(ctr) >= target) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
     __nanosleep(20);
     if (ld_acquire(ctr) >= target) return true;
     if (*reinterpret_cast<volatile unsigned*>(gabort)) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit) {
       atomicExch(status, (int)kStatusGridTimeout);
       atomicExch(gabort, 1u);
       return false;
@@ -98,13 +98,13 @@ __device__ bool grid_wait(const unsigned* ctr, unsigned target, unsigned* gabort
 
 // Warp-uniform bounded wait on an mbarrier phase that also gives up when this
 // CTA has aborted.
-__device__ bool pwait(uint64_t* bar, uint32_t parity, volatile int* cta_abort) {
+__device__ bool pwait(uint64_t* bar, uint32_t parity, volatile int* cta_abort, uint64_t limit) {
   bool done = mbar_try_wait(bar, parity);
   if (__all_sync(0xffffffffu, done)) return true;
   const uint64_t t0 = global_ns();
   while (!__all_sync(0xffffffffu, done)) {
     if (!done) done = mbar_try_wait_sleep(bar, parity);
-    const bool give_up = *cta_abort || global_ns() - t0 > kWaitLimitNs;
+    const bool give_up = *cta_abort || global_ns() - t0 > limit;
     if (__any_sync(0xffffffffu, !done && give_up)) break;
   }
   return __all_sync(0xffffffffu, done);
@@ -320,13 +320,13 @@ __device__ __forceinline__ void mbar_arrive_a(uint32_t a) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
 }
 // pwait on a 32-bit address; cta_abort is the CTA abort word in shared memory.
-__device__ bool pwait_a(uint32_t bar, uint32_t parity, const volatile int* cta_abort) {
+__device__ bool pwait_a(uint32_t bar, uint32_t parity, const volatile int* cta_abort, uint64_t limit) {
   bool done = mbar_test_a(bar, parity);
   if (__all_sync(0xffffffffu, done)) return true;
   const uint64_t t0 = global_ns();
   while (!__all_sync(0xffffffffu, done)) {
     if (!done) done = mbar_sleep_a(bar, parity);
-    const bool give_up = *cta_abort || global_ns() - t0 > kWaitLimitNs;
+    const bool give_up = *cta_abort || global_ns() - t0 > limit;
     if (__any_sync(0xffffffffu, !done && give_up)) break;
   }
   return __all_sync(0xffffffffu, done);
@@ -373,7 +373,7 @@ struct Copier {
         uint64_t* bar = sm.full + k % n_slots;
         const uint32_t par = (uint32_t)((k / n_slots) & 1);
         while (!mbar_try_wait(bar, par))
-          if (global_ns() - t0 > kWaitLimitNs) { atomicExch(st.status, (int)kStatusDrainTimeout); return; }
+          if (global_ns() - t0 > st.wait_ns) { atomicExch(st.status, (int)kStatusDrainTimeout); return; }
       }
     }
     __syncwarp();
@@ -384,7 +384,7 @@ struct Copier {
     int s = 0;
     uint32_t ph = 0;
     while (it.valid(np)) {
-      if (!pwait(sm.empty + s, ph, sm.misc)) {
+      if (!pwait(sm.empty + s, ph, sm.misc, st.wait_ns)) {
         if (lane == 0) {
           atomicExch(sm.misc, 1);
           atomicExch(st.sync + st.abort_index, 1u);
@@ -479,7 +479,7 @@ struct Epilogue {
     if (nst > 0) epi.preload(r0, (int)min64(TR, r1 - r0), lane);
     for (int i = 0; i < nst; ++i, ++q) {
       const int slot = q % kPRed;
-      if (!pwait(sm.rfull + slot, (uint32_t)((q / kPRed) & 1), sm.misc)) return false;
+      if (!pwait(sm.rfull + slot, (uint32_t)((q / kPRed) & 1), sm.misc, st.wait_ns)) return false;
       const int64_t rs = r0 + (int64_t)i * TR;
       const int nr = (int)min64(TR, r1 - rs);
       const float* rd = sm.red + (size_t)slot * red_floats;
@@ -509,7 +509,7 @@ struct Epilogue {
     epi.begin(r0, r1, lane);
     for (int i = 0; i < nst; ++i, ++q) {
       const int slot = q % kPRed;
-      if (!pwait(sm.rfull + slot, (uint32_t)((q / kPRed) & 1), sm.misc)) return false;
+      if (!pwait(sm.rfull + slot, (uint32_t)((q / kPRed) & 1), sm.misc, st.wait_ns)) return false;
       const int rs = r0 + i * TR;
       const int nr = min(TR, r1 - rs);
       const float* rd = sm.red + (size_t)slot * red_floats;
@@ -650,8 +650,9 @@ struct Consumer {
     const uint32_t ring_c = (uint32_t)c * QTraits<QT>::SEG;
     for (int i = 0; i < nst; ++i, ++q) {
       const uint32_t rslot = (uint32_t)q % kPRed;
-      bool ok = pwait_a(sb + o_full + 8 * s, ph, cta_abort);
-      if (ok && busy) ok = pwait_a(sb + o_rempty + 8 * rslot, (uint32_t)(((q / kPRed) & 1) ^ 1), cta_abort);
+      bool ok = pwait_a(sb + o_full + 8 * s, ph, cta_abort, st.wait_ns);
+      if (ok && busy)
+        ok = pwait_a(sb + o_rempty + 8 * rslot, (uint32_t)(((q / kPRed) & 1) ^ 1), cta_abort, st.wait_ns);
       if (!ok) {
         if (lane == 0) {
           atomicExch(sm.misc, 1);
@@ -667,9 +668,10 @@ struct Consumer {
           const int s2 = s + 1 == (int)S ? 0 : s + 1;
           const uint32_t ph2 = s + 1 == (int)S ? ph ^ 1u : ph;
           const uint32_t rslot2 = (uint32_t)(q + 1) % kPRed;
-          bool ok2 = pwait_a(sb + o_full + 8 * s2, ph2, cta_abort);
+          bool ok2 = pwait_a(sb + o_full + 8 * s2, ph2, cta_abort, st.wait_ns);
           if (ok2 && busy)
-            ok2 = pwait_a(sb + o_rempty + 8 * rslot2, (uint32_t)((((q + 1) / kPRed) & 1) ^ 1), cta_abort);
+            ok2 = pwait_a(sb + o_rempty + 8 * rslot2, (uint32_t)((((q + 1) / kPRed) & 1) ^ 1), cta_abort,
+                          st.wait_ns);
           if (!ok2) {
             if (lane == 0) {
               atomicExch(sm.misc, 1);
@@ -1104,7 +1106,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
       const PGeom g = sm.kg[kind].g;
       // the epilogue reads what earlier phases wrote
       int wok = 1;
-      if (lane == 0) wok = grid_wait(st.sync + (p - 1), G, gabort, st.status);
+      if (lane == 0) wok = grid_wait(st.sync + (p - 1), G, gabort, st.status, st.wait_ns);
       if (!__shfl_sync(0xffffffffu, wok, 0)) { ok = false; break; }
       // RMSNorm phases: the sum-of-squares partials of the phase input
       const float* parts = kind == PK_GU ? st.stats_o
@@ -1201,7 +1203,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
       int* go = sm.misc + 1 + (p & 1);
       if (ctid == 0) {
         bool ok = !*reinterpret_cast<volatile int*>(sm.misc);
-        if (ok && p > 0) ok = grid_wait(st.sync + (p - 1), G, gabort, st.status);
+        if (ok && p > 0) ok = grid_wait(st.sync + (p - 1), G, gabort, st.status, st.wait_ns);
         if (!ok) atomicExch(sm.misc, 1);  // the other warps stop waiting for these
         *go = ok;
       }
@@ -1230,9 +1232,11 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
         }
       }
       if (kind == PK_EMBED || kind == PK_ATTN) {
-        // publish (release by one thread after the CTA barrier)
+        // publish (release by one thread after the CTA barrier); a CTA named
+        // by the host's stall setting withholds its embed publication, so
+        // that the other CTAs' bounded waits run out (failure-path testing)
         cons_bar();
-        if (ctid == 0) {
+        if (ctid == 0 && !(p == 0 && (int)blockIdx.x == st.stall_cta)) {
           red_release_add(st.sync + p, 1u);
           if (st.probe_ts) st.probe_ts[(size_t)(1 + p) * G + blockIdx.x] = global_ns();
         }

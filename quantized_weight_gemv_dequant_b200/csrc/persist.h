@@ -7,6 +7,7 @@
 
 namespace ntx {
 
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // the persistent kernel's wait limit unless a test lowers it
 constexpr int kPConsumers = 14;      // consumer warps per CTA (plus an epilogue warp and a copy warp)
 constexpr int kPRed = 8;             // depth of the row-partial ring between consumers and the epilogue warp
 constexpr int kPPartsPerLane = 8;    // CTAs at most: 32 * this (sum-of-squares partials read per lane)
@@ -60,6 +61,8 @@ struct PStep {
   int qt[7];           // block type of each GEMV phase kind (indexed by PKind)
   int slot_bytes, n_slots, xstage_bytes, red_floats;
   int* status;  // device status word
+  uint64_t wait_ns;  // limit on every wait of the kernel (nanoseconds of %globaltimer)
+  int stall_cta;     // a CTA that withholds its embed publication (failure-path tests), -1: none
   unsigned long long* probe_ts;  // nullable: [1 + phases][grid] %globaltimer ns (row 0: kernel start,
                                  // row 1 + p: when the CTA published phase p)
 };

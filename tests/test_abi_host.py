@@ -207,3 +207,24 @@ def test_new_formats_argument_checks():
         assert _rc(ntx.ntx_dequant, qt, FAKE, FAKE + 0x1000, 255) == ntx.NTX_ERR_SHAPE
     assert _rc(ntx.ntx_gemv_q, ntx.NTX_MIXED, FAKE, 16, 256, FAKE + 0x100000, FAKE + 0x200000) == ntx.NTX_ERR_QTYPE
     assert _rc(ntx.ntx_dequant, 3, FAKE, FAKE + 0x1000, 256) == ntx.NTX_ERR_QTYPE
+
+
+def test_injected_pinned_alloc_failure_enqueues_nothing(monkeypatch):
+    """NTX_FAULT=pinned_alloc: ntx_engine_create fails with NTX_ERR_NOMEM at its
+    first allocation, before any stream work (the made-up addresses are never
+    touched: the call returns before enqueuing)."""
+    d = wl.MODEL_8B
+    cfg = _cfg(d, layers=1)
+    _, lw = ntx.ntx_layer_layout(cfg, ntx.NTX_Q8_0)
+    lw.base = FAKE
+    ews = ntx.ntx_engine_workspace_bytes(cfg)
+    monkeypatch.setenv("NTX_FAULT", "host_wait,pinned_alloc")
+    rc = _rc(ntx.ntx_engine_create, cfg, [lw], [0], None, None, 0, FAKE, FAKE, FAKE, ntx.NTX_Q8_0, [FAKE], [FAKE],
+             FAKE, ews, 1, None)
+    assert rc == ntx.NTX_ERR_NOMEM and "injected" in ntx.ntx_last_error()
+
+
+def test_host_wait_limit_argument():
+    assert ntx.lib().ntx_set_host_wait_limit(0) == ntx.NTX_ERR_INVALID_ARG
+    assert ntx.lib().ntx_set_host_wait_limit(60000) == ntx.NTX_OK
+    assert ntx.lib().ntx_engine_set_fault(None, -1, 0) == ntx.NTX_ERR_INVALID_ARG
