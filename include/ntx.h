@@ -304,6 +304,29 @@ NTX_API int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_weigh
 NTX_API int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* logits, int32_t* next_token, int flags,
                     float* cos_out);
 
+/* Self-speculative decoding ([README] 主な機能: Self-speculative decoding, the
+ * VRAM-resident layers as the draft model, no extra model; クイックスタート
+ * --self-spec --draft-k 3).  Given `token` at position `pos` (not yet
+ * processed), the draft -- the resident (tier 0) layers only, then the head --
+ * proposes draft_k greedy tokens for positions pos+1..pos+draft_k, one step
+ * each; then the whole model verifies the token and the proposals at
+ * positions pos..pos+draft_k in one pass, layer by layer, so each host layer
+ * crosses the link once for all draft_k + 1 tokens.  The longest prefix of
+ * proposals equal to the whole model's greedy tokens is accepted, followed by
+ * the whole model's next token: tokens_out[0..*n_out-1] (host int32,
+ * capacity draft_k + 1, 1 <= *n_out <= draft_k + 1) are exactly the greedy
+ * continuation t_(pos+1), ..., t_(pos+n_out); the KV caches then hold the
+ * positions up to pos + n_out - 1, and the next call passes
+ * tokens_out[n_out-1] at position pos + n_out (or ntx_decode_step with
+ * token -1).
+ *   draft_k: 1..7; pos + draft_k < max_ctx; token in [0, V).
+ *   flags: NTX_USE_SKIP (the recorded skip set applies to draft and
+ *   verification), NTX_NO_PERSIST (the draft as the per-op chain).
+ * Needs executed layers in both tiers (NTX_ERR_INVALID_ARG otherwise).  The
+ * call waits for the pass to finish (it reads the tokens back). */
+NTX_API int ntx_decode_spec(ntx_engine* e, int32_t token, int pos, int draft_k, int32_t* tokens_out, int* n_out,
+                            int flags);
+
 /* Profiling: while set, every ntx_decode_step made with NTX_NO_GRAPH records
  * begin_events[k] and end_events[k] (caller-created cudaEvent_t, passed as
  * void*) on the compute stream.  Per-op chain: immediately before and after

@@ -40,7 +40,7 @@ EXPORTS = (
     "ntx_engine_create", "ntx_decode_step", "ntx_engine_skip_mask", "ntx_engine_destroy", "ntx_engine_set_probe",
     "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
     "ntx_persistent_plan", "ntx_layer_layout_mixed", "ntx_engine_device_bytes", "ntx_auto_tier_map",
-    "ntx_memory_budget", "ntx_set_host_wait_limit", "ntx_engine_set_fault",
+    "ntx_memory_budget", "ntx_set_host_wait_limit", "ntx_engine_set_fault", "ntx_decode_spec",
 )
 
 
@@ -100,6 +100,7 @@ def lib():
                                    vp, vp, sz, vp, vp, P(vp)], i32),
             "ntx_decode_step": ([vp, ctypes.c_int32, i32, vp, vp, i32, vp], i32),
             "ntx_engine_skip_mask": ([vp, vp], i32),
+            "ntx_decode_spec": ([vp, ctypes.c_int32, i32, i32, P(ctypes.c_int32), P(i32), i32], i32),
             "ntx_engine_destroy": ([vp], i32),
             "ntx_set_host_wait_limit": ([ctypes.c_uint64], i32),
             "ntx_engine_set_fault": ([vp, i32, ctypes.c_uint64], i32),
@@ -270,6 +271,14 @@ def ntx_engine_create(cfg, layers, tier_map, slot0, slot1, slot_bytes, embed, fi
 
 def ntx_decode_step(engine, token, pos, logits=None, next_token=None, flags=0, cos_out=None):
     _check(lib().ntx_decode_step(engine, token, pos, _p(logits), _p(next_token), flags, _p(cos_out)))
+
+
+def ntx_decode_spec(engine, token, pos, draft_k, flags=0):
+    """Self-speculative step; returns the emitted greedy tokens (a list of 1 .. draft_k + 1)."""
+    out = (ctypes.c_int32 * (draft_k + 1))()
+    n = ctypes.c_int(0)
+    _check(lib().ntx_decode_spec(engine, token, pos, draft_k, out, ctypes.byref(n), flags))
+    return [int(t) for t in out[:n.value]]
 
 
 def ntx_engine_skip_mask(engine, n_layers):

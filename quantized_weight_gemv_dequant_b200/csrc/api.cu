@@ -180,6 +180,8 @@ struct Carve {
 
 int max_parts() { return ntx::sm_count() * 4; }
 
+constexpr int kMaxDraft = 7;  // draft tokens per self-speculative step at most
+
 struct LayerWs {
   float *q, *attn_out, *attn_part, *h1, *u, *stats_in, *stats_o, *stats_down, *cos_tmp;
 };
@@ -476,8 +478,15 @@ struct ntx_engine {
   ntx::PStep pst;
   size_t psmem;
   int pgrid;
-  ntx::PLayer *pl_all, *pl_skip;
+  ntx::PLayer *pl_all, *pl_skip, *pl_draft;
   int n_skip_run;  // executed layers under the skip set
+  // self-speculative decoding: the draft model is the resident layers
+  int n_draft;         // resident layers (the draft's run list without a skip set)
+  bool persist_draft;  // the draft runs as the persistent kernel over pl_draft
+  float* spec_hidden;  // [kMaxDraft + 1][H] residual streams of the verified tokens
+  float* spec_stats;   // [kMaxDraft + 1][2][P * 4] their statistics (ping-pong by layer)
+  int* spec_tok;       // [kMaxDraft + 1] the token and the draft's proposals
+  int* verify_tok;     // [kMaxDraft + 1] the full model's greedy token after each
   unsigned* psync;
   unsigned long long* phase_ts;  // phase probe (kernel-by-kernel steps only)
   size_t phase_ts_words;
@@ -507,9 +516,15 @@ size_t engine_carve(const ntx_model_config* c, uint8_t* base, ntx_engine* e) {
   int* ll = k.take<int>(L);
   ntx::PLayer* pla = k.take<ntx::PLayer>(L);
   ntx::PLayer* pls = k.take<ntx::PLayer>(L);
+  ntx::PLayer* pld = k.take<ntx::PLayer>(L);
   unsigned* psync = k.take<unsigned>(ntx::persist_sync_words(L, c->n_kv_heads));
+  float* sph = k.take<float>((uint64_t)(kMaxDraft + 1) * c->hidden);
+  float* sps = k.take<float>((uint64_t)(kMaxDraft + 1) * 2 * P * 4);
+  int* spt = k.take<int>(16);
+  int* vft = k.take<int>(16);
   if (e) {
-    e->pl_all = pla; e->pl_skip = pls; e->psync = psync;
+    e->pl_all = pla; e->pl_skip = pls; e->pl_draft = pld; e->psync = psync;
+    e->spec_hidden = sph; e->spec_stats = sps; e->spec_tok = spt; e->verify_tok = vft;
     e->hidden = hidden; e->q = q; e->attn_out = ao; e->attn_part = ap; e->h1 = h1; e->u = u;
     e->stats_embed = se; e->stats_o = so; e->stats_down = sd; e->arg_parts = apart; e->cos_int = ci;
     e->logits_int = li; e->params = params; e->token_state = ts; e->layer_list = ll;
@@ -560,15 +575,16 @@ cudaError_t upload_players(ntx_engine* e, const std::vector<int>& list, ntx::PLa
   return cudaMemcpy(dst, t.data(), sizeof(ntx::PLayer) * t.size(), cudaMemcpyHostToDevice);
 }
 
-// The whole step as one persistent kernel (plus the cosine finalisation when asked).
+// The whole step as one persistent kernel (plus the cosine finalisation when
+// asked) over the run list `table` of nrun layers (NULL: the skip set's or all).
 cudaError_t persist_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t* next_token, float* cos_out,
-                            bool calibrate, bool probe) {
+                            bool calibrate, bool probe, const ntx::PLayer* table = nullptr, int ntable = 0) {
   const ntx_model_config& c = e->cfg;
   cudaStream_t s = e->cs;
   const bool sk = use_skip && e->skip_valid;
-  const int nrun = sk ? e->n_skip_run : c.n_layers;
+  const int nrun = table ? ntable : sk ? e->n_skip_run : c.n_layers;
   ntx::PStep st = e->pst;
-  st.layers = sk ? e->pl_skip : e->pl_all;
+  st.layers = table ? table : sk ? e->pl_skip : e->pl_all;
   st.n_layers = nrun;
   st.logits = logits ? logits : e->logits_int;
   st.next_token = next_token;
@@ -598,8 +614,16 @@ cudaError_t persist_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t
 
 // Enqueue the per-token launch sequence (everything after the parameter copy).
 cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t* next_token, float* cos_out,
-                           bool calibrate, bool probe, bool no_persist) {
-  if (e->persist && !no_persist) {
+                           bool calibrate, bool probe, bool no_persist, bool draft = false) {
+  if (draft) {  // the resident layers only (minus the skip set): no host layer, no cosines
+    const bool sk = use_skip && e->skip_valid;
+    if (e->persist_draft && !no_persist && !sk)
+      return persist_enqueue(e, false, logits, next_token, nullptr, false, false, e->pl_draft, e->n_draft);
+    if (e->persist_draft && !no_persist && sk && e->persist_skip)  // the skip run list is all resident
+      return persist_enqueue(e, true, logits, next_token, nullptr, false, false, e->pl_skip, e->n_skip_run);
+    cos_out = nullptr;
+    calibrate = false;
+  } else if (e->persist && !no_persist) {
     const bool sk = use_skip && e->skip_valid;
     if (sk ? e->persist_skip : e->persist_full)
       return persist_enqueue(e, use_skip, logits, next_token, cos_out, calibrate, probe);
@@ -617,7 +641,7 @@ cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t*
   // host-tier layers in execution order
   std::vector<int> host_layers;
   for (int l = 0; l < c.n_layers; ++l)
-    if (e->tier[l] == 1 && !(use_skip && e->skip[l])) host_layers.push_back(l);
+    if (e->tier[l] == 1 && !(use_skip && e->skip[l]) && !draft) host_layers.push_back(l);
   auto issue_copy = [&](int k) -> cudaError_t {
     const int l = host_layers[k], sl = k & 1;
     cudaError_t r = cudaStreamWaitEvent(e->xs, e->slot_free[sl], 0);
@@ -638,7 +662,7 @@ cudaError_t engine_enqueue(ntx_engine* e, bool use_skip, float* logits, int32_t*
   int hk = 0;  // index into host_layers
   std::vector<int> computed;
   for (int l = 0; l < c.n_layers; ++l) {
-    if (use_skip && e->skip[l]) continue;
+    if ((use_skip && e->skip[l]) || (draft && e->tier[l] == 1)) continue;
     const uint8_t* base = static_cast<const uint8_t*>(e->layers[l].base);
     bool on_host = e->tier[l] == 1;
     if (on_host) {
@@ -763,7 +787,8 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
     engine_free(e);
     return fail(NTX_ERR_NOMEM, "ntx_engine_create: pinned parameter block allocation failed (injected)");
   }
-  cudaError_t err = cudaHostAlloc(reinterpret_cast<void**>(&e->pinned), 64 * 4 * sizeof(int), cudaHostAllocDefault);
+  cudaError_t err = cudaHostAlloc(reinterpret_cast<void**>(&e->pinned), (64 * 4 + 64) * sizeof(int),
+                                  cudaHostAllocDefault);
   for (int i = 0; i < 64 && err == cudaSuccess; ++i) err = cudaEventCreateWithFlags(&e->ring_ev[i], cudaEventDisableTiming);
   for (int i = 0; i < 2 && err == cudaSuccess; ++i) {
     err = cudaEventCreateWithFlags(&e->copy_done[i], cudaEventDisableTiming);
@@ -776,7 +801,9 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   // layers, a type pair it is built for, shapes and alignment it handles; it runs the steps whose executed
   // layers are all resident (all steps without a host tier; with one, the steps under a skip set that skips
   // every host layer)
-  e->persist = e->persist_full = e->persist_skip = false;
+  e->persist = e->persist_full = e->persist_skip = e->persist_draft = false;
+  e->n_draft = 0;
+  for (int l = 0; l < cfg->n_layers; ++l) e->n_draft += e->tier[l] == 0;
   int kt[7] = {0, 0, 0, 0, 0, 0, 0};
   kt[ntx::PK_HEAD] = head_qtype;
   bool uniform = true;
@@ -825,6 +852,13 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
           for (int l = 0; l < cfg->n_layers; ++l) all[l] = l;
           err = upload_players(e, all, e->pl_all);
         }
+        std::vector<int> resident;
+        for (int l = 0; l < cfg->n_layers; ++l)
+          if (e->tier[l] == 0) resident.push_back(l);
+        if (err == cudaSuccess && !resident.empty()) {
+          err = upload_players(e, resident, e->pl_draft);
+          e->persist_draft = err == cudaSuccess;
+        }
         if (err == cudaSuccess) {
           e->pst = st;
           e->psmem = psm;
@@ -849,6 +883,25 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   return NTX_OK;
 }
 
+namespace {
+
+// Step parameters (position, token) through a ring of pinned host slots to the
+// device words the kernels read, on the compute stream.
+int enqueue_params(ntx_engine* e, int pos, int token) {
+  const int slot = e->ring_pos;
+  cudaError_t err = wait_event(e->ring_ev[slot]);
+  if (err != cudaSuccess) return wait_fail(err, "param ring");
+  e->ring_pos = (e->ring_pos + 1) % 64;
+  e->pinned[slot * 4 + 0] = pos;
+  e->pinned[slot * 4 + 1] = token;
+  err = cudaMemcpyAsync(e->params, e->pinned + slot * 4, 2 * sizeof(int), cudaMemcpyHostToDevice, e->cs);
+  if (err == cudaSuccess) err = cudaEventRecord(e->ring_ev[slot], e->cs);
+  if (err != cudaSuccess) return cuda_fail(err, "param copy");
+  return NTX_OK;
+}
+
+}  // namespace
+
 extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* logits, int32_t* next_token, int flags,
                                float* cos_out) {
   if (!e) return fail(NTX_ERR_INVALID_ARG, "engine is NULL");
@@ -864,9 +917,6 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
   cudaGetDevice(&cur);
   if (cur != e->dev) return fail(NTX_ERR_INVALID_ARG, "engine was created on device %d, current is %d", e->dev, cur);
 
-  // step parameters: pinned ring slot -> device
-  const int slot = e->ring_pos;
-  e->ring_pos = (e->ring_pos + 1) % 64;
   // a step that streams host layers: the copies are submitted below (injected failure: nothing enqueued)
   if (fault("h2d_submit")) {
     bool streams = false;
@@ -874,13 +924,10 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
       streams = e->tier[l] == 1 && !(use_skip && e->skip[l]);
     if (streams) return fail(NTX_ERR_CUDA, "ntx_decode_step: host-to-device copy submission failed (injected)");
   }
-  cudaError_t err = wait_event(e->ring_ev[slot]);
-  if (err != cudaSuccess) return wait_fail(err, "param ring");
-  e->pinned[slot * 4 + 0] = pos;
-  e->pinned[slot * 4 + 1] = token;
-  err = cudaMemcpyAsync(e->params, e->pinned + slot * 4, 2 * sizeof(int), cudaMemcpyHostToDevice, e->cs);
-  if (err == cudaSuccess) err = cudaEventRecord(e->ring_ev[slot], e->cs);
-  if (err != cudaSuccess) return cuda_fail(err, "param copy");
+  // step parameters: pinned ring slot -> device
+  int rc = enqueue_params(e, pos, token);
+  if (rc) return rc;
+  cudaError_t err = cudaSuccess;
 
   if ((flags & NTX_NO_GRAPH) || calibrate) {
     err = engine_enqueue(e, use_skip, logits, next_token, cos_out, calibrate, (flags & NTX_NO_GRAPH) != 0,
@@ -943,6 +990,152 @@ extern "C" int ntx_decode_step(ntx_engine* e, int32_t token, int pos, float* log
   return NTX_OK;
 }
 
+namespace {
+
+// The verification pass of a self-speculative step: the tokens spec_tok[0..k]
+// at positions pos..pos+k through every executed layer, layer by layer (each
+// host layer crosses the link once for all k+1 tokens), then the head and the
+// greedy token of each into verify_tok[0..k].  The kernels and their order
+// for one token are those of an ordinary per-op step, so each token's logits
+// are the ones an ordinary step at that position would give.
+cudaError_t verify_enqueue(ntx_engine* e, int pos, int k, bool use_skip) {
+  const ntx_model_config& c = e->cfg;
+  cudaStream_t s = e->cs;
+  const bool pdl = true;
+  const int P4 = max_parts() * 4;
+  const int nparts = ntx::layer_stats_parts(c.hidden);
+  auto hid = [&](int t) { return e->spec_hidden + (int64_t)t * c.hidden; };
+  auto stats = [&](int t, int par) { return e->spec_stats + ((int64_t)t * 2 + par) * P4; };
+  cudaError_t err = cudaSuccess;
+  for (int t = 0; t <= k && err == cudaSuccess; ++t)
+    err = ntx::launch_embed(e->embed, c.hidden, c.vocab, e->spec_tok + t, e->token_state, hid(t), stats(t, 0),
+                            kEmbedParts, s, pdl);
+  if (err != cudaSuccess) return err;
+  std::vector<int> host_layers;
+  for (int l = 0; l < c.n_layers; ++l)
+    if (e->tier[l] == 1 && !(use_skip && e->skip[l])) host_layers.push_back(l);
+  auto issue_copy = [&](int j) -> cudaError_t {
+    const int l = host_layers[j], sl = j & 1;
+    cudaError_t r = cudaStreamWaitEvent(e->xs, e->slot_free[sl], 0);
+    if (r == cudaSuccess)
+      r = cudaMemcpyAsync(e->slot[sl], e->layers[l].base, e->extent[l], cudaMemcpyHostToDevice, e->xs);
+    if (r == cudaSuccess) r = cudaEventRecord(e->copy_done[sl], e->xs);
+    return r;
+  };
+  if (!host_layers.empty()) {
+    err = cudaEventRecord(e->fork_ev, s);
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(e->xs, e->fork_ev, 0);
+    if (err == cudaSuccess) err = cudaEventRecord(e->slot_free[0], s);
+    if (err == cudaSuccess) err = cudaEventRecord(e->slot_free[1], s);
+    for (int j = 0; j < (int)host_layers.size() && j < 2 && err == cudaSuccess; ++j) err = issue_copy(j);
+    if (err != cudaSuccess) return err;
+  }
+  int hk = 0, par = 0, n_in = kEmbedParts;
+  for (int l = 0; l < c.n_layers; ++l) {
+    if (use_skip && e->skip[l]) continue;
+    const uint8_t* base = static_cast<const uint8_t*>(e->layers[l].base);
+    const bool on_host = e->tier[l] == 1;
+    if (on_host) {
+      err = cudaStreamWaitEvent(s, e->copy_done[hk & 1], 0);
+      if (err != cudaSuccess) return err;
+      base = e->slot[hk & 1];
+    }
+    for (int t = 0; t <= k; ++t) {
+      ntx::LayerArgs a = layer_args(&c, base, &e->layers[l]);
+      a.k_cache = e->kc[l]; a.v_cache = e->vc[l]; a.hidden = hid(t);
+      a.stats_in = stats(t, par); a.n_stats_in = n_in;
+      a.stats_o = e->stats_o;
+      a.stats_down = stats(t, par ^ 1);
+      a.q = e->q; a.attn_out = e->attn_out; a.attn_part = e->attn_part; a.h1 = e->h1; a.u = e->u;
+      a.pos = pos + t; a.pos_dev = nullptr; a.n_split = e->n_split;
+      a.attn_cluster = ntx::attn_cluster_size(c.n_heads, c.n_kv_heads, c.max_ctx);
+      err = ntx::launch_layer(a, s, pdl);
+      if (err != cudaSuccess) return err;
+    }
+    par ^= 1;
+    n_in = nparts;
+    if (on_host) {
+      err = cudaEventRecord(e->slot_free[hk & 1], s);
+      if (err == cudaSuccess && hk + 2 < (int)host_layers.size()) err = issue_copy(hk + 2);
+      if (err != cudaSuccess) return err;
+      ++hk;
+    }
+  }
+  if (!host_layers.empty()) {
+    err = cudaEventRecord(e->join_ev, e->xs);
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(s, e->join_ev, 0);
+    if (err != cudaSuccess) return err;
+  }
+  for (int t = 0; t <= k && err == cudaSuccess; ++t) {
+    err = ntx::launch_head(e->head_qtype, e->head, c.vocab, c.hidden, hid(t), e->final_norm, stats(t, par), n_in,
+                           c.eps, e->logits_int, e->arg_parts, s, pdl);
+    if (err == cudaSuccess)
+      err = ntx::launch_argmax_finalize(e->arg_parts, ntx::head_parts(c.vocab), e->token_state, e->verify_tok + t, s,
+                                        pdl);
+  }
+  return err;
+}
+
+}  // namespace
+
+extern "C" int ntx_decode_spec(ntx_engine* e, int32_t token, int pos, int draft_k, int32_t* tokens_out, int* n_out,
+                               int flags) {
+  if (!e || !tokens_out || !n_out) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  const ntx_model_config& c = e->cfg;
+  if (draft_k < 1 || draft_k > kMaxDraft) return fail(NTX_ERR_INVALID_ARG, "draft_k %d outside [1, %d]", draft_k, kMaxDraft);
+  if (pos < 0 || pos + draft_k >= c.max_ctx)
+    return fail(NTX_ERR_SHAPE, "positions %d..%d outside [0, max_ctx=%d)", pos, pos + draft_k, c.max_ctx);
+  if (token < 0 || token >= c.vocab) return fail(NTX_ERR_INVALID_ARG, "token %d outside [0, vocab)", token);
+  if (flags & ~(NTX_USE_SKIP | NTX_NO_PERSIST)) return fail(NTX_ERR_INVALID_ARG, "unknown flags");
+  const bool use_skip = (flags & NTX_USE_SKIP) && e->skip_valid;
+  int n_res = 0, n_host = 0;
+  for (int l = 0; l < c.n_layers; ++l) {
+    if (use_skip && e->skip[l]) continue;
+    if (e->tier[l] == 0) ++n_res;
+    else ++n_host;
+  }
+  if (n_res == 0 || n_host == 0)
+    return fail(NTX_ERR_INVALID_ARG,
+                "self-speculative decoding needs executed layers in both tiers (the resident ones are the draft)");
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != e->dev) return fail(NTX_ERR_INVALID_ARG, "engine was created on device %d, current is %d", e->dev, cur);
+  if (fault("h2d_submit")) return fail(NTX_ERR_CUDA, "ntx_decode_spec: host-to-device copy submission failed (injected)");
+  cudaStream_t s = e->cs;
+  int* hp = e->pinned + 64 * 4;  // [0..15] read-back area, [16] token
+  // the pinned read-back area is reused: the previous call's copies have completed (it waited for them)
+  hp[16] = token;
+  cudaError_t err = cudaMemcpyAsync(e->spec_tok, hp + 16, sizeof(int), cudaMemcpyHostToDevice, s);
+  if (err != cudaSuccess) return cuda_fail(err, "ntx_decode_spec: token copy");
+  // draft: k steps of the resident layers, each proposing the next token
+  for (int i = 0; i < draft_k; ++i) {
+    int rc = enqueue_params(e, pos + i, i == 0 ? token : -1);
+    if (rc) return rc;
+    err = engine_enqueue(e, use_skip, nullptr, e->spec_tok + i + 1, nullptr, false, false,
+                         (flags & NTX_NO_PERSIST) != 0, true);
+    if (err != cudaSuccess) return cuda_fail(err, "ntx_decode_spec: draft step");
+  }
+  // verification of the token and the k proposals by the whole model
+  err = verify_enqueue(e, pos, draft_k, use_skip);
+  if (err != cudaSuccess) return cuda_fail(err, "ntx_decode_spec: verification");
+  err = cudaMemcpyAsync(hp, e->spec_tok, sizeof(int) * (draft_k + 1), cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess)
+    err = cudaMemcpyAsync(hp + 8, e->verify_tok, sizeof(int) * (draft_k + 1), cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess) err = wait_stream(s, e->sync_ev);
+  if (err != cudaSuccess) return wait_fail(err, "ntx_decode_spec: read-back");
+  // accept the longest prefix of proposals the whole model agrees with, then its own next token
+  int n = 0;
+  while (n < draft_k && hp[1 + n] == hp[8 + n]) ++n;
+  for (int i = 0; i <= n; ++i) tokens_out[i] = hp[8 + i];
+  *n_out = n + 1;
+  // the engine's greedy state continues from the last emitted token
+  err = cudaMemcpyAsync(e->token_state, hp + 8 + n, sizeof(int), cudaMemcpyHostToDevice, s);
+  if (err == cudaSuccess) err = wait_stream(s, e->sync_ev);
+  if (err != cudaSuccess) return wait_fail(err, "ntx_decode_spec: token state");
+  e->launches = -1;  // not a single-step launch sequence
+  return NTX_OK;
+}
+
 extern "C" int ntx_engine_skip_mask(ntx_engine* e, uint8_t* mask_host) {
   if (!e || !mask_host) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
   int n = 0;
@@ -1000,6 +1193,7 @@ extern "C" int ntx_persistent_plan(const ntx_model_config* cfg, int qtype, int* 
 
 extern "C" int ntx_engine_launches_per_step(ntx_engine* e) {
   if (!e) return fail(NTX_ERR_INVALID_ARG, "engine is NULL");
+  if (e->launches < 0) return fail(NTX_ERR_INVALID_ARG, "the last call was a self-speculative step");
   return e->launches;
 }
 

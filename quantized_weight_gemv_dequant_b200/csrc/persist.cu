@@ -336,12 +336,20 @@ __device__ bool pwait_a(uint32_t bar, uint32_t parity, const volatile int* cta_a
 // Streams every weight stage of this CTA, phase after phase, into the ring.
 // It waits only for slots to be released: weights never depend on
 // activations, so the stream runs ahead across phase boundaries.
+//
+// Beyond the ring, the warp keeps a window of pf_stages further stages
+// requested into L2 (bulk prefetch, no completion to wait for): while the
+// consumers wait at a phase boundary and the ring is full, HBM keeps
+// streaming those stages into L2, and the ring refills from L2 (several times
+// the HBM rate) once the consumers resume.  Each weight byte still crosses
+// HBM once.
 struct Copier {
   const PStep& st;
   PSmem sm;
   int lane, np, n_slots, slot_bytes;
   uint64_t policy;
-  PIssue it;
+  PIssue it;   // next stage into the ring
+  PIssue pit;  // next stage into L2, pf_stages ahead of it
   long issued, done;
 
   __device__ Copier(const PStep& st_, PSmem sm_, int lane_, int np_)
@@ -365,6 +373,14 @@ struct Copier {
     ++issued;
   }
 
+  __device__ __forceinline__ void prefetch_one() {
+    if (!pit.valid(np)) return;
+    const int64_t rs = pit.r0 + (int64_t)pit.j * pit.TR;
+    const int nr = (int)min64(pit.TR, pit.r1 - rs);
+    for (int r = lane; r < nr; r += 32) l2_prefetch(pit.row(rs + r), (uint32_t)pit.rb);
+    pit.advance(st, np);
+  }
+
   // Lets every issued copy land (bounded) before the warp exits.
   __device__ void drain() {
     if (lane == 0) {
@@ -381,6 +397,8 @@ struct Copier {
 
   __device__ void run() {
     for (int k = 0; k < n_slots && it.valid(np); ++k) issue(k);
+    pit = it;
+    for (int k = 0; k < st.pf_stages; ++k) prefetch_one();
     int s = 0;
     uint32_t ph = 0;
     while (it.valid(np)) {
@@ -392,6 +410,7 @@ struct Copier {
         break;
       }
       issue(s);
+      prefetch_one();
       ++done;
       if (++s == n_slots) { s = 0; ph ^= 1u; }
     }
@@ -1378,6 +1397,7 @@ int persist_plan(const int* kt, int H, int Hq, int Hkv, int D, int F, int64_t V,
   }
   st->slot_bytes = best_Z;
   st->n_slots = best_S;
+  st->pf_stages = (kPPrefetchBytes + best_Z - 1) / best_Z;
   st->xstage_bytes = (xbz + 15) / 16 * 16;
   st->red_floats = (rf + 3) / 4 * 4;  // keeps the tables after it 16-byte aligned
   *smem = psmem_bytes(best_S, best_Z, st->xstage_bytes, st->red_floats, n_layers);

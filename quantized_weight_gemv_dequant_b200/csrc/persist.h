@@ -8,6 +8,10 @@
 namespace ntx {
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // the persistent kernel's wait limit unless a test lowers it
+#ifndef NTX_PF_BYTES
+#define NTX_PF_BYTES (192 * 1024)
+#endif
+constexpr int kPPrefetchBytes = NTX_PF_BYTES;  // weight bytes per CTA requested into L2 beyond the ring
 constexpr int kPConsumers = 14;      // consumer warps per CTA (plus an epilogue warp and a copy warp)
 constexpr int kPRed = 8;             // depth of the row-partial ring between consumers and the epilogue warp
 constexpr int kPPartsPerLane = 8;    // CTAs at most: 32 * this (sum-of-squares partials read per lane)
@@ -60,6 +64,7 @@ struct PStep {
   PGeom g[7];          // indexed by PKind
   int qt[7];           // block type of each GEMV phase kind (indexed by PKind)
   int slot_bytes, n_slots, xstage_bytes, red_floats;
+  int pf_stages;  // stages of weight rows kept requested into L2 ahead of the ring
   int* status;  // device status word
   uint64_t wait_ns;  // limit on every wait of the kernel (nanoseconds of %globaltimer)
   int stall_cta;     // a CTA that withholds its embed publication (failure-path tests), -1: none
