@@ -16,7 +16,6 @@ constexpr int kPConsumers = 14;      // consumer warps per CTA (plus an epilogue
 constexpr int kPRed = 8;             // depth of the row-partial ring between consumers and the epilogue warp
 constexpr int kPPartsPerLane = 8;    // CTAs at most: 32 * this (sum-of-squares partials read per lane)
 constexpr int kPMaxTR = 32;          // rows per ring slot at most
-constexpr int kPChunk = 64;          // attention positions per K/V tile
 constexpr int kPMinSplit = 128;      // attention positions per (KV head, split) unit at least, where possible
 constexpr int kPSplitsPerRound = 4;  // split (m, l) loads per lane in flight during the merge
 constexpr int kPD = 128;             // head dimension
