@@ -78,7 +78,7 @@ WORKLOADS = {
                           model="MODEL_70B", qtype=14, head_qtype=14, workload_id=5, max_ctx=2080, n_prior=2048,
                           prompt=1),
 }
-QNAME = {8: "Q8_0", 14: "Q6_K", 2: "Q4_0"}
+QNAME = {8: "Q8_0", 14: "Q6_K", 2: "Q4_0", 12: "Q4_K", 13: "Q5_K", 1: "F16", 0: "F32"}
 
 
 # ---------------------------------------------------------------- distributed
@@ -318,14 +318,14 @@ class Run:
         spans = np.array(spans)
         H, F, Hq, Hkv, D = d["hidden"], d["ffn"], d["n_heads"], d["n_kv_heads"], d["head_dim"]
         from synthgen import workloads as wl
-        kinds = {"q/k/v (RMSNorm, RoPE, KV append)": (0, (Hq + 2 * Hkv) * D, H),
-                 "o (+ residual)": (2, H, Hq * D),
-                 "gate/up (RMSNorm, SwiGLU)": (3, 2 * F, H),
-                 "down (+ residual, cosine statistics)": (4, H, F)}
+        kinds = {"q/k/v (RMSNorm, RoPE, KV append)": (0, (Hq + 2 * Hkv) * D, H, 0),
+                 "o (+ residual)": (2, H, Hq * D, 3),
+                 "gate/up (RMSNorm, SwiGLU)": (3, 2 * F, H, 4),
+                 "down (+ residual, cosine statistics)": (4, H, F, 6)}
         out = []
-        for name, (j, M, K) in kinds.items():
+        for name, (j, M, K, mi) in kinds.items():
             us = float(spans[:, [1 + 5 * k + j for k in range(L_run)]].mean())
-            by = wl.mat_bytes(qt, M, K)
+            by = wl.mat_bytes(wl.mat_types(qt)[mi], M, K)
             out.append({"phase": name, "M": M, "K": K, "weight_bytes": by, "us": round(us, 3),
                         "GBs": round(by / (us * 1e-6) / 1e9, 1), "frac": round(by / (us * 1e-6) / 1e9 / peak, 4)})
         us = float(spans[:, 1 + 5 * L_run].mean())
@@ -609,6 +609,26 @@ def run_70b(args, dist, ntx, torch, sg, wl, peak, peak_kind, dev_index):
                       "note": ("every host layer is skipped: nothing crosses the link and the step runs as one "
                                "persistent kernel over the resident executed layers") if not host_run else
                               "the executed host layers stream through the slots"}
+    # self-speculative decoding on the tiered engine: the resident layers 0-39 draft 3 tokens, the whole
+    # model verifies the 4 in one pass that streams layers 40-79 once
+    rb.steps([start], [p0])
+    rb.cs.synchronize()
+    n_calls, k = min(args.steps, 4), 3
+    tok, pos, emitted, acc = start, p0 + 1, 0, []
+    t0 = time.perf_counter()
+    for _ in range(n_calls):
+        got = ntx.ntx_decode_spec(rb.eng, tok, pos, k)
+        acc.append(len(got) - 1)
+        emitted += len(got)
+        pos += len(got)
+        tok = got[-1]
+    spec_s = time.perf_counter() - t0
+    b["self_spec"] = {"value": round(emitted / spec_s, 3), "unit": "tok/s", "draft_k": k, "calls": n_calls,
+                      "tokens": emitted, "accepted_per_call": acc,
+                      "how": "ntx_decode_spec on the tiered engine (draft = resident layers 0-39 + head, "
+                             "verification streams layers 40-79 once per call); host wall clock, the call "
+                             "waits for its tokens",
+                      "note": "random-init weights: the draft rarely agrees with the whole model"}
     rb.close()
     del rb
     res["5b_tiered"] = b
@@ -616,6 +636,27 @@ def run_70b(args, dist, ntx, torch, sg, wl, peak, peak_kind, dev_index):
     if not args.no_cpu_baseline and dist.rank == 0 and dist.world == 1:
         res["cpu_baseline"] = cpu_baseline_70b(m, d, wk, start)
     del m
+    torch.cuda.empty_cache()
+
+    # ---- 5c: the same shapes as Q4_K_M (Q4_K matrices, Q6_K down projections and head), resident
+    qm = wl.Q4_K_M
+    m = DeviceModel(d, qm, wl.Q4_K_M_HEAD, sd, wk["max_ctx"], wk["n_prior"], source="device")
+    rc = Run(ntx, torch, m, d, L, qm, wl.Q4_K_M_HEAD, wk["max_ctx"], [0] * L)
+    rc.steps([start], [p0])
+    rc.steps([-1] * args.warmup, [pos_of(i) for i in range(args.warmup)])
+    ms_c, kms_c = rc.timed([pos_of(args.warmup + i) for i in range(n_a)])
+    c_bytes = wl.bytes_per_token(d, qm, wl.Q4_K_M_HEAD, n_ctx)
+    res["5c_q4_k_m_resident"] = {
+        "value": round(n_a / (ms_c / 1e3), 3), "unit": "tok/s", "steps": n_a, "ms_per_step": round(ms_c / n_a, 4),
+        "weights": "Q4_K (wq wk wv wo wg wu), Q6_K (wd, head)",
+        "launches_per_step": ntx.ntx_engine_launches_per_step(rc.eng),
+        "roofline": roofline(kms_c, c_bytes, peak, peak_kind, 12, None, ms_c / n_a, "5c's timed region"),
+        "decode_roofline": {"bytes_per_token": c_bytes, "roofline_tok_s": round(peak * 1e9 / c_bytes, 2),
+                            "frac": round((n_a / (ms_c / 1e3)) / (peak * 1e9 / c_bytes), 4)},
+        "gemv_in_step": rc.phases([pos_of(args.warmup + n_a + i) for i in range(4)], L, d, qm, wl.Q4_K_M_HEAD,
+                                  peak)}
+    rc.close()
+    del rc, m
     torch.cuda.empty_cache()
     return res
 
@@ -689,7 +730,10 @@ GEMV_SHAPES = [(8, 4096, 4096, "Q8_0 GEMV 4096x4096, batch 1")] + \
     [(2, M, K, "Q4_0 GEMV sweep over Llama-3-8B projection shapes, batch 1") for M, K in
      ((4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336))] + \
     [(14, M, K, "Q6_K GEMV over Llama-3-70B projection shapes, batch 1") for M, K in
-     ((8192, 8192), (28672, 8192), (8192, 28672))]
+     ((8192, 8192), (28672, 8192), (8192, 28672))] + \
+    [(12, M, K, "Q4_K GEMV over Llama-3-70B projection shapes, batch 1") for M, K in
+     ((8192, 8192), (28672, 8192), (8192, 28672))] + \
+    [(13, 8192, 8192, "Q5_K GEMV 8192x8192, batch 1"), (1, 4096, 4096, "F16 GEMV 4096x4096, batch 1")]
 
 
 def gemv_sweep(ntx, sg, wl, torch, peak):
