@@ -12,7 +12,8 @@ from synthgen import workloads as wl
 SMEM_MAX = 227 * 1024
 CONSUMERS = 14
 SLICE = 2048
-BLOCK = {ntx.NTX_Q8_0: (32, 34), ntx.NTX_Q4_0: (32, 18), ntx.NTX_Q6_K: (256, 210)}
+BLOCK = {ntx.NTX_Q8_0: (32, 34), ntx.NTX_Q4_0: (32, 18), ntx.NTX_Q6_K: (256, 210), ntx.NTX_Q4_K: (256, 144),
+         ntx.NTX_Q5_K: (256, 176)}
 PHASES = ["qkv", "o", "gu", "down", "head"]
 PAIRED = {"qkv", "gu"}
 
@@ -40,6 +41,9 @@ CASES = [
     ("llama8b-q4_0", wl.MODEL_8B, ntx.NTX_Q4_0, 144),
     ("llama70b", wl.MODEL_70B, ntx.NTX_Q6_K, 2080),
     ("tiny-q6_k", TINY_Q6, ntx.NTX_Q6_K, 64),
+    ("llama70b-q4_k", wl.MODEL_70B, ntx.NTX_Q4_K, 2080),
+    ("llama70b-q5_k", wl.MODEL_70B, ntx.NTX_Q5_K, 2080),
+    ("llama8b-q4_k", wl.MODEL_8B, ntx.NTX_Q4_K, 144),
 ]
 
 
@@ -77,6 +81,8 @@ def test_plan_argument_errors():
     L = ntx.lib()
     cfg = _cfg(wl.MODEL_8B, 144)
     assert L.ntx_persistent_plan(None, ntx.NTX_Q8_0, None, None, None, None) == ntx.NTX_ERR_INVALID_ARG
+    # F16 / F32 layers run on the per-op chain only
+    assert L.ntx_persistent_plan(cfg, ntx.NTX_F16, None, None, None, None) == ntx.NTX_ERR_SHAPE
     assert L.ntx_persistent_plan(cfg, 99, None, None, None, None) == ntx.NTX_ERR_QTYPE
     bad = dict(wl.MODEL_8B, head_dim=64)  # the persistent kernel takes head_dim 128 only
     assert L.ntx_persistent_plan(_cfg(bad, 144), ntx.NTX_Q8_0, None, None, None, None) == ntx.NTX_ERR_SHAPE
