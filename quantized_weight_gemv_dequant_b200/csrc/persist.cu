@@ -266,20 +266,24 @@ __device__ __forceinline__ PSmem psmem_at(uint8_t* base, int S, int Z, int XB, i
 }
 
 // Attention scratch inside the x staging region (consumer warps only).
+// A warp's partial result for one head: unnormalised output o[0..127] (16-byte
+// aligned for the lanes' float4 stores), then max, sum and two pad floats.
+constexpr int kWpStride = kPD + 4;
+constexpr int kWpMax = kPD, kWpSum = kPD + 1;
 struct AttnSmem {
   float* qs;  // [G][kPD] the unit's query heads, scaled by 1/sqrt(D)
-  float* wp;  // [kPConsumers][4][kPD + 2] each warp's (max, sum, unnormalised output) for its <= 4 heads
+  float* wp;  // [kPConsumers][4][kWpStride] each warp's partial results for its <= 4 heads
   float* ml;  // [G][2] the unit's (max, sum) per head
   float* sw;  // [G][n_split] merge weights
 };
 __host__ __device__ inline size_t attn_smem_bytes(int G, int ns) {
-  return (size_t)G * kPD * 4 + (size_t)kPConsumers * 4 * (kPD + 2) * 4 + (size_t)G * 2 * 4 + (size_t)G * ns * 4;
+  return (size_t)G * kPD * 4 + (size_t)kPConsumers * 4 * kWpStride * 4 + (size_t)G * 2 * 4 + (size_t)G * ns * 4;
 }
 __device__ __forceinline__ AttnSmem attn_smem(uint8_t* base, int G) {
   AttnSmem a;
-  a.qs = reinterpret_cast<float*>(base);
-  a.wp = a.qs + G * kPD;
-  a.ml = a.wp + kPConsumers * 4 * (kPD + 2);
+  a.qs = reinterpret_cast<float*>(base);                   // base 16-byte aligned; G * 512 bytes
+  a.wp = a.qs + G * kPD;                                   // entries of 528 bytes: every o[] 16-byte aligned
+  a.ml = a.wp + kPConsumers * 4 * kWpStride;
   a.sw = a.ml + 2 * G;
   return a;
 }
@@ -903,11 +907,11 @@ struct Consumer {
       if (w_on) {
 #pragma unroll
         for (int h = 0; h < GW; ++h) {
-          float* dst = a.wp + ((size_t)warp * 4 + h) * (kPD + 2);
-          *reinterpret_cast<float4*>(dst + 2 + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
+          float* dst = a.wp + ((size_t)warp * 4 + h) * kWpStride;
+          *reinterpret_cast<float4*>(dst + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
           if (lane == 0) {
-            dst[0] = m[h];
-            dst[1] = l[h];
+            dst[kWpMax] = m[h];
+            dst[kWpSum] = l[h];
           }
         }
       }
@@ -917,14 +921,14 @@ struct Consumer {
         const int h = idx / kPD, d = idx % kPD;
         const int g = h / GW, hl = h % GW;
         float M = -INFINITY;
-        for (int w = 0; w < WPG; ++w) M = fmaxf(M, a.wp[((size_t)(w * NH + g) * 4 + hl) * (kPD + 2)]);
+        for (int w = 0; w < WPG; ++w) M = fmaxf(M, a.wp[((size_t)(w * NH + g) * 4 + hl) * kWpStride + kWpMax]);
         float Ls = 0.f, O = 0.f;
         for (int w = 0; w < WPG; ++w) {
-          const float* src = a.wp + ((size_t)(w * NH + g) * 4 + hl) * (kPD + 2);
-          const float mw = src[0];
+          const float* src = a.wp + ((size_t)(w * NH + g) * 4 + hl) * kWpStride;
+          const float mw = src[kWpMax];
           const float f = mw == -INFINITY ? 0.f : expf(mw - M);
-          Ls = fmaf(src[1], f, Ls);
-          O = fmaf(src[2 + d], f, O);
+          Ls = fmaf(src[kWpSum], f, Ls);
+          O = fmaf(src[d], f, O);
         }
         if (ns == 1) {
           st.attn_out[(int64_t)(kvh * G + h) * kPD + d] = O / Ls;
