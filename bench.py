@@ -77,8 +77,20 @@ WORKLOADS = {
                                "pinned host RAM streamed through two device slots",
                           model="MODEL_70B", qtype=14, head_qtype=14, workload_id=5, max_ctx=2080, n_prior=2048,
                           prompt=1),
+    "llama70b-q4_k_m": dict(desc="Llama-3-70B-shaped 80-layer Q4_K_M model (Q4_K matrices, Q6_K down projections "
+                                 "and head), 2048 prior KV positions, greedy batch-1 decode from position 2048, "
+                                 "resident",
+                            model="MODEL_70B", qtype=(12, 12, 12, 12, 12, 12, 14), head_qtype=14, workload_id=5,
+                            max_ctx=2080, n_prior=2048, prompt=1),
 }
 QNAME = {8: "Q8_0", 14: "Q6_K", 2: "Q4_0", 12: "Q4_K", 13: "Q5_K", 1: "F16", 0: "F32"}
+
+
+def qname(qt) -> str:
+    """Name of one block type, or of a per-matrix mix (wq..wd)."""
+    if isinstance(qt, (list, tuple)):
+        return "Q4_K_M" if tuple(qt) == (12, 12, 12, 12, 12, 12, 14) else "/".join(QNAME[t] for t in qt)
+    return QNAME[qt]
 
 
 # ---------------------------------------------------------------- distributed
@@ -373,8 +385,8 @@ def run_ntx(args, dist: Dist):
     from synthgen import workloads as wl
     from synthgen.devmodel import DeviceModel
 
-    wk = WORKLOADS["llama8b-q8_0"]
-    d = dict(wl.MODEL_8B)
+    wk = WORKLOADS[args.workload]
+    d = dict(getattr(wl, wk["model"]))
     if args.layers is not None:
         d["n_layers"] = args.layers
     L = d["n_layers"]
@@ -468,7 +480,7 @@ def run_ntx(args, dist: Dist):
 
     # ------------------------------------------------------------ 70B configs
     configs = None
-    if not args.no_70b and args.layers is None and dist.world == 1:
+    if not args.no_70b and args.layers is None and dist.world == 1 and args.workload == "llama8b-q8_0":
         configs = run_70b(args, dist, ntx, torch, sg, wl, peak, peak_kind, dev_index)
 
     bpt = wl.bytes_per_token(d, qt, hqt, p_first + span // 2)
@@ -477,7 +489,7 @@ def run_ntx(args, dist: Dist):
         "metric": METRIC, "value": round(value, 3), "unit": "tok/s", "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; random-init weights of the named shapes)",
-        "config": {"workload": desc, "weights": QNAME[qt], "layers": L, "hidden": d["hidden"], "ffn": d["ffn"],
+        "config": {"workload": desc, "weights": qname(qt), "layers": L, "hidden": d["hidden"], "ffn": d["ffn"],
                    "vocab": d["vocab"], "batch": 1,
                    "parallelism": f"replicas x{dist.world}" if dist.world > 1 else "single GPU",
                    "l2": "weights per step >> 126 MB L2 (inputs larger than L2; no flush)",
@@ -886,7 +898,7 @@ def run_reference(args, world):
             "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded; random-init weights of the named shapes)",
-            "config": {"workload": desc, "weights": QNAME[qt], "layers": L, "hidden": H, "ffn": d["ffn"],
+            "config": {"workload": desc, "weights": qname(qt), "layers": L, "hidden": H, "ffn": d["ffn"],
                        "vocab": V, "batch": 1, "parallelism": "single process, host threads",
                        "l2": "n/a (host)", "graph": "n/a (host)"},
             "impl": "reference",
@@ -904,6 +916,9 @@ def main():
     ap.add_argument("--steps", type=int, default=128)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ntx", "reference"], default="ntx")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama8b-q8_0",
+                    help="the model of the headline line (profiling: the 70B models with --layers); the 70B "
+                         "configurations are added only to the default workload's line")
     ap.add_argument("--no-gemv", action="store_true", help="skip the standalone quantized GEMV sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-chain", action="store_true", help="skip timing the per-op kernel chain for comparison")
