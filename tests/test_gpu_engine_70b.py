@@ -89,3 +89,33 @@ def test_engine_llama70b_q6_k_resident_and_tiered_with_skip():
                                     fed[1], 2049, skip=mask, nthreads=nt)
         check_logits(lg1[0], ref1, int(nx1[0]), 1)
         print(f"{name}: skipped {sum(mask)}/{L} layers at tau 0.98")
+
+
+def test_engine_llama70b_q4_k_m_resident_persistent():
+    """The 70B shapes as Q4_K_M (Q4_K matrices, Q6_K down projections and head):
+    the persistent kernel with two block types (Q4_K phases over 4 K-slices,
+    the Q6_K down projection over 14), checked teacher-forced for 2 steps."""
+    d = dict(wl.MODEL_70B)
+    L = d["n_layers"]
+    sd = wl.seed(5)
+    m = DeviceModel(d, wl.Q4_K_M, wl.Q4_K_M_HEAD, sd, max_ctx=2080, n_prior=2048, source="device")
+    for l in (0, L - 1):
+        t = m.host_layer_tensors(l)
+        for (name, (M, K)), qt in zip(wl.mat_shapes(d).items(), wl.Q4_K_M):
+            ref = sg.quant_rows(qt, sd, wl.tensor_name(l, name), M, K, sigma=wl.W_SIGMA, row0=7, nrows=1)
+            assert np.array_equal(t[name][7], ref[0]), (l, name)
+    prompt = [int(sg.tokens(sd, "prompt", 1, d["vocab"])[0])]
+    e = Engine(m)
+    lg, fed, nx, _ = e.run(prompt + [-1], pos0=2048)
+    launches = ntx.ntx_engine_launches_per_step(e.h)
+    e.close()
+    assert launches == 1
+    ocfg = oracle.make_config(d["hidden"], d["n_heads"], d["n_kv_heads"], d["head_dim"], d["ffn"], d["vocab"], L,
+                              d["eps"], d["theta"], 2080)
+    emb, fn, head = m.host_embed(), m.host_final_norm(), m.host_head()
+    kcs, vcs = zip(*[m.host_kv(l) for l in range(L)])
+    kcs, vcs = [k.copy() for k in kcs], [v.copy() for v in vcs]
+    for s in range(2):
+        ref, _ = oracle.model_step(ocfg, wl.Q4_K_M, m.host_layer_tensors, wl.Q4_K_M_HEAD, head, fn, emb, kcs, vcs,
+                                   fed[s], 2048 + s, nthreads=os.cpu_count())
+        check_logits(lg[s], ref, int(nx[s]), s)
