@@ -119,6 +119,12 @@ __device__ __forceinline__ void bulk_g2s_nohint(void* dst, const void* src, uint
                : "memory");
 }
 
+// Bulk prefetch into L2 (16-byte aligned address, size a multiple of 16); no
+// completion to wait for.
+__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Programmatic dependent launch: allow the next kernel in the stream to be
 // scheduled, and wait for the previous one's results.  Both are no-ops when
 // the kernel was not launched with the programmatic-serialisation attribute.

@@ -50,6 +50,10 @@ constexpr int kMaxTR = 32;                               // rows per stage
 constexpr int kStageTarget = NTX_GEMV_STAGE_BYTES;       // bytes a stage aims at
 constexpr int kGemvThreads = (kMaxConsumers + 1) * 32;
 constexpr int kEpiTable = 128;        // float2 entries of the epilogue table (RoPE: head_dim/2)
+#ifndef NTX_GEMV_PF_BYTES
+#define NTX_GEMV_PF_BYTES 0
+#endif
+constexpr int kGemvPrefetchBytes = NTX_GEMV_PF_BYTES;  // weight bytes per CTA requested into L2 ahead of the ring
 
 template <int QT>
 struct QTraits;
@@ -100,6 +104,7 @@ struct GemvPlan {
   int row_bytes;
   int stage_bytes;
   int xstage_bytes;  // shared memory holding x for the lanes (16-byte multiple)
+  int pf_stages;     // stages kept requested into L2 ahead of the ring (0: none)
 };
 
 // ------------------------------------------------------------- row maps
@@ -973,9 +978,19 @@ __global__ void __launch_bounds__((MAXC + 1) * 32, MAXC <= 8 ? 2 : 1)
         bulk_g2s(ring + (size_t)s * p.stage_bytes + (size_t)r * p.row_bytes, map.row(rs + r), (uint32_t)p.row_bytes,
                  &full[s], policy);
     };
-    // Weights do not depend on the previous kernel: start streaming them first.
+    // Weights do not depend on the previous kernel: start streaming them first,
+    // the ring's stages by bulk copy and a window of further stages into L2
+    // (so a kernel that became resident while its predecessor drains has its
+    // weights on the way before it may read x).
+    auto prefetch = [&](int i) {
+      const int64_t rs = r0 + (int64_t)i * p.TR;
+      const int nr = (int)min64(p.TR, r1 - rs);
+      for (int r = lane; r < nr; r += 32) l2_prefetch(map.row(rs + r), (uint32_t)p.row_bytes);
+    };
     const int pre = min(p.S, n_stages);
     for (int i = 0; i < pre; ++i) issue(i, i);
+    int pf_next = pre;
+    for (const int pf_end = min(n_stages, pre + p.pf_stages); pf_next < pf_end; ++pf_next) prefetch(pf_next);
     pdl_launch_dependents();
     pdl_wait();
     epi.init(esm, lane);
@@ -1000,6 +1015,7 @@ __global__ void __launch_bounds__((MAXC + 1) * 32, MAXC <= 8 ? 2 : 1)
       __syncwarp();
       // 2. refill the slot before any global-memory epilogue work
       if (i + p.S < n_stages) issue(i + p.S, s);
+      if (pf_next < n_stages) prefetch(pf_next++);
       if (++s == p.S) { s = 0; ph ^= 1u; }
       // 3. epilogue; the next stage's inputs are requested first
       epi.rotate();
@@ -1092,6 +1108,7 @@ inline GemvPlan make_gemv_plan(int qtype, int64_t K, int align, int smem_budget,
   if (S > 8) S = 8;
   if (S < 2) S = 2;
   p.S = S;
+  p.pf_stages = kGemvPrefetchBytes / p.stage_bytes;
   return p;
 }
 

@@ -103,9 +103,11 @@ cudaError_t gemv_tma_v(Map map, Pro pro, Epi epi, int64_t M, int64_t K, int grid
                        int ring) {
   static unsigned long long done = 0;  // unique per instantiation
   auto kern = gemv_tma_kernel<QT, Map, Pro, Epi, MAXC>;
-  // the ring gives up what x staging needs beyond the per-CTA ceiling
+  // the ring gives up what x staging needs beyond the per-CTA ceiling (half the
+  // SM's shared memory when two CTAs are to share an SM)
   const int xst = qt_float(QT) ? 0 : (int)((xstage_bytes(QT, K) + 15) / 16 * 16);
-  if (ring > kSmemMax - 8192 - xst) ring = kSmemMax - 8192 - xst;
+  const int cap = MAXC <= 8 ? 112 * 1024 : kSmemMax;
+  if (ring > cap - 8192 - xst) ring = cap - 8192 - xst;
   const GemvPlan plan = make_gemv_plan(QT, K, Epi::kAlign, ring, MAXC);
   const size_t smem = gemv_smem_bytes(plan);
   cudaError_t e = ensure_smem(kern, kSmemMax, done);

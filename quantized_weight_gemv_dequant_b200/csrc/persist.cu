@@ -62,6 +62,10 @@ constexpr int kPEpiWarp = kPConsumers, kPCopyWarp = kPConsumers + 1;
 constexpr int kPThreads = kPWarps * 32;
 constexpr int kPCThreads = kPConsumers * 32;
 constexpr float kAttnScale = 0.08838834764831845f;  // 1 / sqrt(128)
+#ifndef NTX_ATTN_PB
+#define NTX_ATTN_PB 4
+#endif
+constexpr int kPB = NTX_ATTN_PB;  // attention positions per warp step (loads in flight together)
 
 __device__ __forceinline__ void cons_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kPCThreads) : "memory"); }
 
@@ -287,10 +291,6 @@ __device__ __forceinline__ AttnSmem attn_smem(uint8_t* base, int G) {
   a.sw = a.ml + 2 * G;
   return a;
 }
-// Bulk prefetch into L2 (16-byte aligned address, size a multiple of 16).
-__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 
 // mbarrier operations on 32-bit shared-window addresses (keeps loop state small).
 __device__ __forceinline__ bool mbar_test_a(uint32_t a, uint32_t parity) {
@@ -404,7 +404,7 @@ struct Copier {
         break;
       }
       issue(s);
-      prefetch_one();
+      if (st.pf_stages > 0) prefetch_one();
       ++done;
       if (++s == n_slots) { s = 0; ph ^= 1u; }
     }
@@ -620,15 +620,20 @@ struct Consumer {
 
   // A GEMV phase in the block type of its kind: QA, or QB where the step's
   // plan gives that kind the second type (QB == QA: one type for all).
+  // A kernel built for two types leaves out the Q6_K paths that keep two
+  // row slices in flight: with both types' code in one kernel their registers
+  // would push the rest into local memory.
   template <int QA, int QB>
   __device__ bool gemv(int kind, const float* h, const float* w) {
     if constexpr (QA != QB) {
-      if (st.qt[kind] == QB) return gemv_t<QB>(kind, h, w);
+      if (st.qt[kind] == QB) return gemv_t<QB, false>(kind, h, w);
+      return gemv_t<QA, false>(kind, h, w);
+    } else {
+      return gemv_t<QA, true>(kind, h, w);
     }
-    return gemv_t<QA>(kind, h, w);
   }
 
-  template <int QT>
+  template <int QT, bool TWO>
   __device__ bool gemv_t(int kind, const float* h, const float* w) {
     const PGeom g = sm.kg[kind].g;
     const PRows rows = sm.kg[kind].rows;
@@ -673,7 +678,7 @@ struct Consumer {
         }
         return false;
       }
-      if constexpr (QT == QT_Q6_K) {
+      if constexpr (QT == QT_Q6_K && TWO) {
         // A Q6_K row slice is a long dependent chain, so a warp keeps two in
         // flight.  With one row per warp per slot (TR == row groups) the next
         // slot is opened too and its row runs beside this one.
@@ -736,7 +741,7 @@ struct Consumer {
         float* rd = reinterpret_cast<float*>(p_smem + o_red) + rslot * RF;
         // the row group that takes the extra rows rotates from stage to stage
         int rr = (gr + nrg - i % nrg) % nrg;
-        if constexpr (QT == QT_Q6_K) {
+        if constexpr (QT == QT_Q6_K && TWO) {
           for (; rr + nrg < nr; rr += 2 * nrg) {  // two rows of this slot side by side
             float va = 0.f, vb = 0.f;
             if (active) {
@@ -848,7 +853,10 @@ struct Consumer {
     const AttnSmem a = attn_smem(sm.xst, G);
     const int units = st.Hkv * ns;
     const int S = kAttnPartStride;
-    constexpr int GW = G < 4 ? G : 4;      // query heads per warp
+#ifndef NTX_ATTN_GW
+#define NTX_ATTN_GW 2
+#endif
+    constexpr int GW = G < NTX_ATTN_GW ? G : NTX_ATTN_GW;  // query heads per warp
     constexpr int NH = G / GW;             // head groups
     constexpr int WPG = kPConsumers / NH;  // warps per head group
     constexpr int LPH = 32 / GW;           // lanes holding one head's score after heads_reduce
@@ -876,30 +884,41 @@ struct Consumer {
       }
       if (w_on) {
         const float4* qv = reinterpret_cast<const float4*>(a.qs + hg * GW * kPD) + lane;
-        for (int p = p0 + wpos; p < p1; p += WPG) {
-          const uint2 k1 = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)p * kPD));
-          const uint2 v1 = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)p * kPD));
-          float qr[GW][4];
+        // kPB positions per step, their K and V loads issued together so that
+        // one L2 round trip serves the batch
+        for (int p = p0 + wpos; p < p1; p += kPB * WPG) {
+          uint2 kk[kPB], vv[kPB];
 #pragma unroll
-          for (int h = 0; h < GW; ++h) {
-            const float4 t = qv[h * (kPD / 4)];
-            qr[h][0] = t.x; qr[h][1] = t.y; qr[h][2] = t.z; qr[h][3] = t.w;
+          for (int b = 0; b < kPB; ++b) {
+            const int pb = min(p + b * WPG, p1 - 1);  // past the end: a repeated row, masked below
+            kk[b] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)pb * kPD));
+            vv[b] = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)pb * kPD));
           }
-          float s1[GW];
-          score_parts<GW>(reinterpret_cast<const uint8_t*>(&k1), qr, s1);
-          const float r1 = heads_reduce<GW>(s1, lane);
-          const float va[4] = {half_bits_to_float(v1.x), half_bits_to_float(v1.x >> 16), half_bits_to_float(v1.y),
-                               half_bits_to_float(v1.y >> 16)};
 #pragma unroll
-          for (int h = 0; h < GW; ++h) {
-            const float sa = __shfl_sync(0xffffffffu, r1, h * LPH);
-            const float mn = fmaxf(m[h], sa);
-            const float c = expf(m[h] - mn);  // exp(-inf) = 0 at the first position
-            const float ea = expf(sa - mn);
-            l[h] = fmaf(l[h], c, ea);
+          for (int b = 0; b < kPB; ++b) {
+            if (p + b * WPG >= p1) break;  // warp-uniform
+            float qr[GW][4];
 #pragma unroll
-            for (int d = 0; d < 4; ++d) o[h][d] = fmaf(o[h][d], c, ea * va[d]);
-            m[h] = mn;
+            for (int h = 0; h < GW; ++h) {
+              const float4 t = qv[h * (kPD / 4)];
+              qr[h][0] = t.x; qr[h][1] = t.y; qr[h][2] = t.z; qr[h][3] = t.w;
+            }
+            float s1[GW];
+            score_parts<GW>(reinterpret_cast<const uint8_t*>(&kk[b]), qr, s1);
+            const float r1 = heads_reduce<GW>(s1, lane);
+            const float va[4] = {half_bits_to_float(vv[b].x), half_bits_to_float(vv[b].x >> 16),
+                                 half_bits_to_float(vv[b].y), half_bits_to_float(vv[b].y >> 16)};
+#pragma unroll
+            for (int h = 0; h < GW; ++h) {
+              const float sa = __shfl_sync(0xffffffffu, r1, h * LPH);
+              const float mn = fmaxf(m[h], sa);
+              const float c = expf(m[h] - mn);  // exp(-inf) = 0 at the first position
+              const float ea = expf(sa - mn);
+              l[h] = fmaf(l[h], c, ea);
+#pragma unroll
+              for (int d = 0; d < 4; ++d) o[h][d] = fmaf(o[h][d], c, ea * va[d]);
+              m[h] = mn;
+            }
           }
         }
       }
