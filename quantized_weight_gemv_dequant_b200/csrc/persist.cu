@@ -62,10 +62,6 @@ constexpr int kPEpiWarp = kPConsumers, kPCopyWarp = kPConsumers + 1;
 constexpr int kPThreads = kPWarps * 32;
 constexpr int kPCThreads = kPConsumers * 32;
 constexpr float kAttnScale = 0.08838834764831845f;  // 1 / sqrt(128)
-#ifndef NTX_ATTN_PB
-#define NTX_ATTN_PB 4
-#endif
-constexpr int kPB = NTX_ATTN_PB;  // attention positions per warp step (loads in flight together)
 
 __device__ __forceinline__ void cons_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kPCThreads) : "memory"); }
 
@@ -270,27 +266,33 @@ __device__ __forceinline__ PSmem psmem_at(uint8_t* base, int S, int Z, int XB, i
 }
 
 // Attention scratch inside the x staging region (consumer warps only).
-// A warp's partial result for one head: unnormalised output o[0..127] (16-byte
-// aligned for the lanes' float4 stores), then max, sum and two pad floats.
-constexpr int kWpStride = kPD + 4;
-constexpr int kWpMax = kPD, kWpSum = kPD + 1;
 struct AttnSmem {
-  float* qs;  // [G][kPD] the unit's query heads, scaled by 1/sqrt(D)
-  float* wp;  // [kPConsumers][4][kWpStride] each warp's partial results for its <= 4 heads
-  float* ml;  // [G][2] the unit's (max, sum) per head
-  float* sw;  // [G][n_split] merge weights
+  uint8_t* k;   // [kPChunk][128] fp16: one tile of K rows
+  uint8_t* v;   // [kPChunk][128] fp16: one tile of V rows
+  float* sc;    // [G][kPChunk] scores, then exp(score - running max)
+  float* ml;    // [G][2] running (max, sum of exp) of the unit
+  float* fac;   // [G] rescale factor of the running output for this tile
+  float* sw;    // [G][n_split] merge weights
 };
 __host__ __device__ inline size_t attn_smem_bytes(int G, int ns) {
-  return (size_t)G * kPD * 4 + (size_t)kPConsumers * 4 * kWpStride * 4 + (size_t)G * 2 * 4 + (size_t)G * ns * 4;
+  return (size_t)2 * kPChunk * kPD * 2 + (size_t)G * kPChunk * 4 + (size_t)G * 3 * 4 + (size_t)G * ns * 4;
 }
 __device__ __forceinline__ AttnSmem attn_smem(uint8_t* base, int G) {
   AttnSmem a;
-  a.qs = reinterpret_cast<float*>(base);                   // base 16-byte aligned; G * 512 bytes
-  a.wp = a.qs + G * kPD;                                   // entries of 528 bytes: every o[] 16-byte aligned
-  a.ml = a.wp + kPConsumers * 4 * kWpStride;
-  a.sw = a.ml + 2 * G;
+  a.k = base;
+  a.v = base + kPChunk * kPD * 2;
+  a.sc = reinterpret_cast<float*>(a.v + kPChunk * kPD * 2);
+  a.ml = a.sc + G * kPChunk;
+  a.fac = a.ml + 2 * G;
+  a.sw = a.fac + G;
   return a;
 }
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 
 // mbarrier operations on 32-bit shared-window addresses (keeps loop state small).
 __device__ __forceinline__ bool mbar_test_a(uint32_t a, uint32_t parity) {
@@ -618,11 +620,11 @@ struct Consumer {
     }
   }
 
-  // A GEMV phase in the block type of its kind: QA, or QB where the step's
-  // plan gives that kind the second type (QB == QA: one type for all).
   // A kernel built for two types leaves out the Q6_K paths that keep two
   // row slices in flight: with both types' code in one kernel their registers
   // would push the rest into local memory.
+  // A GEMV phase in the block type of its kind: QA, or QB where the step's
+  // plan gives that kind the second type (QB == QA: one type for all).
   template <int QA, int QB>
   __device__ bool gemv(int kind, const float* h, const float* w) {
     if constexpr (QA != QB) {
@@ -831,20 +833,18 @@ struct Consumer {
   }
 
   // Split-KV attention.  This step's context is cut into ns splits per KV
-  // head (attn_splits).  Inside a unit (KV head, split) the warps work
-  // independently: the G query heads of the group are taken GW <= 4 at a time
-  // by NH = G / GW groups of WPG warps, and warp w of a head group takes the
-  // positions p0 + w, p0 + w + WPG, ... .  Each lane holds 4 dimensions of q
-  // and of the running output of each of its warp's heads; per position it
-  // reads its 4 dimensions of the K and V rows straight from L2 (the rows were
-  // prefetched at the start of the layer's Q/K/V phase; the current token's
-  // row was just written by this launch), forms the GW scores with one
-  // transposed warp reduction (heads_reduce) and a broadcast, and updates its
-  // running (max, sum, output) -- online softmax.  One
-  // CTA barrier later the warps' partial results are merged per head in a
-  // fixed order.  With one split the unit writes the head output; otherwise
-  // it writes its (max, sum, unnormalised output) and the last unit of each
-  // KV head to finish merges the splits (log-sum-exp).
+  // head (attn_splits); a unit walks its positions in tiles of kPChunk rows of
+  // K and V (contiguous in the cache, brought to shared memory with 16-byte
+  // asynchronous copies) with a running max and sum (online softmax).
+  // Scores: a warp per position and group of at most 4 query heads (two
+  // positions in flight), each lane 4 dimensions of each of those heads,
+  // reduced for all of them at once (heads_reduce).
+  // P V: thread (d8, h, pg) keeps dimensions 8 d8 .. 8 d8 + 7 of head h over
+  // the tile positions pg, pg + NPG, ...; the NPG position groups are summed
+  // in a fixed order at the end of the unit.  With one split the unit writes
+  // the head output; otherwise it writes its (max, sum, unnormalised output)
+  // and the last unit of each KV head to finish merges the splits
+  // (log-sum-exp).
   template <int G>
   __device__ void attention(const LRow& L, int lk) {
     const int n_ctx = st.params[0] + 1;
@@ -853,110 +853,131 @@ struct Consumer {
     const AttnSmem a = attn_smem(sm.xst, G);
     const int units = st.Hkv * ns;
     const int S = kAttnPartStride;
-#ifndef NTX_ATTN_GW
-#define NTX_ATTN_GW 2
-#endif
-    constexpr int GW = G < NTX_ATTN_GW ? G : NTX_ATTN_GW;  // query heads per warp
-    constexpr int NH = G / GW;             // head groups
-    constexpr int WPG = kPConsumers / NH;  // warps per head group
-    constexpr int LPH = 32 / GW;           // lanes holding one head's score after heads_reduce
-    const int hg = warp % NH, wpos = warp / NH;
-    const bool w_on = wpos < WPG;
+    constexpr int NPG = kPCThreads / (16 * G);  // P V position groups
+    constexpr int GW = G < 4 ? G : 4;           // query heads per warp in the score step
+    constexpr int NH = G / GW;                  // warps per position (head groups)
+    constexpr int WPG = kPConsumers / NH;       // warps per head group
+    constexpr int LPH = 32 / GW;                // lanes holding one head's score after heads_reduce
+    const int hh0 = (warp % NH) * GW, wpos = warp / NH;
+    const int d8 = ctid % 16, hv = (ctid / 16) % G, pg = ctid / (16 * G);
+    const bool pv_on = pg < NPG;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       const int kvh = u / ns, split = u % ns;
       const int p0 = split * chunk;
       const int p1 = min(p0 + chunk, n_ctx);
-      const uint16_t* kb = L.kc + (int64_t)kvh * st.max_ctx * kPD + 4 * lane;
-      const uint16_t* vb = L.vc + (int64_t)kvh * st.max_ctx * kPD + 4 * lane;
-      // the group's query heads, scaled, into shared memory (read per position)
-      for (int i = ctid; i < G * kPD / 4; i += kPCThreads) {
-        const float4 t = __ldcg(reinterpret_cast<const float4*>(st.q + (int64_t)kvh * G * kPD) + i);
-        reinterpret_cast<float4*>(a.qs)[i] =
-            make_float4(t.x * kAttnScale, t.y * kAttnScale, t.z * kAttnScale, t.w * kAttnScale);
+      const int np = p1 > p0 ? p1 - p0 : 0;
+      const uint8_t* kbase = reinterpret_cast<const uint8_t*>(L.kc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
+      const uint8_t* vbase = reinterpret_cast<const uint8_t*>(L.vc + ((int64_t)kvh * st.max_ctx + p0) * kPD);
+      const float* qg = st.q + (int64_t)kvh * G * kPD + 4 * lane;
+      if (ctid < G) {
+        a.ml[2 * ctid] = -INFINITY;
+        a.ml[2 * ctid + 1] = 0.f;
       }
-      cons_bar();
-      float o[GW][4], m[GW], l[GW];
+      float o[8];
 #pragma unroll
-      for (int h = 0; h < GW; ++h) {
-        o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0.f;
-        m[h] = -INFINITY;
-        l[h] = 0.f;
-      }
-      if (w_on) {
-        const float4* qv = reinterpret_cast<const float4*>(a.qs + hg * GW * kPD) + lane;
-        // kPB positions per step, their K and V loads issued together so that
-        // one L2 round trip serves the batch
-        for (int p = p0 + wpos; p < p1; p += kPB * WPG) {
-          uint2 kk[kPB], vv[kPB];
-#pragma unroll
-          for (int b = 0; b < kPB; ++b) {
-            const int pb = min(p + b * WPG, p1 - 1);  // past the end: a repeated row, masked below
-            kk[b] = __ldcg(reinterpret_cast<const uint2*>(kb + (int64_t)pb * kPD));
-            vv[b] = __ldcg(reinterpret_cast<const uint2*>(vb + (int64_t)pb * kPD));
+      for (int k = 0; k < 8; ++k) o[k] = 0.f;
+      cons_bar();  // the running (max, sum) start values are visible
+      for (int t0 = 0; t0 < np; t0 += kPChunk) {
+        const int nt = min(kPChunk, np - t0);
+        {  // K, V rows of the tile -> shared memory (nt * 256 bytes each)
+          const int n16 = nt * (kPD * 2 / 16);
+          const int off = t0 * kPD * 2;
+          for (int i = ctid; i < 2 * n16; i += kPCThreads) {
+            const bool isv = i >= n16;
+            const int ob = (isv ? i - n16 : i) * 16;
+            cp_async16((isv ? a.v : a.k) + ob, (isv ? vbase : kbase) + off + ob);
           }
-#pragma unroll
-          for (int b = 0; b < kPB; ++b) {
-            if (p + b * WPG >= p1) break;  // warp-uniform
-            float qr[GW][4];
-#pragma unroll
-            for (int h = 0; h < GW; ++h) {
-              const float4 t = qv[h * (kPD / 4)];
-              qr[h][0] = t.x; qr[h][1] = t.y; qr[h][2] = t.z; qr[h][3] = t.w;
-            }
-            float s1[GW];
-            score_parts<GW>(reinterpret_cast<const uint8_t*>(&kk[b]), qr, s1);
-            const float r1 = heads_reduce<GW>(s1, lane);
-            const float va[4] = {half_bits_to_float(vv[b].x), half_bits_to_float(vv[b].x >> 16),
-                                 half_bits_to_float(vv[b].y), half_bits_to_float(vv[b].y >> 16)};
-#pragma unroll
-            for (int h = 0; h < GW; ++h) {
-              const float sa = __shfl_sync(0xffffffffu, r1, h * LPH);
-              const float mn = fmaxf(m[h], sa);
-              const float c = expf(m[h] - mn);  // exp(-inf) = 0 at the first position
-              const float ea = expf(sa - mn);
-              l[h] = fmaf(l[h], c, ea);
-#pragma unroll
-              for (int d = 0; d < 4; ++d) o[h][d] = fmaf(o[h][d], c, ea * va[d]);
-              m[h] = mn;
-            }
-          }
+          cp_async_commit();
         }
-      }
-      // this warp's partial results -> shared memory
-      if (w_on) {
+        // this lane's 4 dimensions of every query head of the group, loaded
+        // per tile (L2) while the tile lands, so they are not held through P V
+        float qr[GW][4];
 #pragma unroll
         for (int h = 0; h < GW; ++h) {
-          float* dst = a.wp + ((size_t)warp * 4 + h) * kWpStride;
-          *reinterpret_cast<float4*>(dst + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
-          if (lane == 0) {
-            dst[kWpMax] = m[h];
-            dst[kWpSum] = l[h];
+          const float4 t = __ldcg(reinterpret_cast<const float4*>(qg + (hh0 + h) * kPD));
+          qr[h][0] = t.x; qr[h][1] = t.y; qr[h][2] = t.z; qr[h][3] = t.w;
+        }
+        cp_async_wait_all();
+        cons_bar();
+        for (int i = wpos; i < nt; i += 2 * WPG) {
+          const int i2 = i + WPG;
+          const bool two = i2 < nt;  // warp-uniform
+          float v1[GW], v2[GW];
+          score_parts<GW>(a.k + (size_t)i * kPD * 2 + 8 * lane, qr, v1);
+          if (two) score_parts<GW>(a.k + (size_t)i2 * kPD * 2 + 8 * lane, qr, v2);
+          else {
+#pragma unroll
+            for (int h = 0; h < GW; ++h) v2[h] = 0.f;
+          }
+          const float s1 = heads_reduce<GW>(v1, lane), s2 = heads_reduce<GW>(v2, lane);
+          if (lane % LPH == 0) {
+            a.sc[(hh0 + lane / LPH) * kPChunk + i] = s1 * kAttnScale;
+            if (two) a.sc[(hh0 + lane / LPH) * kPChunk + i2] = s2 * kAttnScale;
           }
         }
+        cons_bar();
+        // running max and sum per head (warp h)
+        for (int h = warp; h < G; h += kPConsumers) {
+          float mt = -INFINITY;
+          for (int i = lane; i < nt; i += 32) mt = fmaxf(mt, a.sc[h * kPChunk + i]);
+          mt = warp_max(mt);
+          const float m_old = a.ml[2 * h], m_new = fmaxf(m_old, mt);
+          float l = 0.f;
+          for (int i = lane; i < nt; i += 32) {
+            const float e = expf(a.sc[h * kPChunk + i] - m_new);
+            a.sc[h * kPChunk + i] = e;
+            l += e;
+          }
+          l = warp_sum(l);
+          if (lane == 0) {
+            const float f = m_old == -INFINITY ? 0.f : expf(m_old - m_new);
+            a.fac[h] = f;
+            a.ml[2 * h] = m_new;
+            a.ml[2 * h + 1] = fmaf(a.ml[2 * h + 1], f, l);
+          }
+        }
+        cons_bar();
+        if (pv_on) {
+          const float f = a.fac[hv];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) o[k] *= f;
+          const float* e = a.sc + hv * kPChunk;
+          for (int i = pg; i < nt; i += NPG) {
+            const uint4 w = *reinterpret_cast<const uint4*>(a.v + (size_t)i * kPD * 2 + 16 * d8);
+            const float ei = e[i];
+            o[0] = fmaf(ei, half_bits_to_float(w.x), o[0]);
+            o[1] = fmaf(ei, half_bits_to_float(w.x >> 16), o[1]);
+            o[2] = fmaf(ei, half_bits_to_float(w.y), o[2]);
+            o[3] = fmaf(ei, half_bits_to_float(w.y >> 16), o[3]);
+            o[4] = fmaf(ei, half_bits_to_float(w.z), o[4]);
+            o[5] = fmaf(ei, half_bits_to_float(w.z >> 16), o[5]);
+            o[6] = fmaf(ei, half_bits_to_float(w.w), o[6]);
+            o[7] = fmaf(ei, half_bits_to_float(w.w >> 16), o[7]);
+          }
+        }
+        cons_bar();  // the next tile overwrites K, V and the scores
+      }
+      // the position groups' partial outputs -> the K tile buffer ([NPG][G][128] floats)
+      float* pr = reinterpret_cast<float*>(a.k);
+      if (pv_on) {
+        float4* dst = reinterpret_cast<float4*>(pr + ((size_t)pg * G + hv) * kPD + 8 * d8);
+        dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_float4(o[4], o[5], o[6], o[7]);
       }
       cons_bar();
-      // merge the WPG warps of each head in a fixed order: element (h, d) per thread
       for (int idx = ctid; idx < G * kPD; idx += kPCThreads) {
         const int h = idx / kPD, d = idx % kPD;
-        const int g = h / GW, hl = h % GW;
-        float M = -INFINITY;
-        for (int w = 0; w < WPG; ++w) M = fmaxf(M, a.wp[((size_t)(w * NH + g) * 4 + hl) * kWpStride + kWpMax]);
-        float Ls = 0.f, O = 0.f;
-        for (int w = 0; w < WPG; ++w) {
-          const float* src = a.wp + ((size_t)(w * NH + g) * 4 + hl) * kWpStride;
-          const float mw = src[kWpMax];
-          const float f = mw == -INFINITY ? 0.f : expf(mw - M);
-          Ls = fmaf(src[kWpSum], f, Ls);
-          O = fmaf(src[d], f, O);
-        }
+        float sum = 0.f;
+#pragma unroll 4
+        for (int g2 = 0; g2 < NPG; ++g2) sum += pr[((size_t)g2 * G + h) * kPD + d];
         if (ns == 1) {
-          st.attn_out[(int64_t)(kvh * G + h) * kPD + d] = O / Ls;
+          st.attn_out[(int64_t)(kvh * G + h) * kPD + d] = sum / a.ml[2 * h + 1];
         } else {
           float* dst = st.attn_part + ((int64_t)(kvh * G + h) * ns + split) * S;
-          dst[2 + d] = O;
+          dst[2 + d] = sum;
           if (d == 0) {
-            dst[0] = M;
-            dst[1] = Ls;
+            dst[0] = a.ml[2 * h];
+            dst[1] = a.ml[2 * h + 1];
           }
         }
       }

@@ -8,10 +8,14 @@
 namespace ntx {
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // the persistent kernel's wait limit unless a test lowers it
+// Weight bytes per CTA requested into L2 beyond the ring (0: none).  Off by
+// default: on B200 the extra requests cost more decode throughput than the
+// L2 hits they bring (the ring alone keeps enough bytes in flight).
 #ifndef NTX_PF_BYTES
-#define NTX_PF_BYTES (192 * 1024)
+#define NTX_PF_BYTES 0
 #endif
-constexpr int kPPrefetchBytes = NTX_PF_BYTES;  // weight bytes per CTA requested into L2 beyond the ring
+constexpr int kPPrefetchBytes = NTX_PF_BYTES;
+constexpr int kPChunk = 64;          // attention positions per K/V tile
 constexpr int kPConsumers = 14;      // consumer warps per CTA (plus an epilogue warp and a copy warp)
 constexpr int kPRed = 8;             // depth of the row-partial ring between consumers and the epilogue warp
 constexpr int kPPartsPerLane = 8;    // CTAs at most: 32 * this (sum-of-squares partials read per lane)
