@@ -656,15 +656,34 @@ def run_70b(args, dist, ntx, torch, sg, wl, peak, peak_kind, dev_index):
     rc = Run(ntx, torch, m, d, L, qm, wl.Q4_K_M_HEAD, wk["max_ctx"], [0] * L)
     rc.steps([start], [p0])
     rc.steps([-1] * args.warmup, [pos_of(i) for i in range(args.warmup)])
-    ms_c, kms_c = rc.timed([pos_of(args.warmup + i) for i in range(n_a)])
+    launches_c = ntx.ntx_engine_launches_per_step(rc.eng)
+    persistent_c = launches_c <= 2
+    ms_c, kms_c = rc.timed([pos_of(args.warmup + i) for i in range(n_a)], kernel_events=persistent_c)
     c_bytes = wl.bytes_per_token(d, qm, wl.Q4_K_M_HEAD, n_ctx)
     res["5c_q4_k_m_resident"] = {
         "value": round(n_a / (ms_c / 1e3), 3), "unit": "tok/s", "steps": n_a, "ms_per_step": round(ms_c / n_a, 4),
         "weights": "Q4_K (wq wk wv wo wg wu), Q6_K (wd, head)",
-        "launches_per_step": ntx.ntx_engine_launches_per_step(rc.eng),
-        "roofline": roofline(kms_c, c_bytes, peak, peak_kind, 12, None, ms_c / n_a, "5c's timed region"),
+        "path": "persistent decode kernel" if persistent_c else
+                "per-op kernel chain (the engine's default for two block types)",
+        "launches_per_step": launches_c,
+        "roofline": roofline(kms_c, c_bytes, peak, peak_kind, 12, None, ms_c / n_a, "5c's timed region")
+                    if persistent_c else None,
         "decode_roofline": {"bytes_per_token": c_bytes, "roofline_tok_s": round(peak * 1e9 / c_bytes, 2),
-                            "frac": round((n_a / (ms_c / 1e3)) / (peak * 1e9 / c_bytes), 4)},
+                            "frac": round((n_a / (ms_c / 1e3)) / (peak * 1e9 / c_bytes), 4)}}
+    rc.close()
+    del rc
+    # the two-type persistent kernel (opt-in), for comparison
+    ntx.ntx_set_persist_two_types(1)
+    try:
+        rc = Run(ntx, torch, m, d, L, qm, wl.Q4_K_M_HEAD, wk["max_ctx"], [0] * L)
+    finally:
+        ntx.ntx_set_persist_two_types(0)
+    rc.steps([-1] * args.warmup, [pos_of(i) for i in range(args.warmup)])
+    ms_p, _ = rc.timed([pos_of(args.warmup + i) for i in range(n_a)], kernel_events=False)
+    res["5c_q4_k_m_resident"]["two_type_persistent"] = {
+        "value": round(n_a / (ms_p / 1e3), 3), "unit": "tok/s", "steps": n_a,
+        "launches_per_step": ntx.ntx_engine_launches_per_step(rc.eng),
+        "how": "ntx_set_persist_two_types(1): one persistent kernel with Q4_K and Q6_K row decoders",
         "gemv_in_step": rc.phases([pos_of(args.warmup + n_a + i) for i in range(4)], L, d, qm, wl.Q4_K_M_HEAD,
                                   peak)}
     rc.close()

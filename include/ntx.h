@@ -114,6 +114,16 @@ NTX_API int ntx_set_gemv_ctas_per_sm(int ctas_per_sm);
  * the previous one's tail.  NTX_ERR_INVALID_ARG for other values. */
 NTX_API int ntx_set_gemv_pdl(int on);
 
+/* Tuning: whether an engine whose GEMV phases use two block types (Q4_K or
+ * Q5_K matrices with Q6_K down projections and head, as in Q4_K_M / Q5_K_M
+ * models) runs its all-resident steps as the persistent decode kernel (1)
+ * or as the per-op kernel chain (0, the default).  With two row decoders in
+ * one kernel its registers overflow; on B200 a 70B-shaped Q4_K_M model
+ * decoded at 34 tok/s that way and 48 tok/s on the chain.  Applies to
+ * engines created after the call, process-wide; NTX_ERR_INVALID_ARG for
+ * other values. */
+NTX_API int ntx_set_persist_two_types(int on);
+
 /* ------------------------------------------------------------ per-op calls */
 
 /* Dequantize n weights ([README] 主な機能: GGUF Q4_0/Q8_0/Q4_K_M/Q5_K/Q6_K/F16/F32;
@@ -271,7 +281,8 @@ NTX_API int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_weight
  * The engine owns only its events, a pinned 16-byte parameter block and the
  * captured CUDA graphs; the caller keeps every buffer alive until
  * ntx_engine_destroy.
- * Execution: when every layer and the head share one block type, a step
+ * Execution: when every layer and the head share one block type (or two,
+ * after ntx_set_persist_two_types(1)), a step
  * whose executed layers are all resident (tier 0) -- every step of an engine
  * without host layers, and the NTX_USE_SKIP steps of one whose recorded skip
  * set skips every host layer -- runs as ONE persistent kernel (one CTA per

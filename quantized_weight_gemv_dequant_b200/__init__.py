@@ -41,6 +41,7 @@ EXPORTS = (
     "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
     "ntx_persistent_plan", "ntx_layer_layout_mixed", "ntx_engine_device_bytes", "ntx_auto_tier_map",
     "ntx_memory_budget", "ntx_set_host_wait_limit", "ntx_engine_set_fault", "ntx_decode_spec",
+    "ntx_set_persist_two_types",
 )
 
 
@@ -103,6 +104,7 @@ def lib():
             "ntx_decode_spec": ([vp, ctypes.c_int32, i32, i32, P(ctypes.c_int32), P(i32), i32], i32),
             "ntx_engine_destroy": ([vp], i32),
             "ntx_set_host_wait_limit": ([ctypes.c_uint64], i32),
+            "ntx_set_persist_two_types": ([i32], i32),
             "ntx_engine_set_fault": ([vp, i32, ctypes.c_uint64], i32),
             "ntx_engine_set_probe": ([vp, vp, vp, i32], i32),
             "ntx_engine_launches_per_step": ([vp], i32),
@@ -291,6 +293,10 @@ def ntx_engine_skip_mask(engine, n_layers):
 
 def ntx_engine_destroy(engine):
     _check(lib().ntx_engine_destroy(engine))
+
+
+def ntx_set_persist_two_types(on: int) -> None:
+    _check(lib().ntx_set_persist_two_types(on))
 
 
 def ntx_set_host_wait_limit(ms: int) -> None:

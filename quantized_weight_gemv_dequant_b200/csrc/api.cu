@@ -82,6 +82,10 @@ cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 // NTX_ERR_TIMEOUT (the GPU work is left running; the caller decides).
 std::atomic<uint64_t> g_host_wait_ms{60000};
 
+// Engines created while this is set run two-block-type steps on the
+// persistent kernel (ntx_set_persist_two_types).
+std::atomic<int> g_persist_two{0};
+
 // Host-side fault injection for tests: NTX_FAULT is a comma-separated list
 // of names; a call that reaches the named point fails as if the underlying
 // operation had failed, before it enqueues any work.
@@ -256,6 +260,12 @@ int ntx_gemv_q(int qtype, const void* W, int64_t M, int64_t K, const float* x, f
 int ntx_set_gemv_ctas_per_sm(int cps) {
   if (cps < 1 || cps > 4) return fail(NTX_ERR_INVALID_ARG, "ctas per SM must be 1..4");
   ntx::set_gemv_ctas_per_sm(cps);
+  return NTX_OK;
+}
+
+int ntx_set_persist_two_types(int on) {
+  if (on != 0 && on != 1) return fail(NTX_ERR_INVALID_ARG, "two-type persistent switch must be 0 or 1");
+  g_persist_two = on;
   return NTX_OK;
 }
 
@@ -818,7 +828,9 @@ extern "C" int ntx_engine_create(const ntx_model_config* cfg, const ntx_layer_we
   for (int l = 1; l < cfg->n_layers && uniform; ++l)
     uniform = mat_qt(&layers[l], 0) == kt[ntx::PK_QKV] && mat_qt(&layers[l], 3) == kt[ntx::PK_O] &&
               mat_qt(&layers[l], 4) == kt[ntx::PK_GU] && mat_qt(&layers[l], 6) == kt[ntx::PK_DOWN];
-  if (err == cudaSuccess && uniform) {
+  bool one_type = true;
+  for (int k : {ntx::PK_O, ntx::PK_GU, ntx::PK_DOWN, ntx::PK_HEAD}) one_type = one_type && kt[k] == kt[ntx::PK_QKV];
+  if (err == cudaSuccess && uniform && (one_type || g_persist_two.load())) {
     ntx::PStep st;
     memset(&st, 0, sizeof st);
     size_t psm = 0;

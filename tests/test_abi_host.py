@@ -99,6 +99,9 @@ def test_tuning_switch_argument_errors():
     assert L.ntx_set_gemv_ctas_per_sm(0) == ntx.NTX_ERR_INVALID_ARG
     assert L.ntx_set_gemv_ctas_per_sm(5) == ntx.NTX_ERR_INVALID_ARG
     assert L.ntx_set_gemv_ctas_per_sm(1) == ntx.NTX_OK
+    assert L.ntx_set_persist_two_types(2) == ntx.NTX_ERR_INVALID_ARG
+    assert L.ntx_set_persist_two_types(-1) == ntx.NTX_ERR_INVALID_ARG
+    assert L.ntx_set_persist_two_types(0) == ntx.NTX_OK
 
 
 def test_small_op_argument_errors():

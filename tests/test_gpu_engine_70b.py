@@ -93,7 +93,8 @@ def test_engine_llama70b_q6_k_resident_and_tiered_with_skip():
 
 def test_engine_llama70b_q4_k_m_resident_persistent():
     """The 70B shapes as Q4_K_M (Q4_K matrices, Q6_K down projections and head):
-    the persistent kernel with two block types (Q4_K phases over 4 K-slices,
+    the persistent kernel with two block types (opted in; the default for
+    two-type steps is the per-op chain) (Q4_K phases over 4 K-slices,
     the Q6_K down projection over 14), checked teacher-forced for 2 steps."""
     d = dict(wl.MODEL_70B)
     L = d["n_layers"]
@@ -105,7 +106,11 @@ def test_engine_llama70b_q4_k_m_resident_persistent():
             ref = sg.quant_rows(qt, sd, wl.tensor_name(l, name), M, K, sigma=wl.W_SIGMA, row0=7, nrows=1)
             assert np.array_equal(t[name][7], ref[0]), (l, name)
     prompt = [int(sg.tokens(sd, "prompt", 1, d["vocab"])[0])]
-    e = Engine(m)
+    ntx.ntx_set_persist_two_types(1)  # opt in: two-type steps default to the per-op chain
+    try:
+        e = Engine(m)
+    finally:
+        ntx.ntx_set_persist_two_types(0)
     lg, fed, nx, _ = e.run(prompt + [-1], pos0=2048)
     launches = ntx.ntx_engine_launches_per_step(e.h)
     e.close()

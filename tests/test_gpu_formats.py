@@ -221,7 +221,8 @@ def test_decode_layer_mixed_types(types):
 def test_engine_k_quant_models_persistent_and_chain(types, head):
     """4-layer K-quant models (Q4_K_M: Q4_K matrices, Q6_K down projections and
     head) through the engine, as the persistent kernel (one launch per step,
-    per-phase block types) and as the per-op chain: every step's logits within
+    per-phase block types; opted in for two-type models), as the engine's
+    default (the chain for two-type models) and as the per-op chain: every step's logits within
     2e-2 * RMS of the oracle's, teacher-forced on the GPU's tokens, greedy
     token where the gap allows."""
     from synthgen.devmodel import DeviceModel
@@ -229,13 +230,21 @@ def test_engine_k_quant_models_persistent_and_chain(types, head):
     d = dict(MIX_D, n_layers=4)
     m = DeviceModel(d, types, head, 91, max_ctx=24, n_prior=0, source="host")
     prompt = [int(t) for t in sg.tokens(91, "prompt", 3, d["vocab"])]
-    for flags in (0, ntx.NTX_NO_PERSIST):
+    two = len(set(types) | {head}) > 1
+    # persistent (two-type kernels are opt-in), the engine's default, the chain
+    for opt_in, flags in ((1, 0), (0, 0), (0, ntx.NTX_NO_PERSIST)):
+        if opt_in == 0 and flags == 0 and not two:
+            continue  # a one-type model's default is the persistent case above
         m.reset_kv()
-        e = Engine(m)
+        ntx.ntx_set_persist_two_types(opt_in)
+        try:
+            e = Engine(m)
+        finally:
+            ntx.ntx_set_persist_two_types(0)
         lg, fed, nx, _ = e.run(prompt + [-1] * 3, flags=flags)
         launches = ntx.ntx_engine_launches_per_step(e.h)
         e.close()
-        assert (launches == 1) == (flags == 0), launches
+        assert (launches == 1) == (flags == 0 and (opt_in == 1 or not two)), launches
         refs, _ = oracle_run(m, fed)
         for s in range(len(fed)):
             check_logits(lg[s], refs[s], int(nx[s]), s)
