@@ -272,10 +272,10 @@ struct AttnSmem {
   float* sc;    // [G][kPChunk] scores, then exp(score - running max)
   float* ml;    // [G][2] running (max, sum of exp) of the unit
   float* fac;   // [G] rescale factor of the running output for this tile
-  float* sw;    // [G][n_split] merge weights
+  float* sw;    // [G][n_split][2] the splits' (max, sum), then (merge weight, sum)
 };
 __host__ __device__ inline size_t attn_smem_bytes(int G, int ns) {
-  return (size_t)2 * kPChunk * kPD * 2 + (size_t)G * kPChunk * 4 + (size_t)G * 3 * 4 + (size_t)G * ns * 4;
+  return (size_t)2 * kPChunk * kPD * 2 + (size_t)G * kPChunk * 4 + (size_t)G * 3 * 4 + (size_t)G * ns * 8;
 }
 __device__ __forceinline__ AttnSmem attn_smem(uint8_t* base, int G) {
   AttnSmem a;
@@ -333,23 +333,24 @@ __device__ bool pwait_a(uint32_t bar, uint32_t parity, const volatile int* cta_a
 // It waits only for slots to be released: weights never depend on
 // activations, so the stream runs ahead across phase boundaries.
 //
-// Beyond the ring, the warp keeps a window of pf_stages further stages
-// requested into L2 (bulk prefetch, no completion to wait for): while the
-// consumers wait at a phase boundary and the ring is full, HBM keeps
-// streaming those stages into L2, and the ring refills from L2 (several times
-// the HBM rate) once the consumers resume.  Each weight byte still crosses
-// HBM once.
+// While the ring is full and the warp waits for a slot -- the consumers are at
+// a phase boundary, in the attention phase or working through a full ring --
+// it requests further stages into L2 (bulk prefetch, no completion to wait
+// for), up to pf_stages beyond the ring, so that HBM keeps streaming; those
+// stages later come into the ring from L2.  Nothing is prefetched while slots
+// turn over as fast as HBM fills them, so the prefetches never compete with
+// the ring's own copies.  Each weight byte still crosses HBM once.
 struct Copier {
   const PStep& st;
   PSmem sm;
   int lane, np, n_slots, slot_bytes;
   uint64_t policy;
   PIssue it;   // next stage into the ring
-  PIssue pit;  // next stage into L2, pf_stages ahead of it
-  long issued, done;
+  PIssue pit;  // next stage into L2 (at or ahead of it)
+  long issued, done, pfn;  // stages issued into the ring; the L2 frontier (stage count)
 
   __device__ Copier(const PStep& st_, PSmem sm_, int lane_, int np_)
-      : st(st_), sm(sm_), lane(lane_), np(np_), issued(0), done(0) {
+      : st(st_), sm(sm_), lane(lane_), np(np_), issued(0), done(0), pfn(0) {
     n_slots = st.n_slots;
     slot_bytes = st.slot_bytes;
     policy = l2_evict_first_policy();
@@ -367,14 +368,38 @@ struct Copier {
     for (int r = lane; r < nr; r += 32) bulk_g2s(dst + (size_t)r * rb, it.row(rs + r), (uint32_t)rb, bar, policy);
     it.advance(st, np);
     ++issued;
+    if (pfn < issued) {  // the L2 frontier never trails the ring
+      pit = it;
+      pfn = issued;
+    }
   }
 
   __device__ __forceinline__ void prefetch_one() {
-    if (!pit.valid(np)) return;
     const int64_t rs = pit.r0 + (int64_t)pit.j * pit.TR;
     const int nr = (int)min64(pit.TR, pit.r1 - rs);
     for (int r = lane; r < nr; r += 32) l2_prefetch(pit.row(rs + r), (uint32_t)pit.rb);
     pit.advance(st, np);
+    ++pfn;
+  }
+
+  // Waits (bounded) for slot s to be released, extending the L2 window while
+  // it is not.
+  __device__ bool wait_slot(int s, uint32_t ph) {
+    uint64_t* bar = sm.empty + s;
+    bool ok = mbar_try_wait(bar, ph);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+      if (pfn < issued + st.pf_stages && pit.valid(np)) {
+        prefetch_one();
+        if (!ok) ok = mbar_try_wait(bar, ph);
+      } else if (!ok) {
+        ok = mbar_try_wait_sleep(bar, ph);
+      }
+      if (__all_sync(0xffffffffu, ok)) return true;
+      const bool give_up = *reinterpret_cast<volatile int*>(sm.misc) || global_ns() - t0 > st.wait_ns;
+      if (__any_sync(0xffffffffu, !ok && give_up)) return false;
+    }
   }
 
   // Lets every issued copy land (bounded) before the warp exits.
@@ -393,12 +418,10 @@ struct Copier {
 
   __device__ void run() {
     for (int k = 0; k < n_slots && it.valid(np); ++k) issue(k);
-    pit = it;
-    for (int k = 0; k < st.pf_stages; ++k) prefetch_one();
     int s = 0;
     uint32_t ph = 0;
     while (it.valid(np)) {
-      if (!pwait(sm.empty + s, ph, sm.misc, st.wait_ns)) {
+      if (!wait_slot(s, ph)) {
         if (lane == 0) {
           atomicExch(sm.misc, 1);
           atomicExch(st.sync + st.abort_index, 1u);
@@ -406,7 +429,6 @@ struct Copier {
         break;
       }
       issue(s);
-      if (st.pf_stages > 0) prefetch_one();
       ++done;
       if (++s == n_slots) { s = 0; ph ^= 1u; }
     }
@@ -985,65 +1007,67 @@ struct Consumer {
         cons_bar();  // scratch reuse by the next unit
         continue;
       }
-      // publish this split (release by one thread after the CTA barrier)
+      // Publish this split, wait (bounded) until every split of this KV head
+      // has published, then merge this unit's share of the head group's
+      // outputs: elements [e0, e1) of the G x 128, each a log-sum-exp
+      // weighted sum over the splits in split order.  Every unit of a KV head
+      // runs on its own CTA (units <= grid), all resident at once.
       cons_bar();
       if (ctid == 0) {
-        const unsigned old = atom_acq_rel_add(st.sync + st.head_ctr_index + lk * st.Hkv + kvh, 1u);
-        sm.misc[3] = old == (unsigned)(ns - 1);
+        unsigned* hctr = st.sync + st.head_ctr_index + lk * st.Hkv + kvh;
+        red_release_add(hctr, 1u);
+        if (!grid_wait(hctr, (unsigned)ns, st.sync + st.abort_index, st.status, st.wait_ns)) atomicExch(sm.misc, 1);
       }
       cons_bar();
-      if (sm.misc[3]) {
-        // (m, l) of every split: one warp per query head, 4 loads per lane in flight
-        for (int h = warp; h < G; h += kPConsumers) {
-          const float* ph0 = st.attn_part + (int64_t)(kvh * G + h) * ns * S;
-          float M = -INFINITY;
-          for (int t0 = 0; t0 < ns; t0 += 32 * kPSplitsPerRound) {
-            float mv[kPSplitsPerRound];
+      const int E = G * kPD;
+      const int e0 = split * E / ns, e1 = (split + 1) * E / ns;
+      const float* pk = st.attn_part + (int64_t)kvh * G * ns * S;  // [G][ns][S]
+      // (m, l) of every split of every head -> shared memory, and the first
+      // element's values of the first kPMergeChunk splits -> registers, in
+      // one round of loads
+      for (int i = ctid; i < G * ns; i += kPCThreads) {
+        const float2 t = __ldcg(reinterpret_cast<const float2*>(pk + (int64_t)i * S));
+        a.sw[2 * i] = t.x;
+        a.sw[2 * i + 1] = t.y;
+      }
+      float v[kPMergeChunk];
+      {
+        const int e = e0 + ctid;
+        const float* pe = pk + (int64_t)(e / kPD) * ns * S + 2 + e % kPD;
 #pragma unroll
-            for (int k = 0; k < kPSplitsPerRound; ++k) {
-              const int t = t0 + lane + 32 * k;
-              mv[k] = t < ns ? __ldcg(ph0 + (int64_t)t * S) : -INFINITY;
-            }
-#pragma unroll
-            for (int k = 0; k < kPSplitsPerRound; ++k) M = fmaxf(M, mv[k]);
-          }
-          M = warp_max(M);
-          float Ls = 0.f;
-          for (int t0 = 0; t0 < ns; t0 += 32 * kPSplitsPerRound) {
-            float mv[kPSplitsPerRound], lv[kPSplitsPerRound];
-#pragma unroll
-            for (int k = 0; k < kPSplitsPerRound; ++k) {
-              const int t = t0 + lane + 32 * k;
-              mv[k] = t < ns ? __ldcg(ph0 + (int64_t)t * S) : -INFINITY;
-              lv[k] = t < ns ? __ldcg(ph0 + (int64_t)t * S + 1) : 0.f;
-            }
-#pragma unroll
-            for (int k = 0; k < kPSplitsPerRound; ++k) {
-              const int t = t0 + lane + 32 * k;
-              const float wgt = mv[k] == -INFINITY ? 0.f : expf(mv[k] - M);
-              Ls = fmaf(wgt, lv[k], Ls);
-              if (t < ns) a.sw[h * ns + t] = wgt;
-            }
-          }
-          Ls = warp_sum(Ls);
-          if (lane == 0) a.ml[2 * h + 1] = Ls;  // this unit's own (m, l) are already stored
+        for (int k = 0; k < kPMergeChunk; ++k) v[k] = (e < e1 && k < ns) ? __ldcg(pe + (int64_t)k * S) : 0.f;
+      }
+      cons_bar();
+      // per head: max over the splits, then weights exp(m_s - M) / L in place of m_s
+      for (int h = ctid; h < G; h += kPCThreads) {
+        float* mlh = a.sw + 2 * h * ns;
+        float M = -INFINITY;
+        for (int t = 0; t < ns; ++t) M = fmaxf(M, mlh[2 * t]);
+        float Ls = 0.f;
+        for (int t = 0; t < ns; ++t) {
+          const float w = mlh[2 * t] == -INFINITY ? 0.f : expf(mlh[2 * t] - M);
+          mlh[2 * t] = w;
+          Ls = fmaf(w, mlh[2 * t + 1], Ls);
         }
-        cons_bar();
-        for (int idx = ctid; idx < G * kPD; idx += kPCThreads) {
-          const int h = idx / kPD, d = idx % kPD;
-          const float* ph0 = st.attn_part + (int64_t)(kvh * G + h) * ns * S + 2 + d;
-          const float* wt = a.sw + h * ns;
-          float O = 0.f;
-          for (int t = 0; t < ns; t += 16) {
-            float v[16];
+        const float inv = 1.f / Ls;
+        for (int t = 0; t < ns; ++t) mlh[2 * t] *= inv;
+      }
+      cons_bar();
+      for (int e = e0 + ctid; e < e1; e += kPCThreads) {
+        const int h = e / kPD;
+        const float* pe = pk + (int64_t)h * ns * S + 2 + e % kPD;
+        const float* wt = a.sw + 2 * h * ns;
+        float O = 0.f;
+        for (int t = 0; t < ns; t += kPMergeChunk) {
+          if (e != e0 + ctid || t > 0) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = t + k < ns ? __ldcg(ph0 + (int64_t)(t + k) * S) : 0.f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-              if (t + k < ns) O = fmaf(wt[t + k], v[k], O);
+            for (int k = 0; k < kPMergeChunk; ++k) v[k] = t + k < ns ? __ldcg(pe + (int64_t)(t + k) * S) : 0.f;
           }
-          st.attn_out[(int64_t)(kvh * G + h) * kPD + d] = O / a.ml[2 * h + 1];
+#pragma unroll
+          for (int k = 0; k < kPMergeChunk; ++k)
+            if (t + k < ns) O = fmaf(wt[2 * (t + k)], v[k], O);
         }
+        st.attn_out[(int64_t)kvh * E + e] = O;
       }
       cons_bar();  // scratch reuse by the next unit
     }

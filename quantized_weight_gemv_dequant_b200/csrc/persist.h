@@ -21,7 +21,7 @@ constexpr int kPRed = 8;             // depth of the row-partial ring between co
 constexpr int kPPartsPerLane = 8;    // CTAs at most: 32 * this (sum-of-squares partials read per lane)
 constexpr int kPMaxTR = 32;          // rows per ring slot at most
 constexpr int kPMinSplit = 128;      // attention positions per (KV head, split) unit at least, where possible
-constexpr int kPSplitsPerRound = 4;  // split (m, l) loads per lane in flight during the merge
+constexpr int kPMergeChunk = 18;     // splits whose values a thread loads at once in the split merge
 constexpr int kPD = 128;             // head dimension
 constexpr int kAttnPartStride = kPD + 2;  // floats per (query head, split) partial: m, l, o[128]
 
