@@ -402,7 +402,11 @@ struct Copier {
     }
   }
 
-  // Lets every issued copy land (bounded) before the warp exits.
+  // Lets every issued copy land (bounded) before the warp exits.  A copy that
+  // has not landed within the wait limit means the memory system is not
+  // completing requests; the warp then records kStatusDrainTimeout and
+  // returns rather than wait without a bound, so the step is reported failed
+  // and its CTA may exit with that copy still outstanding.
   __device__ void drain() {
     if (lane == 0) {
       const uint64_t t0 = global_ns();
