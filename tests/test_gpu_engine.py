@@ -168,10 +168,13 @@ def test_engine_tiny_teacher_forced_graph_and_nograph(chain):
     (ntx.NTX_Q8_0, dict(TINY, n_heads=16, n_kv_heads=2, n_layers=2), 20000, 19990),
     (ntx.NTX_Q4_0, dict(TINY, n_heads=4, n_kv_heads=4, n_layers=2), 600, 590),
     (ntx.NTX_Q6_K, dict(TINY, hidden=2048, n_heads=16, n_kv_heads=8, ffn=6144, n_layers=2), 300, 290),
-], ids=["q8_0_g8_ctx20000", "q4_0_g1_ctx600", "q6_k_g2_ctx300"])
+    (ntx.NTX_Q8_0, dict(TINY, n_heads=8, n_kv_heads=1, n_layers=2), 20000, 19990),
+], ids=["q8_0_g8_ctx20000", "q4_0_g1_ctx600", "q6_k_g2_ctx300", "q8_0_one_kv_head_ctx20000"])
 def test_engine_persistent_long_context(qtype, d, max_ctx, n_prior):
     """Persistent kernel at contexts where a (KV head, split) unit holds many
-    positions and (first case) there are more units than CTAs."""
+    positions, and where the splits of one KV head are many: 74 per KV head
+    (first case), one per CTA for a single KV head (last case), so that each
+    split merges a few outputs over every split in several rounds of loads."""
     m = DeviceModel(d, qtype, qtype, 49, max_ctx=max_ctx, n_prior=n_prior, source="host")
     toks = list(sg.tokens(49, "prompt", 2, d["vocab"])) + [-1] * 2
     e = Engine(m)
