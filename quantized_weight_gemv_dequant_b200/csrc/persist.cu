@@ -18,8 +18,8 @@
 // Phases (index p; one grid-wide counter each):
 //   0            EMBED  h = fp16 row of the token, sum(h^2) partials
 //   1 + 5k + 0   QKV    RMSNorm(h) prologue, q/k/v rows, RoPE, KV append
-//   1 + 5k + 1   ATTN   split-KV GQA attention, the last CTA of each KV head
-//                       merges the splits (log-sum-exp)
+//   1 + 5k + 1   ATTN   split-KV GQA attention; the splits of a KV head merge
+//                       their outputs (log-sum-exp), each split a share
 //   1 + 5k + 2   O      h1 = h + Wo a, sum(h1^2) partials
 //   1 + 5k + 3   GU     RMSNorm(h1) prologue, u = silu(Wg n) * (Wu n)
 //   1 + 5k + 4   DOWN   h = h1 + Wd u, residual and cosine statistics
@@ -868,9 +868,9 @@ struct Consumer {
   // P V: thread (d8, h, pg) keeps dimensions 8 d8 .. 8 d8 + 7 of head h over
   // the tile positions pg, pg + NPG, ...; the NPG position groups are summed
   // in a fixed order at the end of the unit.  With one split the unit writes
-  // the head output; otherwise it writes its (max, sum, unnormalised output)
-  // and the last unit of each KV head to finish merges the splits
-  // (log-sum-exp).
+  // the head output; otherwise it writes its (max, sum, unnormalised output),
+  // waits for the other splits of its KV head and merges its share of the
+  // head group's outputs (log-sum-exp).
   template <int G>
   __device__ void attention(const LRow& L, int lk) {
     const int n_ctx = st.params[0] + 1;
