@@ -641,6 +641,30 @@ def run_70b(args, dist, ntx, torch, sg, wl, peak, peak_kind, dev_index):
                              "verification streams layers 40-79 once per call); host wall clock, the call "
                              "waits for its tokens",
                       "note": "random-init weights: the draft rarely agrees with the whole model"}
+    # the same after making layers 40-79 the identity (their O and down projections zeroed in the pinned
+    # blobs): the draft is then the whole model, every proposal is accepted, and one verification pass's
+    # stream of the host layers serves k + 1 tokens -- the other end of the acceptance range
+    for l in range(40, L):
+        for name in ("wo", "wd"):
+            M_, K_ = wl.mat_shapes(d)[name]
+            off = m.offsets[name]
+            m.layers[l][off:off + wl.mat_bytes(qt, M_, K_)].zero_()
+    rb.steps([start], [p0])
+    rb.cs.synchronize()
+    tok, pos, emitted_i, acc_i = start, p0 + 1, 0, []
+    t0 = time.perf_counter()
+    for _ in range(n_calls):
+        got = ntx.ntx_decode_spec(rb.eng, tok, pos, k)
+        acc_i.append(len(got) - 1)
+        emitted_i += len(got)
+        pos += len(got)
+        tok = got[-1]
+    spec_i = time.perf_counter() - t0
+    b["self_spec"]["identity_host_layers"] = {
+        "value": round(emitted_i / spec_i, 3), "unit": "tok/s", "calls": n_calls, "tokens": emitted_i,
+        "accepted_per_call": acc_i,
+        "how": "layers 40-79 made the identity (O and down projections zeroed), same engine and calls; plain "
+               "decode streams the same bytes per token as above"}
     rb.close()
     del rb
     res["5b_tiered"] = b
