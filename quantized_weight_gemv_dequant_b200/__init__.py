@@ -14,7 +14,8 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libntx.so")
+# NTX_LIB selects another build of the library (the bounds-checked one, for tests)
+LIB_PATH = os.environ.get("NTX_LIB") or os.path.join(HERE, "libntx.so")
 
 NTX_OK = 0
 NTX_ERR_INVALID_ARG = -1
@@ -41,7 +42,7 @@ EXPORTS = (
     "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
     "ntx_persistent_plan", "ntx_layer_layout_mixed", "ntx_engine_device_bytes", "ntx_auto_tier_map",
     "ntx_memory_budget", "ntx_set_host_wait_limit", "ntx_engine_set_fault", "ntx_decode_spec",
-    "ntx_set_persist_two_types",
+    "ntx_set_persist_two_types", "ntx_check_enabled", "ntx_check_report",
 )
 
 
@@ -81,6 +82,8 @@ def lib():
             "ntx_last_error": ([], ctypes.c_char_p),
             "ntx_version": ([], i32),
             "ntx_device_status": ([P(ctypes.c_int)], i32),
+            "ntx_check_enabled": ([], i32),
+            "ntx_check_report": ([P(ctypes.c_int), P(ctypes.c_longlong)], i32),
             "ntx_sm_count": ([], i32),
             "ntx_set_gemv_ctas_per_sm": ([i32], i32),
             "ntx_set_gemv_pdl": ([i32], i32),
@@ -164,6 +167,17 @@ def ntx_device_status() -> int:
     code = ctypes.c_int(0)
     _check(lib().ntx_device_status(ctypes.byref(code)))
     return code.value
+
+
+def ntx_check_enabled() -> int:
+    return lib().ntx_check_enabled()
+
+
+def ntx_check_report() -> tuple:
+    """(site, index) of the first failed bounds check of the debug build; (0, 0) if none."""
+    site, index = ctypes.c_int(0), ctypes.c_longlong(0)
+    _check(lib().ntx_check_report(ctypes.byref(site), ctypes.byref(index)))
+    return site.value, index.value
 
 
 def ntx_sm_count() -> int:

@@ -9,6 +9,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libntx.so")
+CHECK_SO = os.path.join(HERE, "libntx_check.so")  # the bounds-checked debug build (NTX_CHECK)
 SOURCES = ["kernels.cu", "api.cu", "noalloc.cu", "persist.cu", "tiers.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -46,6 +47,14 @@ def build(force: bool = False, verbose: bool = False, out: str = SO, defines=())
     return out
 
 
+def build_check(force: bool = False) -> str:
+    """The bounds-checked debug build (kernels check their buffer indices, see ntx_check_report)."""
+    return build(force=force, out=CHECK_SO, defines=("NTX_CHECK",))
+
+
 if __name__ == "__main__":
     import sys
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    if "--check" in sys.argv:
+        print(build_check(force="--force" in sys.argv))
+    else:
+        print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

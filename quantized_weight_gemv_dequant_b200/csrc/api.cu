@@ -231,6 +231,21 @@ int ntx_device_status(int* code) {
 
 int ntx_sm_count(void) { return ntx::sm_count(); }
 
+int ntx_check_enabled(void) {
+#ifdef NTX_CHECK
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int ntx_check_report(int* site, long long* index) {
+  if (!site || !index) return fail(NTX_ERR_INVALID_ARG, "site or index is NULL");
+  const int e = ntx::read_check_report(site, index);
+  if (e) return cuda_fail((cudaError_t)e, "ntx_check_report");
+  return NTX_OK;
+}
+
 int ntx_dequant(int qtype, const void* blocks, float* out, int64_t n, void* stream) {
   if (!qtype_ok(qtype)) return fail(NTX_ERR_QTYPE, "unsupported weight type %d", qtype);
   if (n < 0 || n % block_elems(qtype)) return fail(NTX_ERR_SHAPE, "n=%lld not a multiple of %d", (long long)n,

@@ -26,6 +26,41 @@ enum : int {
   kStatusGridTimeout = 4,  // a grid-wide barrier of the persistent decode kernel ran out
 };
 
+// Bounds checks of a debug build (compiled with NTX_CHECK): chk() is true
+// when i lies in [0, n); otherwise it records the first failing site and
+// index after the status word (status[1], status[2..3]) and returns false, and
+// the caller skips the access.  It never traps.  In the release build it is
+// always true and compiles to nothing.  Sites:
+enum : int {
+  kChkRingRead = 1,      // persistent kernel: a consumer's row inside its weight slot
+  kChkPartialWrite = 2,  // persistent kernel: a row partial inside its partial slot
+  kChkPartialRead = 3,   // persistent kernel: the epilogue's read of a row partial
+  kChkKvAppend = 4,      // persistent kernel: the KV cache position this step appends
+  kChkKvTile = 5,        // persistent kernel: attention K/V tile copy (positions, tile bytes)
+  kChkAttnOut = 6,       // persistent kernel: attention output and split-partial stores
+  kChkXStage = 7,        // persistent kernel: x staging stores
+  kChkSlotWrite = 8,     // persistent kernel: the copy warp's rows inside a slot
+  kChkGemvRing = 9,      // per-op GEMV: a consumer's row inside its stage
+  kChkGemvPartial = 10,  // per-op GEMV: row partials
+};
+#ifdef NTX_CHECK
+constexpr bool kCheck = true;
+#else
+constexpr bool kCheck = false;
+#endif
+__device__ __forceinline__ bool chk(int* status, int site, int64_t i, int64_t n) {
+  if constexpr (!kCheck) {
+    return true;
+  } else {
+    if (i >= 0 && i < n) return true;
+    if (status && atomicCAS(status + 1, 0, site) == 0) {
+      atomicExch(status + 2, (int)(uint32_t)(uint64_t)i);
+      atomicExch(status + 3, (int)(uint32_t)((uint64_t)i >> 32));
+    }
+    return false;
+  }
+}
+
 // Limit on any single wait (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

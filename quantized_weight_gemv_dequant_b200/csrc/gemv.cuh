@@ -1066,9 +1066,11 @@ __global__ void __launch_bounds__((MAXC + 1) * 32, MAXC <= 8 ? 2 : 1)
       const uint8_t* st = ring + (size_t)s * p.stage_bytes + (size_t)c * QTraits<QT>::SEG;
       float* rd = red + (size_t)s * p.TR * p.n_slices;
       for (int r = g; r < nr; r += p.n_rg) {
-        float v = active ? xr.dot(st + (size_t)r * p.row_bytes, lane) : 0.f;
+        const bool in = chk(status, kChkGemvRing, (int64_t)(r + 1) * p.row_bytes - 1, p.stage_bytes);
+        float v = active && in ? xr.dot(st + (size_t)r * p.row_bytes, lane) : 0.f;
         v = warp_sum(v);
-        if (lane == 0) rd[r * p.n_slices + c] = v;
+        if (lane == 0 && chk(status, kChkGemvPartial, r * p.n_slices + c, (int64_t)p.TR * p.n_slices))
+          rd[r * p.n_slices + c] = v;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);

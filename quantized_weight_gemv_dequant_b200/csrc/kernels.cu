@@ -11,7 +11,9 @@
 
 namespace ntx {
 
-__device__ int g_status = 0;
+// [0] the device status word; [1..3] the bounds-check record of a build with
+// NTX_CHECK defined (site, index low and high words), 0 otherwise.
+__device__ int g_status[4] = {0, 0, 0, 0};
 
 namespace {
 
@@ -425,6 +427,20 @@ int read_device_status(int* code) {
   e2 = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
   if (e2 != cudaSuccess) return (int)e2;
   *code = v;
+  return 0;
+}
+
+int read_check_report(int* site, long long* index) {
+  const cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return (int)e;
+  int v[4] = {0, 0, 0, 0};
+  cudaError_t e2 = cudaMemcpyFromSymbol(v, g_status, sizeof v);
+  if (e2 != cudaSuccess) return (int)e2;
+  const int zero[3] = {0, 0, 0};
+  e2 = cudaMemcpyToSymbol(g_status, zero, sizeof zero, sizeof(int));
+  if (e2 != cudaSuccess) return (int)e2;
+  *site = v[1];
+  *index = (long long)(((unsigned long long)(unsigned)v[3] << 32) | (unsigned)v[2]);
   return 0;
 }
 

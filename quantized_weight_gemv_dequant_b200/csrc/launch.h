@@ -76,6 +76,7 @@ cudaError_t launch_cos_finalize(const float* stats, int nparts, const int* layer
                                 float* cos_out, cudaStream_t s, bool pdl);
 
 int read_device_status(int* code);
+int read_check_report(int* site, long long* index);
 int* device_status_ptr();
 
 // Record a failure for ntx_last_error() on the calling thread; returns code.

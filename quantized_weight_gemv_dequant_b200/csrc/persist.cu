@@ -362,10 +362,13 @@ struct Copier {
     const int nr = (int)min64(it.TR, it.r1 - rs);
     const int rb = it.rb;
     uint64_t* bar = sm.full + slot;
-    if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(nr * rb));
+    // (debug build) rows past the slot are not copied; the slot still completes
+    const bool in = chk(st.status, kChkSlotWrite, (int64_t)nr * rb - 1, slot_bytes);
+    if (lane == 0) mbar_arrive_expect_tx(bar, in ? (uint32_t)(nr * rb) : 0u);
     __syncwarp();
     uint8_t* dst = sm.ring + (size_t)slot * slot_bytes;
-    for (int r = lane; r < nr; r += 32) bulk_g2s(dst + (size_t)r * rb, it.row(rs + r), (uint32_t)rb, bar, policy);
+    if (in)
+      for (int r = lane; r < nr; r += 32) bulk_g2s(dst + (size_t)r * rb, it.row(rs + r), (uint32_t)rb, bar, policy);
     it.advance(st, np);
     ++issued;
     if (pfn < issued) {  // the L2 frontier never trails the ring
@@ -526,7 +529,7 @@ struct Epilogue {
       const float* rd = sm.red + (size_t)slot * red_floats;
       float a = 0.f, b = 0.f;
       const bool mine = row_a < nr;
-      if (mine) {
+      if (mine && chk(st.status, kChkPartialRead, (row_a + A) * nsl - 1, red_floats)) {
         for (int c = 0; c < nsl; ++c) {
           a += rd[row_a * nsl + c];
           if (A == 2) b += rd[(row_a + 1) * nsl + c];
@@ -556,7 +559,7 @@ struct Epilogue {
       const float* rd = sm.red + (size_t)slot * red_floats;
       float a = 0.f;
       const bool mine = lane < nr;
-      if (mine)
+      if (mine && chk(st.status, kChkPartialRead, (lane + 1) * nsl - 1, red_floats))
         for (int c = 0; c < nsl; ++c) a += rd[lane * nsl + c];
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.rempty + slot);
@@ -675,6 +678,14 @@ struct Consumer {
     const bool active = busy && lane_active<QT>(lane, ucols);
     XRegs<QT> xr;
     const XStage xs = xstage_at(sm.xst, K);
+    // (debug build) the plan's staging region must hold this phase's x
+    if (g.staged && !chk(st.status, kChkXStage, (int64_t)xstage_bytes(QT, K) - 1, st.xstage_bytes)) {
+      if (ctid == 0) {
+        atomicExch(sm.misc, 1);
+        atomicExch(st.sync + st.abort_index, 1u);
+      }
+      return false;
+    }
     if (g.staged) {
       if (w) stage<QT, true>(h, w, K, xs);
       else stage<QT, false>(h, w, K, xs);
@@ -729,7 +740,10 @@ struct Consumer {
             const int rsa = r0 + i * TR;
             const int nra = min(TR, r1 - rsa), nrb = min(TR, r1 - rsa - TR);
             const int ra = (gr + nrg - i % nrg) % nrg, rb = (gr + nrg - (i + 1) % nrg) % nrg;
-            const bool ha = ra < nra, hb = rb < nrb;
+            const bool ha = ra < nra && chk(st.status, kChkRingRead, (int64_t)(ra + 1) * rbytes - 1, Z) &&
+                            chk(st.status, kChkPartialWrite, ra * nsl + c, RF);
+            const bool hb = rb < nrb && chk(st.status, kChkRingRead, (int64_t)(rb + 1) * rbytes - 1, Z) &&
+                            chk(st.status, kChkPartialWrite, rb * nsl + c, RF);
             const uint8_t* sta = p_smem + ring_c + (uint32_t)s * Z + (uint32_t)ra * (uint32_t)rbytes;
             const uint8_t* stb = p_smem + ring_c + (uint32_t)s2 * Z + (uint32_t)rb * (uint32_t)rbytes;
             float va = 0.f, vb = 0.f;
@@ -772,22 +786,25 @@ struct Consumer {
         if constexpr (QT == QT_Q6_K && TWO) {
           for (; rr + nrg < nr; rr += 2 * nrg) {  // two rows of this slot side by side
             float va = 0.f, vb = 0.f;
-            if (active) {
+            const bool in = chk(st.status, kChkRingRead, (int64_t)(rr + nrg + 1) * rbytes - 1, Z) &&
+                            chk(st.status, kChkPartialWrite, (rr + nrg) * nsl + c, RF);
+            if (active && in) {
               va = xr.dot(stg + (uint32_t)rr * (uint32_t)rbytes, lane);
               vb = xr.dot(stg + (uint32_t)(rr + nrg) * (uint32_t)rbytes, lane);
             }
             va = warp_sum(va);
             vb = warp_sum(vb);
-            if (lane == 0) {
+            if (lane == 0 && in) {
               rd[rr * nsl + c] = va;
               rd[(rr + nrg) * nsl + c] = vb;
             }
           }
         }
         for (; rr < nr; rr += nrg) {
-          float v = active ? xr.dot(stg + (uint32_t)rr * (uint32_t)rbytes, lane) : 0.f;
+          const bool in = chk(st.status, kChkRingRead, (int64_t)(rr + 1) * rbytes - 1, Z);
+          float v = active && in ? xr.dot(stg + (uint32_t)rr * (uint32_t)rbytes, lane) : 0.f;
           v = warp_sum(v);
-          if (lane == 0) rd[rr * nsl + c] = v;
+          if (lane == 0 && chk(st.status, kChkPartialWrite, rr * nsl + c, RF)) rd[rr * nsl + c] = v;
         }
       }
       __syncwarp();
@@ -908,7 +925,10 @@ struct Consumer {
         {  // K, V rows of the tile -> shared memory (nt * 256 bytes each)
           const int n16 = nt * (kPD * 2 / 16);
           const int off = t0 * kPD * 2;
-          for (int i = ctid; i < 2 * n16; i += kPCThreads) {
+          // (debug build) positions past the cache or a tile past its buffer are not copied
+          const bool in = chk(st.status, kChkKvTile, p0 + t0 + nt - 1, st.max_ctx) &&
+                          chk(st.status, kChkKvTile, (int64_t)nt * kPD * 2 - 1, (int64_t)kPChunk * kPD * 2);
+          for (int i = ctid; in && i < 2 * n16; i += kPCThreads) {
             const bool isv = i >= n16;
             const int ob = (isv ? i - n16 : i) * 16;
             cp_async16((isv ? a.v : a.k) + ob, (isv ? vbase : kbase) + off + ob);
@@ -997,13 +1017,17 @@ struct Consumer {
 #pragma unroll 4
         for (int g2 = 0; g2 < NPG; ++g2) sum += pr[((size_t)g2 * G + h) * kPD + d];
         if (ns == 1) {
-          st.attn_out[(int64_t)(kvh * G + h) * kPD + d] = sum / a.ml[2 * h + 1];
+          const int64_t oi = (int64_t)(kvh * G + h) * kPD + d;
+          if (chk(st.status, kChkAttnOut, oi, (int64_t)st.Hq * kPD)) st.attn_out[oi] = sum / a.ml[2 * h + 1];
         } else {
-          float* dst = st.attn_part + ((int64_t)(kvh * G + h) * ns + split) * S;
-          dst[2 + d] = sum;
-          if (d == 0) {
-            dst[0] = a.ml[2 * h];
-            dst[1] = a.ml[2 * h + 1];
+          const int64_t pi = ((int64_t)(kvh * G + h) * ns + split) * S;
+          if (chk(st.status, kChkAttnOut, pi + S - 1, (int64_t)st.Hq * st.n_split * S)) {
+            float* dst = st.attn_part + pi;
+            dst[2 + d] = sum;
+            if (d == 0) {
+              dst[0] = a.ml[2 * h];
+              dst[1] = a.ml[2 * h + 1];
+            }
           }
         }
       }
@@ -1071,7 +1095,8 @@ struct Consumer {
           for (int k = 0; k < kPMergeChunk; ++k)
             if (t + k < ns) O = fmaf(wt[2 * (t + k)], v[k], O);
         }
-        st.attn_out[(int64_t)kvh * E + e] = O;
+        if (chk(st.status, kChkAttnOut, (int64_t)kvh * E + e, (int64_t)st.Hq * kPD))
+          st.attn_out[(int64_t)kvh * E + e] = O;
       }
       cons_bar();  // scratch reuse by the next unit
     }
@@ -1162,6 +1187,8 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
                                                                     : sm.lt[(p - 2) / 5].stats_down;
       switch (kind) {
         case PK_QKV: {
+          // (debug build) a position outside the cache stops the step instead of appending
+          if (!chk(st.status, kChkKvAppend, st.params[0], st.max_ctx)) { ok = false; break; }
           EpiQKV epi{st.q, L->kc, L->vc, nullptr, st.params[0], (int64_t)st.Hq * st.D, (int64_t)st.Hkv * st.D,
                      st.D, st.max_ctx, st.theta, sm.rope};
           ok = ep.run(epi, rows, g, ep.rms_scale(parts));

@@ -102,6 +102,9 @@ def test_tuning_switch_argument_errors():
     assert L.ntx_set_persist_two_types(2) == ntx.NTX_ERR_INVALID_ARG
     assert L.ntx_set_persist_two_types(-1) == ntx.NTX_ERR_INVALID_ARG
     assert L.ntx_set_persist_two_types(0) == ntx.NTX_OK
+    # the release build reports no bounds checks; the report call checks its arguments first
+    assert L.ntx_check_enabled() == 0
+    assert L.ntx_check_report(None, None) == ntx.NTX_ERR_INVALID_ARG
 
 
 def test_small_op_argument_errors():
