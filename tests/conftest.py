@@ -47,3 +47,26 @@ def _built_cpu_libs():
     oracle.build()
     synthgen.build()
     yield
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """When the session ran against the bounds-checked build (NTX_LIB naming
+    libntx_check.so), every index check of every kernel the tests launched
+    must have passed: a recorded failure fails the session."""
+    ntx = sys.modules.get("quantized_weight_gemv_dequant_b200")
+    if ntx is None or getattr(ntx, "_lib", None) is None:
+        return
+    try:
+        import torch
+        if not torch.cuda.is_available() or ntx.ntx_check_enabled() != 1:
+            return
+        site, index = ntx.ntx_check_report()
+    except Exception as e:  # pragma: no cover
+        print(f"\nbounds-check report unavailable: {e}")
+        session.exitstatus = 1
+        return
+    if site != 0:
+        print(f"\nbounds check failed: site {site}, index {index}")
+        session.exitstatus = 1
+    else:
+        print("\nbounds-checked build: every index check passed")
