@@ -101,12 +101,13 @@ NTX_API int ntx_device_status(int* code);
  * decode kernel and the per-op GEMV check the indices of their shared-memory
  * weight slots and row partials, the copy warp's slot writes, the KV append
  * position, the attention tile copies and output stores, and the x staging
- * region against their buffers; an index outside records the first failing
+ * region against their buffers, and the per-op attention and Q/K/V epilogue
+ * check the step's cache position; an index outside records the first failing
  * site and index and the access is skipped (never trapped), so the results
  * are wrong but no memory outside a buffer is touched.  Sites: 1 slot read,
  * 2 partial write, 3 partial read, 4 KV append, 5 K/V tile, 6 attention
  * output, 7 x staging, 8 slot write, 9 per-op GEMV stage read, 10 per-op GEMV
- * partial.  ntx_check_enabled: 1 in that build, 0 in the release build.
+ * partial, 11 per-op attention context, 12 per-op KV append.  ntx_check_enabled: 1 in that build, 0 in the release build.
  * ntx_check_report: waits for the device, then returns and clears the
  * record (site 0: every check passed, or the release build). */
 NTX_API int ntx_check_enabled(void);

@@ -25,7 +25,8 @@ __host__ __device__ inline int attn_part_stride() { return kAttnD + 2; }
 template <int G>
 __global__ void __launch_bounds__(kAttnWarps * 32)
     attn_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc,
-                      float* __restrict__ part, int n_ctx_host, const int* pos_dev, int max_ctx, int n_split) {
+                      float* __restrict__ part, int n_ctx_host, const int* pos_dev, int max_ctx, int n_split,
+                      int* status) {
   __shared__ float s_sc[G][kAttnMaxChunk];
   __shared__ float s_o[kAttnWarps][G][kAttnD];
   __shared__ float s_ml[G][2];
@@ -34,7 +35,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32)
 
   pdl_launch_dependents();
   pdl_wait();
-  const int n_ctx = pos_dev ? *pos_dev + 1 : n_ctx_host;
+  int n_ctx = pos_dev ? *pos_dev + 1 : n_ctx_host;
+  if (!chk(status, kChkAttnCtx, n_ctx - 1, max_ctx)) n_ctx = 0;  // (debug build) read nothing past the cache
   const int chunk = (n_ctx + n_split - 1) / n_split;
   const int p0 = split * chunk;
   const int p1 = min(p0 + chunk, n_ctx);
@@ -154,7 +156,7 @@ template <int G>
 __global__ void __launch_bounds__(kAttnWarps * 32)
     attn_cluster_kernel(const float* __restrict__ q, const uint16_t* __restrict__ kc,
                         const uint16_t* __restrict__ vc, float* __restrict__ out, int n_ctx_host, const int* pos_dev,
-                        int max_ctx) {
+                        int max_ctx, int* status) {
   namespace cg = cooperative_groups;
   __shared__ float s_sc[G][kAttnMaxChunk];
   __shared__ float s_o[kAttnWarps][G][kAttnD];
@@ -167,7 +169,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32)
 
   pdl_launch_dependents();
   pdl_wait();
-  const int n_ctx = pos_dev ? *pos_dev + 1 : n_ctx_host;
+  int n_ctx = pos_dev ? *pos_dev + 1 : n_ctx_host;
+  if (!chk(status, kChkAttnCtx, n_ctx - 1, max_ctx)) n_ctx = 0;  // (debug build) read nothing past the cache
   const int chunk = (n_ctx + CS - 1) / CS;
   const int p0 = rank * chunk;
   const int p1 = min(p0 + chunk, n_ctx);

@@ -42,6 +42,8 @@ enum : int {
   kChkSlotWrite = 8,     // persistent kernel: the copy warp's rows inside a slot
   kChkGemvRing = 9,      // per-op GEMV: a consumer's row inside its stage
   kChkGemvPartial = 10,  // per-op GEMV: row partials
+  kChkAttnCtx = 11,      // per-op attention: the step's context inside the cache
+  kChkKvAppendOp = 12,   // per-op Q/K/V epilogue: the KV cache position it appends
 };
 #ifdef NTX_CHECK
 constexpr bool kCheck = true;

@@ -789,6 +789,7 @@ struct EpiQKV {
   int head_dim, max_ctx;
   float theta;
   const float2* cs;  // shared: (cos, sin) of pair i
+  int* status = nullptr;  // bounds-check record (debug build)
   static constexpr int kAlign = 2;
   __device__ __forceinline__ void init(float2* esm, int lane) {
     if (pos_dev) pos = *pos_dev;
@@ -817,6 +818,7 @@ struct EpiQKV {
       const bool is_k = r < nq + nkv;
       const int64_t kr = is_k ? r - nq : r - nq - nkv;
       const int64_t head = kr / head_dim;
+      if (!chk(status, kChkKvAppendOp, pos, max_ctx)) return;  // (debug build) no append past the cache
       uint16_t* cache = is_k ? k_cache : v_cache;
       const uint32_t packed = (uint32_t)float_to_half_bits(a) | ((uint32_t)float_to_half_bits(b) << 16);
       *reinterpret_cast<uint32_t*>(cache + (head * max_ctx + pos) * head_dim + i2) = packed;

@@ -245,10 +245,10 @@ cudaError_t launch_attn(const float* q, const uint16_t* kc, const uint16_t* vc, 
   const dim3 block(kAttnWarps * 32);
   cudaError_t e;
   switch (G) {
-    case 1: e = launch_k(attn_split_kernel<1>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split); break;
-    case 2: e = launch_k(attn_split_kernel<2>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split); break;
-    case 4: e = launch_k(attn_split_kernel<4>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split); break;
-    case 8: e = launch_k(attn_split_kernel<8>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split); break;
+    case 1: e = launch_k(attn_split_kernel<1>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split, status_ptr()); break;
+    case 2: e = launch_k(attn_split_kernel<2>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split, status_ptr()); break;
+    case 4: e = launch_k(attn_split_kernel<4>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split, status_ptr()); break;
+    case 8: e = launch_k(attn_split_kernel<8>, grid, block, 0, s, pdl, q, kc, vc, part, n_ctx, pos_dev, max_ctx, n_split, status_ptr()); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
@@ -284,7 +284,7 @@ static cudaError_t attn_cluster_g(const float* q, const uint16_t* kc, const uint
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, q, kc, vc, out, n_ctx, pos_dev, max_ctx);
+  return cudaLaunchKernelEx(&cfg, kern, q, kc, vc, out, n_ctx, pos_dev, max_ctx, status_ptr());
 }
 
 int attn_cluster_size(int Hq, int Hkv, int n_ctx_max) {
@@ -339,6 +339,7 @@ cudaError_t launch_layer(const LayerArgs& a, cudaStream_t s, bool pdl) {
     constexpr int QT = decltype(t)::value;
     ProRms pro{a.hidden, a.attn_norm, a.stats_in, a.n_stats_in, (int)a.H, a.eps, 0.f};
     EpiQKV epi{a.q, a.k_cache, a.v_cache, a.pos_dev, a.pos, nq, nkv, (int)a.D, a.max_ctx, a.theta};
+    epi.status = status_ptr();
     const int64_t M = nq + 2 * nkv;
     return gemv_tma<QT>(MapQKV{a.wq, a.wk, a.wv, row_bytes_of<QT>(a.H), nq, nkv}, pro, epi, M, a.H,
                         gemv_grid(M, 2), s, pdl);

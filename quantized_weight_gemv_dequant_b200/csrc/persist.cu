@@ -1191,6 +1191,7 @@ __global__ void __launch_bounds__(kPThreads, 1) persist_kernel(const __grid_cons
           if (!chk(st.status, kChkKvAppend, st.params[0], st.max_ctx)) { ok = false; break; }
           EpiQKV epi{st.q, L->kc, L->vc, nullptr, st.params[0], (int64_t)st.Hq * st.D, (int64_t)st.Hkv * st.D,
                      st.D, st.max_ctx, st.theta, sm.rope};
+          epi.status = st.status;
           ok = ep.run(epi, rows, g, ep.rms_scale(parts));
           break;
         }
