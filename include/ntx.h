@@ -273,9 +273,11 @@ NTX_API size_t ntx_layer_workspace_bytes(const ntx_model_config* cfg);
  *   k_cache, v_cache: device fp16 bits [Hkv][max_ctx][D] of this layer.
  *   cos_out: device float or NULL; receives cos(h_in, h_out).
  *   workspace: device scratch >= ntx_layer_workspace_bytes(cfg), 256-B aligned.
- * Limits: head_dim 128; query group in {1, 2, 4, 8}; H, F and Hq*D
- * multiples of 256 (Q8_0, Q4_0) or 2048 (Q6_K); 0 <= pos < max_ctx; weight
- * offsets 16-B aligned.  hidden, base and the caches 16-B aligned. */
+ * Limits: head_dim 128; query group in {1, 2, 4, 8}; each matrix's input
+ * length (H, F or Hq*D) a multiple of 2048 for Q6_K and of 256 for every
+ * other type; wq, wk, wv of one type and wg, wu of one type (NTX_MIXED);
+ * 0 <= pos < max_ctx; weight offsets 16-B aligned.  hidden, base and the
+ * caches 16-B aligned, workspace 256-B aligned. */
 NTX_API int ntx_decode_layer(const ntx_model_config* cfg, const ntx_layer_weights* w, uint16_t* k_cache, uint16_t* v_cache,
                      float* hidden, int pos, float* cos_out, void* workspace, size_t ws_bytes, void* stream);
 
