@@ -395,7 +395,12 @@ def run_ntx(args, dist: Dist):
     torch.cuda.init()
     dev_index = torch.cuda.current_device()
     m = DeviceModel(d, qt, hqt, sd, wk["max_ctx"], wk["n_prior"], source="device")
-    r = Run(ntx, torch, m, d, L, qt, hqt, wk["max_ctx"], [0] * L)
+    if args.persist_two:
+        ntx.ntx_set_persist_two_types(1)  # read when the engine is created
+    try:
+        r = Run(ntx, torch, m, d, L, qt, hqt, wk["max_ctx"], [0] * L)
+    finally:
+        ntx.ntx_set_persist_two_types(0)
     prompt = sg.tokens(sd, "prompt", wk["prompt"], d["vocab"])
     p_first = wk["n_prior"] + wk["prompt"]
     span = wk["max_ctx"] - p_first
@@ -490,7 +495,7 @@ def run_ntx(args, dist: Dist):
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; random-init weights of the named shapes)",
         "config": {"workload": desc, "weights": qname(qt), "layers": L, "hidden": d["hidden"], "ffn": d["ffn"],
-                   "vocab": d["vocab"], "batch": 1,
+                   "vocab": d["vocab"], "batch": 1, "persist_two_types": bool(args.persist_two),
                    "parallelism": f"replicas x{dist.world}" if dist.world > 1 else "single GPU",
                    "l2": "weights per step >> 126 MB L2 (inputs larger than L2; no flush)",
                    "graph": ("kernel-by-kernel steps: parameter copy, sync-word reset, one persistent kernel "
@@ -969,6 +974,9 @@ def main():
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling and tests only: run the headline model with this many layers (the line then "
                          "describes that smaller model and is not a benchmark of the named workload)")
+    ap.add_argument("--persist-two", action="store_true",
+                    help="run a two-block-type model (llama70b-q4_k_m) on the two-type persistent kernel "
+                         "(ntx_set_persist_two_types(1)) instead of the per-op chain that is the default for it")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture (reported as is)")
     args = ap.parse_args()
