@@ -116,6 +116,17 @@ NTX_API int ntx_check_report(int* site, long long* index);
 /* Number of SMs the kernels size their grids for on the current device. */
 NTX_API int ntx_sm_count(void);
 
+/* Measurement helper, not a step of the decode: reads the device buffer buf
+ * (bytes long) once with streaming loads and writes the sum of its 32-bit
+ * words modulo 2^32 to the device word *sum (zeroed by the call first), so
+ * the read cannot be dropped and its result can be checked.  Timed over a
+ * buffer much larger than L2 it gives the read-only HBM bandwidth, the
+ * streaming ceiling of a weight-bound decode (the pages put decode time at
+ * weight bytes over memory bandwidth: "RTX 3090 1枚でLlama 70B...", VRAMの壁).
+ * buf must be 16-byte aligned and bytes a multiple of 16 (NTX_ERR_ALIGN);
+ * buf may be NULL only when bytes is 0.  Asynchronous on stream. */
+NTX_API int ntx_hbm_read_probe(const void* buf, uint64_t bytes, uint32_t* sum, void* stream);
+
 /* Tuning: persistent GEMV CTAs per SM (1..4, default 1) for launches made
  * after the call, process-wide.  Workspace sizes do not depend on it. */
 NTX_API int ntx_set_gemv_ctas_per_sm(int ctas_per_sm);

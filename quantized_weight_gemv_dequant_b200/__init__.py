@@ -42,7 +42,7 @@ EXPORTS = (
     "ntx_engine_launches_per_step", "ntx_attn_decode_static", "ntx_engine_set_phase_probe",
     "ntx_persistent_plan", "ntx_layer_layout_mixed", "ntx_engine_device_bytes", "ntx_auto_tier_map",
     "ntx_memory_budget", "ntx_set_host_wait_limit", "ntx_engine_set_fault", "ntx_decode_spec",
-    "ntx_set_persist_two_types", "ntx_check_enabled", "ntx_check_report",
+    "ntx_set_persist_two_types", "ntx_check_enabled", "ntx_check_report", "ntx_hbm_read_probe",
 )
 
 
@@ -85,6 +85,7 @@ def lib():
             "ntx_check_enabled": ([], i32),
             "ntx_check_report": ([P(ctypes.c_int), P(ctypes.c_longlong)], i32),
             "ntx_sm_count": ([], i32),
+            "ntx_hbm_read_probe": ([vp, ctypes.c_uint64, vp, vp], i32),
             "ntx_set_gemv_ctas_per_sm": ([i32], i32),
             "ntx_set_gemv_pdl": ([i32], i32),
             "ntx_dequant": ([i32, vp, vp, i64, vp], i32),
@@ -182,6 +183,11 @@ def ntx_check_report() -> tuple:
 
 def ntx_sm_count() -> int:
     return lib().ntx_sm_count()
+
+
+def ntx_hbm_read_probe(buf, nbytes, sum_out, stream=None):
+    """Read buf (device, nbytes) once; *sum_out (device uint32) = sum of its 32-bit words mod 2^32."""
+    _check(lib().ntx_hbm_read_probe(_p(buf), nbytes, _p(sum_out), _s(stream)))
 
 
 def ntx_set_gemv_ctas_per_sm(cps: int) -> None:

@@ -342,6 +342,14 @@ int ntx_swiglu(const float* gate, const float* up, float* out, int64_t n, void* 
   return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_swiglu");
 }
 
+int ntx_hbm_read_probe(const void* buf, uint64_t bytes, uint32_t* sum, void* stream) {
+  if (!sum || (!buf && bytes)) return fail(NTX_ERR_INVALID_ARG, "NULL pointer");
+  if (bytes % 16 || reinterpret_cast<uintptr_t>(buf) % 16)
+    return fail(NTX_ERR_ALIGN, "buffer must be 16-byte aligned and a multiple of 16 bytes long");
+  const cudaError_t e = ntx::launch_read_probe(buf, bytes, sum, S(stream));
+  return e == cudaSuccess ? NTX_OK : cuda_fail(e, "ntx_hbm_read_probe");
+}
+
 uint64_t ntx_layer_layout_mixed(const ntx_model_config* cfg, const int32_t* qtypes, ntx_layer_weights* out) {
   if (!cfg || !out || !qtypes || cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 || cfg->n_kv_heads <= 0 ||
       cfg->head_dim <= 0)

@@ -238,6 +238,38 @@ cudaError_t launch_swiglu(const float* g, const float* u, float* out, int64_t n,
   return cudaGetLastError();
 }
 
+// Read-only HBM stream (a measurement helper, not a step of the decode): each
+// thread loads its 16-byte words with streaming (evict-first) loads, four in
+// flight, and the sum of all 32-bit words modulo 2^32 goes to *sum, so no load
+// can be dropped and the sum shows that every byte was read.
+__global__ void __launch_bounds__(256) read_probe_kernel(const uint4* __restrict__ p, uint64_t n16, unsigned* sum) {
+  constexpr int U = 4;
+  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+  uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  unsigned acc = 0;
+  for (; i + (U - 1) * stride < n16; i += U * stride) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) v[u] = __ldcs(p + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc += v[u].x + v[u].y + v[u].z + v[u].w;
+  }
+  for (; i < n16; i += stride) {
+    const uint4 v = __ldcs(p + i);
+    acc += v.x + v.y + v.z + v.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) atomicAdd(sum, acc);
+}
+
+cudaError_t launch_read_probe(const void* buf, uint64_t bytes, unsigned* sum, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(sum, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess || bytes == 0) return e;
+  read_probe_kernel<<<sm_count() * 8, 256, 0, s>>>(static_cast<const uint4*>(buf), bytes / 16, sum);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn(const float* q, const uint16_t* kc, const uint16_t* vc, float* out, float* part, int Hq,
                         int Hkv, int n_ctx, const int* pos_dev, int max_ctx, int n_split, cudaStream_t s, bool pdl) {
   const int G = Hq / Hkv;

@@ -25,6 +25,7 @@ cudaError_t launch_gemv(int qtype, const void* W, int64_t M, int64_t K, const fl
 cudaError_t launch_rmsnorm(const float* x, const float* w, float* y, int64_t n, float eps, cudaStream_t s);
 cudaError_t launch_rope(float* q, float* k, int nq, int nkv, int head_dim, int pos, float theta, cudaStream_t s);
 cudaError_t launch_swiglu(const float* g, const float* u, float* out, int64_t n, cudaStream_t s);
+cudaError_t launch_read_probe(const void* buf, uint64_t bytes, unsigned* sum, cudaStream_t s);
 cudaError_t launch_attn(const float* q, const uint16_t* kc, const uint16_t* vc, float* out, float* part, int Hq,
                         int Hkv, int n_ctx, const int* pos_dev, int max_ctx, int n_split, cudaStream_t s, bool pdl);
 

@@ -116,6 +116,11 @@ def test_small_op_argument_errors():
     assert _rc(ntx.ntx_rope, FAKE, None, 4, 2, 128, 0, 5e5) == ntx.NTX_ERR_INVALID_ARG
     assert _rc(ntx.ntx_rope, FAKE, FAKE, 4, 2, 128, -1, 5e5) == ntx.NTX_ERR_INVALID_ARG
     assert _rc(ntx.ntx_swiglu, FAKE, FAKE, FAKE, -1) == ntx.NTX_ERR_SHAPE
+    # the HBM read probe checks pointers and alignment before any CUDA call
+    assert _rc(ntx.ntx_hbm_read_probe, FAKE, 1 << 20, None) == ntx.NTX_ERR_INVALID_ARG
+    assert _rc(ntx.ntx_hbm_read_probe, None, 1 << 20, FAKE) == ntx.NTX_ERR_INVALID_ARG
+    assert _rc(ntx.ntx_hbm_read_probe, FAKE + 4, 1 << 20, FAKE + 0x1000) == ntx.NTX_ERR_ALIGN
+    assert _rc(ntx.ntx_hbm_read_probe, FAKE, (1 << 20) + 8, FAKE + 0x1000) == ntx.NTX_ERR_ALIGN
     # attention
     args = [FAKE, FAKE + 0x10000, FAKE + 0x20000, FAKE + 0x30000]
     assert _rc(ntx.ntx_attn_decode, *args, 32, 8, 64, 10, 100, FAKE + 0x40000, 1 << 30) == ntx.NTX_ERR_SHAPE

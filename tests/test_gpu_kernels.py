@@ -247,6 +247,22 @@ def test_swiglu():
     assert ok, e
 
 
+@pytest.mark.parametrize("nbytes", [0, 16, 16 * 7, (1 << 20) + 48, (64 << 20) + 16 * 1001])
+def test_hbm_read_probe_reads_every_word(nbytes):
+    """The read probe bench.py times for the read-only HBM peak: its sum of
+    32-bit words modulo 2^32 equals the host's, so every word was read once."""
+    import torch
+    rs = np.random.RandomState(nbytes % 1000 + 7)
+    words = rs.randint(0, 1 << 32, size=nbytes // 4, dtype=np.uint64).astype(np.uint32)
+    buf = torch.from_numpy(words.view(np.int32)).cuda() if nbytes else torch.empty(4, dtype=torch.int32).cuda()
+    out = torch.full((4,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    ntx.ntx_hbm_read_probe(buf.data_ptr(), nbytes, out[1:].data_ptr())
+    _sync()
+    got = out.cpu().numpy().view(np.uint32)
+    assert int(got[1]) == int(words.astype(np.uint64).sum() % (1 << 32))
+    assert got[0] == 0x5A5A5A5A and got[2] == 0x5A5A5A5A and got[3] == 0x5A5A5A5A
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(32, 8), (64, 8), (8, 8), (16, 8), (4, 2)])
 @pytest.mark.parametrize("n_ctx", [1, 2, 17, 300, 1025])
 def test_attention(Hq, Hkv, n_ctx):
