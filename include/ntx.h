@@ -146,8 +146,9 @@ NTX_API int ntx_set_gemv_pdl(int on);
  * Q5_K matrices with Q6_K down projections and head, as in Q4_K_M / Q5_K_M
  * models) runs its all-resident steps as the persistent decode kernel (1)
  * or as the per-op kernel chain (0, the default).  With two row decoders in
- * one kernel its registers overflow; on B200 a 70B-shaped Q4_K_M model
- * decoded at 34 tok/s that way and 48 tok/s on the chain.  Applies to
+ * one kernel its registers overflow and the spills are reloaded inside the
+ * row loops; on B200 a 70B-shaped Q4_K_M model decoded at 33 tok/s that way
+ * and 49 tok/s on the chain.  Applies to
  * engines created after the call, process-wide; NTX_ERR_INVALID_ARG for
  * other values. */
 NTX_API int ntx_set_persist_two_types(int on);
