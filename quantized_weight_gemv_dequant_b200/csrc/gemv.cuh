@@ -542,11 +542,12 @@ struct XStage {
   int np;
 };
 
-// Q6_K keeps one correction triple per 16-column run (K / 16 of them), the
-// other formats one per 32-column block (used by Q4_0).
+// Q6_K keeps one correction triple per 16-column run (K / 16 of them), Q4_0
+// and the K-quants one per 32-column block; Q8_0 codes carry no offset, so it
+// keeps none (the persistent kernel's plan gives the space to its weight ring).
 __host__ __device__ inline size_t xstage_bytes(int qtype, int64_t K) {
   const int64_t nslices = (K + kSliceCols - 1) / kSliceCols;
-  const int64_t ncorr = qtype == QT_Q6_K ? K / 16 : K / 32;
+  const int64_t ncorr = qtype == QT_Q6_K ? K / 16 : qtype == QT_Q8_0 ? 0 : K / 32;
   return (size_t)3 * 16 * (32 * nslices + 2) * 4 + (size_t)(K / 32) * 4 + (size_t)ncorr * 12;
 }
 

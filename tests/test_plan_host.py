@@ -70,8 +70,8 @@ def test_plan_invariants(name, d, qt, max_ctx):
 def test_plan_of_the_bench_models():
     """The plans the measured numbers were taken with."""
     p8 = ntx.ntx_persistent_plan(_cfg(wl.MODEL_8B, 144), ntx.NTX_Q8_0)
-    assert (p8["slot_bytes"], p8["n_slots"]) == (34816, 5)
-    assert [p8["rows"][k] for k in PHASES] == [8, 8, 8, 2, 8]
+    assert (p8["slot_bytes"], p8["n_slots"]) == (60928, 3)
+    assert [p8["rows"][k] for k in PHASES] == [14, 14, 14, 4, 14]  # two rows for every row-group warp
     p70 = ntx.ntx_persistent_plan(_cfg(wl.MODEL_70B, 2080), ntx.NTX_Q6_K)
     assert (p70["slot_bytes"], p70["n_slots"]) == (40320, 4)
     assert [p70["rows"][k] for k in PHASES] == [6, 6, 6, 1, 6]
