@@ -50,11 +50,11 @@ METRIC = "batch-1 decode tok/s; quantized GEMV achieved HBM GB/s vs B200 peak"
 # DRAM bytes read + written per algorithmic byte by the persistent decode
 # kernel, from one ncu capture (--set full) per instantiation of a cut-down
 # case that fits the capture size rule: Q8_0, 4 layers of the 8B shapes,
-# 1,485,805,312 + 4,185,088 bytes against 1,485,578,240 algorithmic bytes;
+# 1,485,863,680 + 4,421,632 bytes against 1,485,578,240 algorithmic bytes;
 # Q6_K, 2 layers of the 70B shapes, 2,283,495,936 + 4,485,632 bytes against
 # 2,282,659,840.  The kernel streams every weight byte once, so a full
 # launch's traffic is this ratio times its algorithmic bytes.
-PERSIST_TRAFFIC_RATIO = {8: (1485805312 + 4185088) / 1485578240, 14: (2283495936 + 4485632) / 2282659840}
+PERSIST_TRAFFIC_RATIO = {8: (1485863680 + 4421632) / 1485578240, 14: (2283495936 + 4485632) / 2282659840}
 FALLBACK_HBM_GBS = 6650.0
 
 
